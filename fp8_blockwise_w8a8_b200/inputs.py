@@ -1,0 +1,128 @@
+"""Seeded synthetic inputs for the blockwise FP8 W8A8 linear layer.
+
+This module is shared by the tests, the benchmark and the oracle-side checks.  It draws random
+numbers and rounds them to bf16 -- nothing else: it holds none of the quantization or GEMM
+arithmetic, and it imports neither the CUDA binding nor the oracle.
+
+bf16 tensors are returned as numpy ``uint16`` bit patterns (host) or torch ``bfloat16`` tensors
+(device generator).  Recipes (per-tensor seed = 1000 * workload_seed + tensor_id):
+
+* tiny linear      A [64, 512] ~ N(0,1), 1% of entries x20; W [256, 512] ~ N(0, 0.02); seed 0
+* decode linear    A [128, 4096] ~ N(0,1), 20 (0.5%) channels x30; W [12288, 4096] ~ N(0,0.02);
+                   seed 1
+* prefill linear   X [8192, 4096] ~ N(0,1); gamma ~ U(0.5, 1.5); eps 1e-6;
+                   W [24576, 4096] ~ N(0, 0.02); seed 2
+* requant sweep    36 layers of {q 4096x4096, k/v 1024x4096, o 4096x4096, gate/up 12288x4096,
+                   down 4096x12288} ~ N(0, 0.02), drawn per matrix with torch's generator on the
+                   chosen device; seed 3
+* MoE              4096 tokens, hidden 2048, 128 experts, top-8 distinct experts per token with
+                   p_i proportional to rank^-1.1 over a seeded permutation of expert ids
+                   (Gumbel-top-k); rows sorted by expert; gate/up input = the token rows
+                   gathered in routed order; down input ~ N(0,1) [routed, 768];
+                   W_gateup [128, 1536, 2048], W_down [128, 2048, 768] ~ N(0, 0.02); seed 4
+"""
+import numpy as np
+import torch
+
+
+def to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """fp32 array -> bf16 bit patterns (uint16), round-to-nearest-even via torch on the CPU."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_bits_to_f32(a: np.ndarray) -> np.ndarray:
+    return (np.ascontiguousarray(a, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def rng_for(seed: int, tensor_id: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(1000 * seed + tensor_id))
+
+
+def randn_bf16(shape, std: float, seed: int, tensor_id: int) -> np.ndarray:
+    r = rng_for(seed, tensor_id)
+    return to_bf16_bits(r.standard_normal(shape, dtype=np.float32) * np.float32(std))
+
+
+# --- workloads ---------------------------------------------------------------------------------
+
+def tiny_linear():
+    seed = 0
+    r = rng_for(seed, 0)
+    a = r.standard_normal((64, 512), dtype=np.float32)
+    mask = r.random((64, 512)) < 0.01
+    a = np.where(mask, a * np.float32(20.0), a)
+    return {"A": to_bf16_bits(a), "W": randn_bf16((256, 512), 0.02, seed, 1)}
+
+
+def decode_linear(M: int = 128, N: int = 12288, K: int = 4096):
+    seed = 1
+    r = rng_for(seed, 0)
+    a = r.standard_normal((M, K), dtype=np.float32)
+    n_out = int(round(0.005 * K))
+    ch = r.choice(K, size=n_out, replace=False)
+    a[:, ch] *= np.float32(30.0)
+    return {"A": to_bf16_bits(a), "W": randn_bf16((N, K), 0.02, seed, 1), "outlier_channels": ch}
+
+
+def prefill_linear(M: int = 8192, N: int = 24576, K: int = 4096, with_weight: bool = True):
+    seed = 2
+    x = randn_bf16((M, K), 1.0, seed, 0)
+    r = rng_for(seed, 1)
+    gamma = to_bf16_bits(r.uniform(0.5, 1.5, size=K).astype(np.float32))
+    out = {"X": x, "gamma": gamma, "eps": 1e-6}
+    if with_weight:
+        out["W"] = randn_bf16((N, K), 0.02, seed, 2)
+    return out
+
+
+SWEEP_LAYERS = 36
+SWEEP_MATRICES = (("q", 4096, 4096), ("k", 1024, 4096), ("v", 1024, 4096), ("o", 4096, 4096),
+                  ("gate", 12288, 4096), ("up", 12288, 4096), ("down", 4096, 12288))
+
+
+def sweep_matrix(layer: int, index: int, device="cpu") -> torch.Tensor:
+    """One weight of the 36-layer requant sweep as a bf16 torch tensor on ``device``."""
+    seed = 3
+    name, n, k = SWEEP_MATRICES[index]
+    g = torch.Generator(device=device)
+    g.manual_seed(1000 * seed + layer * len(SWEEP_MATRICES) + index)
+    w = torch.randn((n, k), generator=g, device=device, dtype=torch.float32) * 0.02
+    return w.to(torch.bfloat16)
+
+
+def sweep_elements() -> int:
+    return SWEEP_LAYERS * sum(n * k for _, n, k in SWEEP_MATRICES)
+
+
+def moe_routing(tokens: int = 4096, experts: int = 128, topk: int = 8, alpha: float = 1.1,
+                seed: int = 4):
+    """Zipf-skewed top-k routing.  Returns (token index per routed row sorted by expert,
+    group offsets int32 [experts + 1])."""
+    r = rng_for(seed, 0)
+    perm = r.permutation(experts)                   # expert id -> popularity rank
+    rank = np.empty(experts, dtype=np.int64)
+    rank[perm] = np.arange(experts)
+    logp = -alpha * np.log(rank + 1.0)
+    gumbel = -np.log(-np.log(r.random((tokens, experts))))
+    choice = np.argsort(-(logp[None, :] + gumbel), axis=1)[:, :topk]  # distinct per token
+    tok = np.repeat(np.arange(tokens), topk)
+    exp = choice.reshape(-1)
+    order = np.lexsort((tok, exp))                  # by expert, then token
+    counts = np.bincount(exp, minlength=experts)
+    off = np.zeros(experts + 1, dtype=np.int32)
+    off[1:] = np.cumsum(counts)
+    return tok[order].astype(np.int64), off
+
+
+def moe(tokens: int = 4096, hidden: int = 2048, experts: int = 128, topk: int = 8,
+        ffn: int = 768, with_weights: bool = True):
+    seed = 4
+    tok, off = moe_routing(tokens, experts, topk, 1.1, seed)
+    x = randn_bf16((tokens, hidden), 1.0, seed, 1)
+    out = {"tok": tok, "offsets": off, "X": x, "A_gateup": x[tok],
+           "A_down": randn_bf16((tok.size, ffn), 1.0, seed, 2)}
+    if with_weights:
+        out["W_gateup"] = randn_bf16((experts, 2 * ffn, hidden), 0.02, seed, 3)
+        out["W_down"] = randn_bf16((experts, hidden, ffn), 0.02, seed, 4)
+    return out

@@ -1,0 +1,233 @@
+"""CPU oracle for the blockwise FP8 (E4M3) W8A8 linear layer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this package.  The CUDA library and its Python binding never do, and this package never imports
+them: the two share no code.  Arrays are numpy: bf16 tensors travel as ``uint16`` bit patterns,
+E4M3 codes and E8M0 scale bytes as ``uint8``.
+
+The arithmetic lives in ``fp8q_oracle.c`` (plain C, fp64 for the GEMM reference); this module is
+argument marshalling.  See the C file's header for the definitions and readings it follows.
+
+Parity status: every function here is pinned by ``tests/test_oracle_*.py`` against library
+decoders/encoders, closed forms, brute force and invariants; none is "parity unpinned".
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        L.oracle_e4m3_decode.restype = ctypes.c_double
+        L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        L.oracle_e8m0_lossless_from_f32.restype = ctypes.c_int
+        L.oracle_e8m0_lossless_from_f32.argtypes = [ctypes.c_float]
+        L.oracle_e8m0_decode.restype = ctypes.c_double
+        L.oracle_e8m0_decode.argtypes = [ctypes.c_uint8]
+        L.oracle_quant_weight_block.restype = None
+        L.oracle_quant_weight_block.argtypes = [P, I64, I64, I64, P, I64, P, ctypes.c_int]
+        L.oracle_quant_token_1x128.restype = None
+        L.oracle_quant_token_1x128.argtypes = [P, I64, I64, I64, P, I64, P, I64]
+        L.oracle_rmsnorm_bf16.restype = None
+        L.oracle_rmsnorm_bf16.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64]
+        L.oracle_rmsnorm_quant_token.restype = None
+        L.oracle_rmsnorm_quant_token.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64,
+                                                 P, I64]
+        L.oracle_gemm_w8a8_block_rows.restype = None
+        L.oracle_gemm_w8a8_block_rows.argtypes = [P, I64, P, I64, P, I64, P, ctypes.c_int,
+                                                  I64, I64, P, I64, P, P]
+        L.oracle_grouped_gemm_w8a8_block_rows.restype = None
+        L.oracle_grouped_gemm_w8a8_block_rows.argtypes = [P, I64, P, I64, P, I64, P,
+                                                          ctypes.c_int, P, I64, I64, I64, P,
+                                                          I64, P, P]
+        L.oracle_e4m3_encode_array.restype = None
+        L.oracle_e4m3_encode_array.argtypes = [P, I64, P]
+        L.oracle_f32_to_bf16_array.restype = None
+        L.oracle_f32_to_bf16_array.argtypes = [P, I64, P]
+        L.oracle_rms_inverse.restype = ctypes.c_float
+        L.oracle_rms_inverse.argtypes = [P, I64, ctypes.c_float]
+        L.oracle_e4m3_encode_exhaustive_check.restype = I64
+        L.oracle_e4m3_encode_exhaustive_check.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+        L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_num_threads.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {a.dtype}")
+    return a
+
+
+SCALE_F32 = 0
+SCALE_E8M0 = 1
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()
+
+
+# --- codec ------------------------------------------------------------------------------------
+
+def e4m3_decode(code: int) -> float:
+    return lib().oracle_e4m3_decode(int(code))
+
+
+def e4m3_decode_all() -> np.ndarray:
+    """Value of each of the 256 codes (fp64; NaN for 0x7F and 0xFF)."""
+    return np.array([e4m3_decode(c) for c in range(256)], dtype=np.float64)
+
+
+def e4m3_encode(values) -> np.ndarray:
+    v = np.ascontiguousarray(np.asarray(values, dtype=np.float32).ravel())
+    out = np.empty(v.shape, dtype=np.uint8)
+    lib().oracle_e4m3_encode_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def f32_to_bf16(values) -> np.ndarray:
+    v = np.ascontiguousarray(np.asarray(values, dtype=np.float32).ravel())
+    out = np.empty(v.shape, dtype=np.uint16)
+    lib().oracle_f32_to_bf16_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def e8m0_lossless_from_f32(s: float):
+    r = lib().oracle_e8m0_lossless_from_f32(float(s))
+    return None if r < 0 else r
+
+
+def e8m0_decode(byte: int) -> float:
+    return lib().oracle_e8m0_decode(int(byte))
+
+
+def e4m3_encode_exhaustive_check():
+    first = ctypes.c_uint32(0)
+    bad = lib().oracle_e4m3_encode_exhaustive_check(ctypes.byref(first))
+    return bad, first.value
+
+
+# --- hot-path operations ----------------------------------------------------------------------
+
+def quant_weight_block(w_bf16: np.ndarray, fmt: int = SCALE_F32):
+    """W bf16 [N, K] (uint16 bits) -> (codes uint8 [N, K], scales [N/128, K/128])."""
+    w = _c(w_bf16, np.uint16)
+    N, K = w.shape
+    if N % 128 or K % 128:
+        raise ValueError("N and K must be multiples of 128")
+    q = np.empty((N, K), dtype=np.uint8)
+    sw = np.empty((N // 128, K // 128), dtype=np.float32 if fmt == SCALE_F32 else np.uint8)
+    lib().oracle_quant_weight_block(_ptr(w), N, K, K, _ptr(q), K, _ptr(sw), int(fmt))
+    return q, sw
+
+
+def quant_token_1x128(x_bf16: np.ndarray, lds: int = None):
+    """X bf16 [M, K] -> (codes [M, K], sa fp32 [K/128, lds]) with sa[kb, m] the scale."""
+    x = _c(x_bf16, np.uint16)
+    M, K = x.shape
+    lds = M if lds is None else lds
+    q = np.empty((M, K), dtype=np.uint8)
+    sa = np.zeros((K // 128, lds), dtype=np.float32)
+    lib().oracle_quant_token_1x128(_ptr(x), M, K, K, _ptr(q), K, _ptr(sa), lds)
+    return q, sa
+
+
+def rmsnorm_bf16(x_bf16: np.ndarray, gamma_bf16: np.ndarray, eps: float = 1e-6):
+    x = _c(x_bf16, np.uint16)
+    g = _c(gamma_bf16, np.uint16)
+    M, K = x.shape
+    y = np.empty((M, K), dtype=np.uint16)
+    lib().oracle_rmsnorm_bf16(_ptr(x), _ptr(g), float(eps), M, K, K, _ptr(y), K)
+    return y
+
+
+def rmsnorm_quant_token(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6,
+                        lds: int = None):
+    """Fused RMSNorm + 1x128 token quant (gamma None: plain token quant)."""
+    x = _c(x_bf16, np.uint16)
+    M, K = x.shape
+    lds = M if lds is None else lds
+    q = np.empty((M, K), dtype=np.uint8)
+    sa = np.zeros((K // 128, lds), dtype=np.float32)
+    if gamma_bf16 is None:
+        gp = None
+    else:
+        g = _c(gamma_bf16, np.uint16)
+        gp = _ptr(g)
+    lib().oracle_rmsnorm_quant_token(_ptr(x), gp, float(eps), M, K, K, _ptr(q), K, _ptr(sa),
+                                     lds)
+    return q, sa
+
+
+def rms_inverse(x_row_bf16: np.ndarray, eps: float = 1e-6) -> float:
+    x = _c(x_row_bf16, np.uint16)
+    return lib().oracle_rms_inverse(_ptr(x), x.size, float(eps))
+
+
+def gemm_w8a8_block(aq, sa, wq, sw, sw_fmt: int = SCALE_F32, rows=None):
+    """fp64 reference (ref, absref), each [len(rows), N]; rows default to all of M."""
+    aq = _c(aq, np.uint8)
+    wq = _c(wq, np.uint8)
+    sa = _c(sa, np.float32)
+    sw = _c(sw, np.float32 if sw_fmt == SCALE_F32 else np.uint8)
+    M, K = aq.shape
+    N = wq.shape[0]
+    rows = np.arange(M, dtype=np.int64) if rows is None else _c(np.asarray(rows, np.int64),
+                                                                 np.int64)
+    ref = np.empty((rows.size, N), dtype=np.float64)
+    absref = np.empty((rows.size, N), dtype=np.float64)
+    lib().oracle_gemm_w8a8_block_rows(_ptr(aq), K, _ptr(sa), sa.shape[1], _ptr(wq), K, _ptr(sw),
+                                      int(sw_fmt), N, K, _ptr(rows), rows.size, _ptr(ref),
+                                      _ptr(absref))
+    return ref, absref
+
+
+def grouped_gemm_w8a8_block(aq, sa, wq, sw, group_offsets, sw_fmt: int = SCALE_F32, rows=None):
+    """Grouped reference: wq [E, N, K], sw [E, N/128, K/128], group_offsets int32 [E+1]."""
+    aq = _c(aq, np.uint8)
+    wq = _c(wq, np.uint8)
+    sa = _c(sa, np.float32)
+    sw = _c(sw, np.float32 if sw_fmt == SCALE_F32 else np.uint8)
+    off = _c(np.asarray(group_offsets, np.int32), np.int32)
+    M, K = aq.shape
+    E, N, _ = wq.shape
+    rows = np.arange(M, dtype=np.int64) if rows is None else _c(np.asarray(rows, np.int64),
+                                                                 np.int64)
+    ref = np.empty((rows.size, N), dtype=np.float64)
+    absref = np.empty((rows.size, N), dtype=np.float64)
+    lib().oracle_grouped_gemm_w8a8_block_rows(_ptr(aq), K, _ptr(sa), sa.shape[1], _ptr(wq), K,
+                                              _ptr(sw), int(sw_fmt), _ptr(off), E, N, K,
+                                              _ptr(rows), rows.size, _ptr(ref), _ptr(absref))
+    return ref, absref
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """One bf16 ulp at |x| (2^(floor(log2|x|) - 7)); 2^-133 at zero and in the subnormal range."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    ulp = np.ldexp(1.0, (e - 7).astype(np.int64))
+    return np.where(a >= 2.0 ** -126, ulp, 2.0 ** -133)
+
+
+def gemm_tolerance(ref: np.ndarray, absref: np.ndarray) -> np.ndarray:
+    """Per-element bound |out - ref| <= 8e-3 * absref + one bf16 ulp of |ref|."""
+    return 8e-3 * absref + bf16_ulp(ref)

@@ -1,0 +1,447 @@
+/*
+ * fp8q_oracle.c -- plain, slow CPU oracle for the blockwise FP8 (E4M3) W8A8 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call this file:
+ * only the test-suite, the smoke check and the benchmark's CPU-baseline leg use it.  It shares
+ * no code, header, table or constant generator with the CUDA library; it is written from the
+ * definitions the source pages give (or, where they are silent, from the stated readings).
+ *
+ * Sources (by page title and section):
+ *   [FP8-RL]      "FP8-RL: A Practical and Stable Low-Precision Stack for LLM Reinforcement
+ *                 Learning", abstract, item (i): W8A8 linear layers with blockwise FP8
+ *                 quantization; policy weights change every step, so they are requantized
+ *                 every step.
+ *   [DSv4-WOA]    "DeepSeek V4 performance: FP8 WO_A output projection (vLLM PR 54894
+ *                 analysis)", section 1 (E8M0 scale normalisation: unsigned exponent, bias
+ *                 127, lossless only for exact powers of two), section 2 (128-divisibility
+ *                 check; scale grid viewed as [groups, out/128, in/128]), section 3 (group-128
+ *                 activation quant feeding a batched FP8 GEMM with per-group weights).
+ *   [SGL-RMSQ]    "SGLang AMD GPU optimisation: fusing RMSNorm with FP8 per-token quantization
+ *                 (SGLang PR 21403 analysis)", section 1 (RMSNorm with weight and epsilon fused
+ *                 with FP8 quant), section 3 (the GEMM takes a pre-quantized (codes, scale)
+ *                 tuple).
+ *   [OCP-FP8]     the OCP 8-bit floating point formats linked from [DSv4-WOA]'s references
+ *                 (OCP Microscaling spec v1.0, element type E4M3): sign, 4 exponent bits with
+ *                 bias 7, 3 mantissa bits, no infinities, S.1111.111 is NaN, max 448.
+ *   [torch-RMS]   torch.nn.RMSNorm documentation linked from [SGL-RMSQ]:
+ *                 y = x / sqrt(mean(x^2) + eps) * weight.
+ *
+ * Readings taken where the pages are silent (each is repeated in the design notes):
+ *   R1  scale s = amax / 448 in fp32 (IEEE round-to-nearest division); an all-zero block takes
+ *       s = 1.  Codes are q = RNEsat(x / s), fp32 IEEE division then round-to-nearest-even to
+ *       E4M3 with saturation to +-448.
+ *   R2  E8M0 scales: s = 2^e with e the smallest integer such that 2^e >= fp32(amax / 448),
+ *       clamped to [-127, 127]; byte = e + 127; all-zero block -> byte 127.
+ *   R3  the sign of zero is kept: a negative value that rounds to zero gives code 0x80.
+ *   R4  RMSNorm: per 128-block fp64 sum of squares in ascending k, then the fp64 sum of the
+ *       block sums in ascending block order; v = S / K + eps (eps widened from fp32);
+ *       r = fp32(1 / sqrt(v)) (fp64 sqrt and division, one final rounding to fp32);
+ *       y_k = bf16_RNE( fp32( fp32(x_k * r) * gamma_k ) ), which is what an unfused bf16
+ *       RMSNorm writes; then the 1x128 token quant runs on y.
+ *   R5  activation scales sa are fp32, stored K-block-major: sa[kb * lds + m].
+ *   R6  GEMM reference: out[m,n] = sum_kb (sa[m,kb] * sw[nb,kb]) * P_kb[m,n], P_kb the exact
+ *       dot product of the decoded codes over K-block kb; all in fp64.
+ *
+ * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math -fopenmp.
+ * fp32 arithmetic below relies on FLT_EVAL_METHOD == 0 (SSE on x86-64), so every float
+ * operation rounds once to nearest-even, as IEEE 754 single precision.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <float.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#if FLT_EVAL_METHOD != 0
+#error "the oracle needs float arithmetic evaluated in single precision"
+#endif
+
+/* ------------------------------------------------------------------------------------------ */
+/* bf16 and fp32 bit-level conversions                                                         */
+/* ------------------------------------------------------------------------------------------ */
+
+/* bf16 is the top half of an IEEE fp32; widening is exact. */
+static float bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* fp32 -> bf16, round to nearest, ties to even (finite inputs).  Drop the low 16 bits and round
+ * up when the dropped part is above half, or exactly half with an odd kept part. */
+static uint16_t f32_to_bf16_rne(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint32_t kept = u >> 16;
+    uint32_t dropped = u & 0xFFFFu;
+    if (dropped > 0x8000u || (dropped == 0x8000u && (kept & 1u))) kept += 1u;
+    return (uint16_t)kept;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* E4M3 codec [OCP-FP8]                                                                       */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Decode one E4M3 code.  Bits: s eeee mmm, exponent bias 7.
+ *   e == 0          : subnormal, (-1)^s * (m / 8) * 2^-6
+ *   e == 15, m == 7 : NaN
+ *   otherwise       : (-1)^s * (1 + m / 8) * 2^(e - 7)                                       */
+double oracle_e4m3_decode(uint8_t code) {
+    int s = code >> 7;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);            /* m/8 * 2^-6 */
+    else        v = ldexp((double)(8 + m), e - 10);  /* (8+m)/8 * 2^(e-7) */
+    return s ? -v : v;
+}
+
+/* Round a non-negative double that holds an exact value to the nearest integer, ties to even. */
+static double rne_integer(double q) {
+    double fl = floor(q);
+    double frac = q - fl;                 /* exact: q has at most 53 significant bits */
+    if (frac > 0.5) return fl + 1.0;
+    if (frac < 0.5) return fl;
+    return (fmod(fl, 2.0) == 0.0) ? fl : fl + 1.0;
+}
+
+/* RNEsat: finite fp32 -> E4M3 code, round to nearest (ties to the even code) with saturation to
+ * +-448 (the largest finite E4M3 magnitude, code 0x7E).  Reading R3 keeps the sign of zero. */
+uint8_t oracle_e4m3_encode(float v) {
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs((double)v);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal range: the grid is k * 2^-9, k = 0..8 (k = 8 is the smallest normal,
+         * code 0x08, whose bit pattern is exactly 8) */
+        double k = rne_integer(a * 512.0);  /* scaling by a power of two is exact */
+        return sign | (uint8_t)k;
+    }
+    int ex;
+    (void)frexp(a, &ex);                    /* a = f * 2^ex, f in [0.5, 1) */
+    int E = ex - 1;                         /* floor(log2 a), in [-6, 8] */
+    double n = rne_integer(ldexp(a, 3 - E));/* significand in eighths: 8..16 */
+    if (n == 16.0) { E += 1; n = 8.0; }
+    return sign | (uint8_t)(((E + 7) << 3) | ((int)n - 8));
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Scales                                                                                     */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Reading R1: fp32 scale from the block's absolute maximum. */
+static float scale_f32_from_amax(float amax) {
+    if (amax == 0.0f) return 1.0f;
+    return amax / 448.0f;                   /* one IEEE fp32 division */
+}
+
+/* Reading R2: E8M0 exponent byte from the block's absolute maximum.  r = fp32(amax / 448);
+ * e = the smallest integer with 2^e >= r (r's unbiased exponent, plus one when r is not an
+ * exact power of two); clamp to [-127, 127]; byte = e + 127 [DSv4-WOA section 1: bias 127]. */
+static uint8_t e8m0_from_amax(float amax) {
+    if (amax == 0.0f) return 127;
+    float r = amax / 448.0f;
+    int ex;
+    double f = frexp((double)r, &ex);       /* r = f * 2^ex, f in [0.5, 1) */
+    int e = (f == 0.5) ? ex - 1 : ex;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return (uint8_t)(e + 127);
+}
+
+/* Value of an E8M0 byte as fp32: 2^(byte - 127); byte 255 is NaN and never produced here. */
+static float e8m0_value(uint8_t byte) {
+    return ldexpf(1.0f, (int)byte - 127);
+}
+
+/* [DSv4-WOA section 1]: an fp32 scale converts to E8M0 only when it is an exact power of two;
+ * e = round(log2 s), accepted iff 2^e == s, byte = e + 127.  Returns the byte, or -1 when the
+ * conversion would lose information (the page's "None"). */
+int oracle_e8m0_lossless_from_f32(float s) {
+    if (!(s > 0.0f) || isinf(s)) return -1;
+    double e = nearbyint(log2((double)s));
+    if (ldexp(1.0, (int)e) != (double)s) return -1;
+    if (e < -127 || e > 127) return -1;
+    return (int)e + 127;
+}
+
+double oracle_e8m0_decode(uint8_t byte) {
+    if (byte == 255) return NAN;
+    return ldexp(1.0, (int)byte - 127);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* a1 / a2: weight requantization in 128x128 blocks [FP8-RL (i)], [DSv4-WOA section 2]         */
+/* ------------------------------------------------------------------------------------------ */
+
+/* W is bf16 [N, K] row-major with leading dimension ldw (elements).  Produces codes q [N, K]
+ * (leading dimension ldq) and one scale per 128x128 block in a row-major [N/128, K/128] grid:
+ * fp32 when fmt == 0, E8M0 bytes when fmt == 1.  N and K are multiples of 128. */
+void oracle_quant_weight_block(const uint16_t *w, int64_t N, int64_t K, int64_t ldw,
+                               uint8_t *q, int64_t ldq, void *sw, int fmt) {
+    int64_t NB = N / 128, KB = K / 128;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t blk = 0; blk < NB * KB; ++blk) {
+        int64_t nb = blk / KB, kb = blk % KB;
+        float amax = 0.0f;
+        for (int64_t i = 0; i < 128; ++i)
+            for (int64_t j = 0; j < 128; ++j) {
+                float a = fabsf(bf16_to_f32(w[(nb * 128 + i) * ldw + kb * 128 + j]));
+                if (a > amax) amax = a;
+            }
+        float s;
+        if (fmt == 0) {
+            s = scale_f32_from_amax(amax);
+            ((float *)sw)[nb * KB + kb] = s;
+        } else {
+            uint8_t byte = e8m0_from_amax(amax);
+            s = e8m0_value(byte);
+            ((uint8_t *)sw)[nb * KB + kb] = byte;
+        }
+        for (int64_t i = 0; i < 128; ++i)
+            for (int64_t j = 0; j < 128; ++j) {
+                float x = bf16_to_f32(w[(nb * 128 + i) * ldw + kb * 128 + j]);
+                q[(nb * 128 + i) * ldq + kb * 128 + j] = oracle_e4m3_encode(x / s);
+            }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* a3: per-token 1x128 activation quantization [DSv4-WOA section 3: quant_group_size=128]      */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Quantize one 128-wide group of fp32 values (already bf16-representable).  Writes 128 codes
+ * and returns the fp32 scale. */
+static float quant_group_1x128(const float *y, uint8_t *q) {
+    float amax = 0.0f;
+    for (int j = 0; j < 128; ++j) {
+        float a = fabsf(y[j]);
+        if (a > amax) amax = a;
+    }
+    float s = scale_f32_from_amax(amax);
+    for (int j = 0; j < 128; ++j) q[j] = oracle_e4m3_encode(y[j] / s);
+    return s;
+}
+
+/* X bf16 [M, K] (leading dimension ldx) -> codes [M, K] (ldq) and fp32 scales sa[kb*lds + m]. */
+void oracle_quant_token_1x128(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                              uint8_t *q, int64_t ldq, float *sa, int64_t lds) {
+    int64_t KB = K / 128;
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t m = 0; m < M; ++m) {
+        float y[128];
+        for (int64_t kb = 0; kb < KB; ++kb) {
+            for (int j = 0; j < 128; ++j) y[j] = bf16_to_f32(x[m * ldx + kb * 128 + j]);
+            sa[kb * lds + m] = quant_group_1x128(y, q + m * ldq + kb * 128);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* a4: RMSNorm followed by the 1x128 token quant [SGL-RMSQ section 1], [torch-RMS], reading R4  */
+/* ------------------------------------------------------------------------------------------ */
+
+/* The per-row inverse RMS of reading R4.  x is one bf16 row of length K. */
+static float rms_inverse(const uint16_t *x, int64_t K, float eps) {
+    int64_t KB = K / 128;
+    double S = 0.0;
+    for (int64_t b = 0; b < KB; ++b) {
+        double P = 0.0;
+        for (int j = 0; j < 128; ++j) {
+            double v = (double)bf16_to_f32(x[b * 128 + j]);
+            P = P + v * v;                  /* v*v is exact in fp64 (<= 16 significant bits) */
+        }
+        S = S + P;
+    }
+    double var = S / (double)K + (double)eps;
+    return (float)(1.0 / sqrt(var));
+}
+
+/* Unfused RMSNorm as a bf16 layer writes it: y bf16 [M, K] (leading dimension ldy). */
+void oracle_rmsnorm_bf16(const uint16_t *x, const uint16_t *gamma, float eps, int64_t M,
+                         int64_t K, int64_t ldx, uint16_t *y, int64_t ldy) {
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t m = 0; m < M; ++m) {
+        float r = rms_inverse(x + m * ldx, K, eps);
+        for (int64_t k = 0; k < K; ++k) {
+            float t = bf16_to_f32(x[m * ldx + k]) * r;   /* fp32, rounded once */
+            float u = t * bf16_to_f32(gamma[k]);         /* fp32, rounded once */
+            y[m * ldy + k] = f32_to_bf16_rne(u);
+        }
+    }
+}
+
+/* Fused front end: RMSNorm (gamma != NULL) then 1x128 token quant; gamma == NULL is the plain
+ * token quant of a3.  The normalised row is never stored. */
+void oracle_rmsnorm_quant_token(const uint16_t *x, const uint16_t *gamma, float eps, int64_t M,
+                                int64_t K, int64_t ldx, uint8_t *q, int64_t ldq, float *sa,
+                                int64_t lds) {
+    if (gamma == NULL) {
+        oracle_quant_token_1x128(x, M, K, ldx, q, ldq, sa, lds);
+        return;
+    }
+    int64_t KB = K / 128;
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t m = 0; m < M; ++m) {
+        float r = rms_inverse(x + m * ldx, K, eps);
+        float y[128];
+        for (int64_t kb = 0; kb < KB; ++kb) {
+            for (int j = 0; j < 128; ++j) {
+                int64_t k = kb * 128 + j;
+                float t = bf16_to_f32(x[m * ldx + k]) * r;
+                float u = t * bf16_to_f32(gamma[k]);
+                y[j] = bf16_to_f32(f32_to_bf16_rne(u));
+            }
+            sa[kb * lds + m] = quant_group_1x128(y, q + m * ldq + kb * 128);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* a5 / a6: block-scaled W8A8 GEMM reference, reading R6                                       */
+/* ------------------------------------------------------------------------------------------ */
+
+/* One output element in fp64: ref = sum_kb (sa*sw) * P_kb, P_kb = sum_{k in kb} dec(a)*dec(w)
+ * (exact in fp64), and absref = sum_k |dec(a) * sa * dec(w) * sw|, the magnitude the error
+ * bound is relative to. */
+static void gemm_element(const uint8_t *arow, const uint8_t *wrow, int64_t K, const float *sa,
+                         int64_t lds, int64_t m, const void *sw_row, int sw_fmt, double *ref,
+                         double *absref) {
+    int64_t KB = K / 128;
+    double acc = 0.0, aacc = 0.0;
+    for (int64_t kb = 0; kb < KB; ++kb) {
+        double P = 0.0, PA = 0.0;
+        for (int j = 0; j < 128; ++j) {
+            double prod = oracle_e4m3_decode(arow[kb * 128 + j]) *
+                          oracle_e4m3_decode(wrow[kb * 128 + j]);
+            P += prod;
+            PA += fabs(prod);
+        }
+        double swv = (sw_fmt == 0) ? (double)((const float *)sw_row)[kb]
+                                   : oracle_e8m0_decode(((const uint8_t *)sw_row)[kb]);
+        double sc = (double)sa[kb * lds + m] * swv;
+        acc += sc * P;
+        aacc += fabs(sc) * PA;
+    }
+    *ref = acc;
+    *absref = aacc;
+}
+
+/* Dense GEMM reference on a subset of rows.  aq [M, K] (lda), wq [N, K] (ldw), sa as R5,
+ * sw [N/128, K/128] (fp32 or E8M0).  rows[i] selects the output row; ref/absref are
+ * [nrows, N] fp64. */
+void oracle_gemm_w8a8_block_rows(const uint8_t *aq, int64_t lda, const float *sa, int64_t lds,
+                                 const uint8_t *wq, int64_t ldw, const void *sw, int sw_fmt,
+                                 int64_t N, int64_t K, const int64_t *rows, int64_t nrows,
+                                 double *ref, double *absref) {
+    int64_t KB = K / 128;
+    size_t sw_elem = (sw_fmt == 0) ? sizeof(float) : 1;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < nrows; ++i)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t m = rows[i];
+            const char *sw_row = (const char *)sw + (size_t)((n / 128) * KB) * sw_elem;
+            gemm_element(aq + m * lda, wq + n * ldw, K, sa, lds, m, sw_row, sw_fmt,
+                         &ref[i * N + n], &absref[i * N + n]);
+        }
+}
+
+/* Grouped GEMM reference [DSv4-WOA section 3: batched per-group GEMM].  Expert e owns the rows
+ * [off[e], off[e+1]) of aq and uses wq[e] ([N, K], stride N*ldw per expert) and
+ * sw[e] ([N/128, K/128]).  Computes the selected rows only. */
+void oracle_grouped_gemm_w8a8_block_rows(const uint8_t *aq, int64_t lda, const float *sa,
+                                         int64_t lds, const uint8_t *wq, int64_t ldw,
+                                         const void *sw, int sw_fmt, const int32_t *off,
+                                         int64_t E, int64_t N, int64_t K, const int64_t *rows,
+                                         int64_t nrows, double *ref, double *absref) {
+    int64_t KB = K / 128, NB = N / 128;
+    size_t sw_elem = (sw_fmt == 0) ? sizeof(float) : 1;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t m = rows[i];
+        int64_t e = 0;
+        while (e < E && !(m >= off[e] && m < off[e + 1])) ++e;
+        for (int64_t n = 0; n < N; ++n) {
+            if (e == E) {                      /* row owned by no expert: no output */
+                ref[i * N + n] = 0.0;
+                absref[i * N + n] = 0.0;
+                continue;
+            }
+            const uint8_t *we = wq + e * N * ldw;
+            const char *sw_row = (const char *)sw + (size_t)((e * NB + n / 128) * KB) * sw_elem;
+            gemm_element(aq + m * lda, we + n * ldw, K, sa, lds, m, sw_row, sw_fmt,
+                         &ref[i * N + n], &absref[i * N + n]);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Helpers exposed for the oracle's own pin tests                                              */
+/* ------------------------------------------------------------------------------------------ */
+
+void oracle_e4m3_encode_array(const float *v, int64_t n, uint8_t *out) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(v[i]);
+}
+
+void oracle_f32_to_bf16_array(const float *v, int64_t n, uint16_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = f32_to_bf16_rne(v[i]);
+}
+
+float oracle_rms_inverse(const uint16_t *x, int64_t K, float eps) {
+    return rms_inverse(x, K, eps);
+}
+
+/* Exhaustive check of the encoder over every fp32 bit pattern whose value is finite, against
+ * an independent formulation: a search of the sorted table of the 127 non-negative finite E4M3
+ * values for the nearest one, ties to the even code, saturating above 448.  Returns the number
+ * of disagreements and stores the first one's bit pattern in *first_bad. */
+int64_t oracle_e4m3_encode_exhaustive_check(uint32_t *first_bad) {
+    double table[127];
+    for (int c = 0; c < 127; ++c) table[c] = oracle_e4m3_decode((uint8_t)c);
+    int64_t bad = 0;
+    uint32_t first = 0;
+    #pragma omp parallel for schedule(static) reduction(+ : bad)
+    for (int64_t u = 0; u < (1LL << 32); ++u) {
+        uint32_t bits = (uint32_t)u;
+        if (((bits >> 23) & 0xFF) == 0xFF) continue;      /* inf / NaN: out of scope */
+        float f;
+        memcpy(&f, &bits, sizeof f);
+        double a = fabs((double)f);
+        int code;
+        if (a >= 448.0) code = 126;
+        else {
+            /* binary search: largest index lo with table[lo] <= a */
+            int lo = 0, hi = 126;
+            while (lo < hi) {
+                int mid = (lo + hi + 1) / 2;
+                if (table[mid] <= a) lo = mid; else hi = mid - 1;
+            }
+            code = lo;
+            if (lo < 126) {
+                double dlo = a - table[lo], dhi = table[lo + 1] - a;
+                if (dhi < dlo || (dhi == dlo && (lo & 1))) code = lo + 1;
+            }
+        }
+        uint8_t expect = (uint8_t)(code | ((bits >> 24) & 0x80));
+        if (oracle_e4m3_encode(f) != expect) {
+            bad += 1;
+            #pragma omp critical
+            { if (first == 0 || bits < first) first = bits; }
+        }
+    }
+    *first_bad = first;
+    return bad;
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
