@@ -1,0 +1,120 @@
+"""Blockwise FP8 (E4M3) W8A8 linear layer on B200 (sm_100a).
+
+Thin torch-facing binding over the C ABI of ``libfp8q.so`` (declared in include/fp8q.h).  These
+functions only marshal arguments -- tensors become device pointers, the current torch CUDA stream
+becomes the launch stream, missing outputs are allocated with torch -- and every step of the
+computation runs in the library's CUDA kernels.  There is no CPU or PyTorch fallback: a missing
+library or a non-sm_100 device raises.
+
+    quant_weight_block(w, fmt)                 bf16 [N, K] -> (codes u8 [N, K], scales [N/128, K/128])
+    rmsnorm_quant_token(x, gamma, eps)         bf16 [M, K] -> (codes u8 [M, K], sa f32 [K/128, lds])
+    gemm_w8a8_block(aq, sa, wq, sw, fmt)       -> bf16 [M, N]
+    grouped_gemm_w8a8_block(aq, sa, wq, sw, offsets, fmt) -> bf16 [M, N]
+"""
+import torch
+
+from . import _lib
+from ._lib import (FP8Q_ERR_ALIGN, FP8Q_ERR_ARCH, FP8Q_ERR_ARG, FP8Q_ERR_LAUNCH, FP8Q_ERR_NULL,
+                   FP8Q_ERR_SHAPE, FP8Q_ERR_TIMEOUT, FP8Q_OK, FP8Q_SCALE_E8M0, FP8Q_SCALE_F32,
+                   Fp8qError)
+
+__all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
+           "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
+           "FP8Q_SCALE_E8M0", "scale_format"]
+
+
+def scale_format(fmt) -> int:
+    if fmt in (FP8Q_SCALE_F32, "f32", "fp32", torch.float32):
+        return FP8Q_SCALE_F32
+    if fmt in (FP8Q_SCALE_E8M0, "e8m0", torch.uint8):
+        return FP8Q_SCALE_E8M0
+    raise ValueError(f"unknown scale format {fmt!r}")
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _ld(t: torch.Tensor) -> int:
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit stride along its last dimension")
+    return t.stride(0)
+
+
+def quant_weight_block(w: torch.Tensor, fmt="f32", out_q=None, out_s=None, stream=None):
+    """bf16 W [N, K] -> (E4M3 codes uint8 [N, K], block scales [N/128, K/128] fp32 or E8M0)."""
+    f = scale_format(fmt)
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=w.device) if out_q is None else out_q
+    s = (torch.empty((N // 128, K // 128), device=w.device,
+                     dtype=torch.float32 if f == FP8Q_SCALE_F32 else torch.uint8)
+         if out_s is None else out_s)
+    st = _lib.lib().fp8q_quant_weight_block(_ptr(w), N, K, _ld(w), _ptr(q), _ld(q), _ptr(s), f,
+                                            _stream(stream))
+    _lib.check(st, "fp8q_quant_weight_block")
+    return q, s
+
+
+def rmsnorm_quant_token(x: torch.Tensor, gamma=None, eps: float = 1e-6, lds=None, out_q=None,
+                        out_sa=None, stream=None):
+    """bf16 X [M, K] -> (codes uint8 [M, K], sa fp32 [K/128, lds]); sa[kb, m] is the scale of
+    row m, K-block kb.  gamma=None: plain 1x128 token quant without RMSNorm."""
+    M, K = x.shape
+    if lds is None:
+        lds = max(4, (M + 3) // 4 * 4)
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if out_q is None else out_q
+    sa = (torch.empty((K // 128, lds), dtype=torch.float32, device=x.device)
+          if out_sa is None else out_sa)
+    st = _lib.lib().fp8q_rmsnorm_quant_token(_ptr(x), _ptr(gamma), float(eps), M, K, _ld(x),
+                                             _ptr(q), _ld(q), _ptr(sa), sa.stride(0),
+                                             _stream(stream))
+    _lib.check(st, "fp8q_rmsnorm_quant_token")
+    return q, sa
+
+
+def gemm_w8a8_block(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                    fmt=None, out=None, stream=None):
+    """Codes aq [M, K] (scales sa [K/128, lds]) x codes wq [N, K] (scales sw [N/128, K/128])
+    -> bf16 [M, N]."""
+    f = scale_format(sw.dtype if fmt is None else fmt)
+    M, K = aq.shape
+    N = wq.shape[0]
+    o = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device) if out is None else out
+    st = _lib.lib().fp8q_gemm_w8a8_block(_ptr(aq), _ld(aq), _ptr(sa), sa.stride(0), _ptr(wq),
+                                         _ld(wq), _ptr(sw), f, M, N, K, _ptr(o), _ld(o),
+                                         _stream(stream))
+    _lib.check(st, "fp8q_gemm_w8a8_block")
+    return o
+
+
+def grouped_gemm_w8a8_block(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor,
+                            sw: torch.Tensor, group_offsets: torch.Tensor, fmt=None, out=None,
+                            stream=None):
+    """Rows [off[e], off[e+1]) of aq times expert e's codes wq[e] ([E, N, K], scales
+    sw [E, N/128, K/128]) -> bf16 [M, N].  group_offsets: int32 [E+1] on the device."""
+    f = scale_format(sw.dtype if fmt is None else fmt)
+    M, K = aq.shape
+    E, N, K2 = wq.shape
+    if K2 != K:
+        raise ValueError("K mismatch")
+    if wq.stride(2) != 1 or wq.stride(0) != N * wq.stride(1):
+        raise ValueError("wq must be [E, N, K] with expert stride N * ldw")
+    if group_offsets.dtype != torch.int32 or group_offsets.numel() != E + 1:
+        raise ValueError("group_offsets must be int32 [E + 1]")
+    o = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device) if out is None else out
+    st = _lib.lib().fp8q_grouped_gemm_w8a8_block(_ptr(aq), _ld(aq), _ptr(sa), sa.stride(0),
+                                                 _ptr(wq), wq.stride(1), _ptr(sw), f,
+                                                 _ptr(group_offsets), E, M, N, K, _ptr(o),
+                                                 _ld(o), _stream(stream))
+    _lib.check(st, "fp8q_grouped_gemm_w8a8_block")
+    return o
+
+
+def check_device_error(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device error word."""
+    return _lib.lib().fp8q_check_device_error(_stream(stream))

@@ -1,0 +1,284 @@
+// fp8q.cu -- the C ABI of libfp8q.so: argument checks, TMA descriptors and kernel launches.
+// The declarations and the contract of every entry point are in include/fp8q.h.
+#include "fp8q.h"
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "gemm_kernel.cuh"
+#include "ptx.cuh"
+#include "quant_kernels.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxTokenK = 16384;
+
+struct DeviceState {
+  bool probed = false;
+  bool is_sm100 = false;
+  int sms = 0;
+  bool attrs_set = false;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_state(DeviceState **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_ARCH;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState &st = g_dev[dev];
+  if (!st.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FP8Q_ERR_ARCH;
+    st.is_sm100 = (major == 10 && minor == 0);
+    st.sms = sms;
+    st.probed = true;
+  }
+  if (!st.is_sm100) return FP8Q_ERR_ARCH;
+  if (!st.attrs_set) {
+    if (cudaFuncSetAttribute(fp8q::k_gemm_w8a8_block<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fp8q::kGemmSmemDense) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_gemm_w8a8_block<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fp8q::kGemmSmemGrouped) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess)
+      return FP8Q_ERR_LAUNCH;
+    st.attrs_set = true;
+  }
+  *out = &st;
+  return FP8Q_OK;
+}
+
+int get_encoder() {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_encode) return FP8Q_OK;
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return FP8Q_ERR_LAUNCH;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return FP8Q_OK;
+}
+
+// 2-D uint8 tensor map over a row-major [rows][ld] matrix, box = box_rows x 128 bytes, 128-byte
+// swizzle, out-of-bounds elements read as zero.
+int make_u8_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, int64_t ld,
+                uint32_t box_rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld)};
+  const cuuint32_t box[2] = {128, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_LAUNCH;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int launch_status() {
+  return cudaGetLastError() == cudaSuccess ? FP8Q_OK : FP8Q_ERR_LAUNCH;
+}
+
+int check_gemm_common(const void *aq, int64_t lda, const float *sa, int64_t lds, const void *wq,
+                      int64_t ldw, const void *sw, int sw_fmt, int64_t M, int64_t N, int64_t K,
+                      const void *out, int64_t ldo) {
+  if (sw_fmt != FP8Q_SCALE_F32 && sw_fmt != FP8Q_SCALE_E8M0) return FP8Q_ERR_ARG;
+  if (M < 0 || N <= 0 || K <= 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
+  if (M > INT32_MAX - 256 || N > (1 << 30) || K > (1 << 30)) return FP8Q_ERR_SHAPE;
+  if (lda < K || ldw < K || ldo < N || lds < M) return FP8Q_ERR_SHAPE;
+  if (M == 0) return FP8Q_OK;
+  if (!aq || !sa || !wq || !sw || !out) return FP8Q_ERR_NULL;
+  if (!aligned16(aq) || !aligned16(wq) || !aligned16(out) || !aligned16(sa) || !aligned16(sw) ||
+      lda % 16 || ldw % 16 || ldo % 8 || lds % 4)
+    return FP8Q_ERR_ALIGN;
+  return FP8Q_OK;
+}
+
+int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int64_t lds,
+                const void *wq, int64_t ldw, const void *sw, int sw_fmt,
+                const int32_t *group_offsets, int64_t E, int64_t M, int64_t N, int64_t K,
+                void *out, int64_t ldo, cudaStream_t stream) {
+  DeviceState *st = nullptr;
+  int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  if ((rc = get_encoder()) != FP8Q_OK) return rc;
+  CUtensorMap tm_a, tm_b;
+  if ((rc = make_u8_map(&tm_a, aq, M, K, lda, fp8q::kBM)) != FP8Q_OK) return rc;
+  const int64_t b_rows = grouped ? E * N : N;
+  if ((rc = make_u8_map(&tm_b, wq, b_rows, K, ldw, fp8q::kBN)) != FP8Q_OK) return rc;
+  fp8q::GemmArgs a;
+  a.sa = sa;
+  a.lds = lds;
+  a.sw = sw;
+  a.sw_fmt = sw_fmt;
+  a.group_offsets = group_offsets;
+  a.E = static_cast<int>(E);
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.out = static_cast<uint16_t *>(out);
+  a.ldo = ldo;
+  a.num_n = static_cast<int>((N + fp8q::kBN - 1) / fp8q::kBN);
+  a.num_m = static_cast<int>((M + fp8q::kBM - 1) / fp8q::kBM);
+  // Upper bound of the tile count (grouped: every expert may add one partial m-tile).
+  const int64_t tiles = (static_cast<int64_t>(a.num_m) + (grouped ? E : 0)) * a.num_n;
+  const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+  if (grouped)
+    fp8q::k_gemm_w8a8_block<true><<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemGrouped, stream>>>(
+        tm_a, tm_b, a);
+  else
+    fp8q::k_gemm_w8a8_block<false><<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemDense, stream>>>(
+        tm_a, tm_b, a);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8q_abi_version(void) { return (1 << 16) | 0; }
+
+const char *fp8q_status_string(int status) {
+  switch (status) {
+    case FP8Q_OK: return "ok";
+    case FP8Q_ERR_NULL: return "null pointer argument";
+    case FP8Q_ERR_SHAPE: return "unsupported shape (K and N must be multiples of 128; sizes >= 0; ld >= extent)";
+    case FP8Q_ERR_ALIGN: return "pointer or leading dimension not 16-byte aligned";
+    case FP8Q_ERR_ARCH: return "current device is not sm_100 (B200)";
+    case FP8Q_ERR_LAUNCH: return "CUDA runtime or launch failure";
+    case FP8Q_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (outputs incomplete)";
+    case FP8Q_ERR_ARG: return "enum argument out of range";
+    default: return "unknown status";
+  }
+}
+
+int fp8q_quant_weight_block(const void *w_bf16, int64_t N, int64_t K, int64_t ldw,
+                            void *wq_e4m3, int64_t ldq, void *sw, int sw_fmt,
+                            cudaStream_t stream) {
+  if (sw_fmt != FP8Q_SCALE_F32 && sw_fmt != FP8Q_SCALE_E8M0) return FP8Q_ERR_ARG;
+  if (N < 0 || K < 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
+  if (ldw < K || ldq < K) return FP8Q_ERR_SHAPE;
+  if (N == 0 || K == 0) return FP8Q_OK;
+  if (!w_bf16 || !wq_e4m3 || !sw) return FP8Q_ERR_NULL;
+  if (!aligned16(w_bf16) || !aligned16(wq_e4m3) || ldw % 8 || ldq % 16) return FP8Q_ERR_ALIGN;
+  if (sw_fmt == FP8Q_SCALE_F32 && (reinterpret_cast<uintptr_t>(sw) & 3u)) return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  const int KB = static_cast<int>(K / 128);
+  const int64_t nblocks = (N / 128) * (K / 128);
+  const int64_t grid = nblocks < (1ll << 30) ? nblocks : (1ll << 30);
+  const auto *w = static_cast<const uint16_t *>(w_bf16);
+  auto *q = static_cast<uint8_t *>(wq_e4m3);
+  if (sw_fmt == FP8Q_SCALE_F32)
+    fp8q::k_quant_weight_block<fp8q::kScaleF32><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        w, ldw, q, ldq, sw, KB, nblocks);
+  else
+    fp8q::k_quant_weight_block<fp8q::kScaleE8M0><<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        w, ldw, q, ldq, sw, KB, nblocks);
+  return launch_status();
+}
+
+int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
+                             int64_t K, int64_t ldx, void *xq_e4m3, int64_t ldq, float *sa,
+                             int64_t lds, cudaStream_t stream) {
+  if (M < 0 || K <= 0 || K % 128 || K > kMaxTokenK) return FP8Q_ERR_SHAPE;
+  if (ldx < K || ldq < K || lds < M) return FP8Q_ERR_SHAPE;
+  if (M == 0) return FP8Q_OK;
+  if (!x_bf16 || !xq_e4m3 || !sa) return FP8Q_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(xq_e4m3) || !aligned16(sa) || ldx % 8 || ldq % 16 ||
+      lds % 4 || (gamma_bf16 && !aligned16(gamma_bf16)))
+    return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  const bool norm = gamma_bf16 != nullptr;
+  const int KB = static_cast<int>(K / 128);
+  const int row_bytes = KB * fp8q::kRowBlockStride;
+  const int gamma_bytes = norm ? row_bytes : 0;
+  const int budget = 227 * 1024;
+  int wpc = (budget - gamma_bytes) / (2 * row_bytes);
+  if (wpc > 4) wpc = 4;
+  if (wpc < 1) return FP8Q_ERR_SHAPE;
+  const int smem = gamma_bytes + wpc * 2 * row_bytes;
+  int per_sm = 1;
+  if (norm)
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_rmsnorm_quant_token<true>,
+                                                  32 * wpc, smem);
+  else
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_rmsnorm_quant_token<false>,
+                                                  32 * wpc, smem);
+  if (per_sm < 1) per_sm = 1;
+  const int64_t need = (M + wpc - 1) / wpc;
+  const int64_t cap = static_cast<int64_t>(st->sms) * per_sm;
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  const auto *x = static_cast<const uint16_t *>(x_bf16);
+  const auto *g = static_cast<const uint16_t *>(gamma_bf16);
+  auto *q = static_cast<uint8_t *>(xq_e4m3);
+  if (norm)
+    fp8q::k_rmsnorm_quant_token<true><<<grid, 32 * wpc, smem, stream>>>(
+        x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, lds);
+  else
+    fp8q::k_rmsnorm_quant_token<false><<<grid, 32 * wpc, smem, stream>>>(
+        x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds);
+  return launch_status();
+}
+
+int fp8q_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                         const void *wq, int64_t ldw, const void *sw, int sw_fmt, int64_t M,
+                         int64_t N, int64_t K, void *out_bf16, int64_t ldo,
+                         cudaStream_t stream) {
+  int rc = check_gemm_common(aq, lda, sa, lds, wq, ldw, sw, sw_fmt, M, N, K, out_bf16, ldo);
+  if (rc != FP8Q_OK || M == 0) return rc;
+  if (sw_fmt == FP8Q_SCALE_F32 && (reinterpret_cast<uintptr_t>(sw) & 3u)) return FP8Q_ERR_ALIGN;
+  return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K, out_bf16,
+                     ldo, stream);
+}
+
+int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                                 const void *wq, int64_t ldw, const void *sw, int sw_fmt,
+                                 const int32_t *group_offsets, int64_t E, int64_t M, int64_t N,
+                                 int64_t K, void *out_bf16, int64_t ldo, cudaStream_t stream) {
+  if (E <= 0 || E > fp8q::kMaxExperts) return FP8Q_ERR_SHAPE;
+  int rc = check_gemm_common(aq, lda, sa, lds, wq, ldw, sw, sw_fmt, M, N, K, out_bf16, ldo);
+  if (rc != FP8Q_OK || M == 0) return rc;
+  if (!group_offsets) return FP8Q_ERR_NULL;
+  if (E * N > INT32_MAX) return FP8Q_ERR_SHAPE;
+  return launch_gemm(true, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, group_offsets, E, M, N, K,
+                     out_bf16, ldo, stream);
+}
+
+int fp8q_check_device_error(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return FP8Q_ERR_LAUNCH;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fp8q::g_device_error, sizeof v) != cudaSuccess)
+    return FP8Q_ERR_LAUNCH;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(fp8q::g_device_error, &zero, sizeof zero) != cudaSuccess)
+      return FP8Q_ERR_LAUNCH;
+  }
+  return v == 0 ? FP8Q_OK : v;
+}
+
+}  // extern "C"

@@ -1,0 +1,406 @@
+// gemm_kernel.cuh -- block-scaled FP8 (E4M3) W8A8 GEMM for sm_100a, dense and grouped (MoE).
+//
+//   out[m, n] = bf16( sum_kb sa[m, kb] * sw[n / 128, kb] * P_kb[m, n] )
+//
+// P_kb, the dot product of the E4M3 codes over one 128-wide K-block, is computed by tcgen05.mma
+// (kind::f8f6f4, fp32 accumulate) into tensor memory; the scale product is applied and the
+// partials are accumulated in fp32 registers ("promotion") by the epilogue warps.
+//
+// Structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
+//   warp 0      TMA producer (lane 0): A tile 128 x 128 B and B tile 256 x 128 B per K-block into
+//               a 4-stage shared-memory ring, 128-byte swizzled
+//   warp 1      TMEM allocator (whole warp) and MMA issuer (lane 0): 4 MMAs (K = 32 each) per
+//               K-block into one of two 256-column TMEM buffers, so the MMAs of K-block kb + 1
+//               run while the epilogue promotes K-block kb
+//   warps 2-3   idle (they complete warpgroup 0 for the register hand-off)
+//   warps 4-11  epilogue/promotion: warp w reads TMEM lanes 32 * (w % 4) (its 32 rows of the
+//               tile) and column half (w - 4) / 4; each thread keeps 128 fp32 accumulators
+// Registers: launched at 168 per thread (384 x 168 = 64512); warpgroup 0 drops to 40 and the two
+// epilogue warpgroups rise to 232 (128 x 40 + 256 x 232 = 64512, per sub-partition 16128).
+// Every wait is bounded: on expiry a kernel records FP8Q_ERR_TIMEOUT in the device error word,
+// all roles leave their loops, in-flight copies and MMAs are drained, and TMEM is released.
+#pragma once
+#include <cuda.h>
+#include "ptx.cuh"
+
+namespace fp8q {
+
+constexpr int kBM = 128, kBN = 256, kBK = 128;
+constexpr int kStages = 4;
+constexpr int kGemmThreads = 384;
+constexpr int kProducerRegs = 40, kEpilogueRegs = 232;
+constexpr int kTileABytes = kBM * kBK;            // 16 KB
+constexpr int kTileBBytes = kBN * kBK;            // 32 KB
+constexpr int kStageBytes = kTileABytes + kTileBBytes;
+constexpr int kStagingBytesPerWarp = 32 * 64;     // 32 rows x 32 bf16 columns
+constexpr int kMaxExperts = 1024;
+constexpr int kGroupM = 16;                       // rasterization: m-blocks per group
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+
+// Shared-memory layout (offsets from a 1024-byte aligned base).
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kStages * kTileABytes;
+constexpr int kOffStaging = kOffB + kStages * kTileBBytes;
+constexpr int kOffBar = kOffStaging + 8 * kStagingBytesPerWarp;
+constexpr int kNumBars = 2 * kStages + 4 + 1;     // full, empty, tmem_full[2], tmem_empty[2], done
+constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
+constexpr int kOffGroups = kOffMisc + 16;          // grouped: offsets[E+1], tile prefix[E+1]
+constexpr int kGemmSmemDense = kOffGroups + 1024;  // + alignment slack
+constexpr int kGemmSmemGrouped = kOffGroups + 2 * (kMaxExperts + 1) * 4 + 1024;
+
+// Instruction descriptor, kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B E4M3 (bits 7-9, 10-12
+// = 0), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (static_cast<uint32_t>(kBN >> 3) << 17) |
+                            (static_cast<uint32_t>(kBM >> 4) << 24);
+
+// Shared-memory matrix descriptor for a K-major tile written by TMA with 128-byte swizzle:
+// rows of 128 bytes, 8-row core groups 1024 bytes apart (stride byte offset), descriptor
+// version 1 (bit 46), swizzle mode 2 = 128B (bits 61-63).  Start address in 16-byte units.
+__device__ __forceinline__ uint64_t sdesc_k128(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+struct GemmArgs {
+  const float *sa;
+  int64_t lds;
+  const void *sw;       // fp32 or E8M0 bytes
+  int sw_fmt;
+  const int32_t *group_offsets;  // nullptr: dense
+  int E;
+  int M, N, K;
+  uint16_t *out;
+  int64_t ldo;
+  int num_n;            // ceil(N / 256)
+  int num_m;            // dense: ceil(M / 128)
+};
+
+struct Tile {
+  int m0;        // first row of the tile in A / out
+  int row_end;   // rows >= row_end are not stored (M, or the expert's end)
+  int n0;        // first column
+  int b_row;     // first row of the tile in the B tensor map (expert * N + n0)
+  int e;         // expert (0 when dense)
+};
+
+// Dense rasterization: groups of kGroupM m-blocks, m fastest inside a group, so that the CTAs
+// running at the same time share A and B tiles in L2.
+__device__ __forceinline__ Tile dense_tile(const GemmArgs &a, int t) {
+  const int per_group = kGroupM * a.num_n;
+  const int g = t / per_group;
+  const int first_m = g * kGroupM;
+  const int gm = min(a.num_m - first_m, kGroupM);
+  const int r = t - g * per_group;
+  Tile tl;
+  tl.m0 = (first_m + r % gm) * kBM;
+  tl.n0 = (r / gm) * kBN;
+  tl.row_end = a.M;
+  tl.b_row = tl.n0;
+  tl.e = 0;
+  return tl;
+}
+
+// Grouped: expert e owns m-tiles [prefix[e], prefix[e+1]); n fastest so the CTAs of one expert
+// share its weight in L2.
+__device__ __forceinline__ Tile grouped_tile(const GemmArgs &a, const int *s_off,
+                                             const int *s_prefix, int t) {
+  const int gm = t / a.num_n;
+  const int nb = t - gm * a.num_n;
+  int lo = 0, hi = a.E - 1;  // largest e with prefix[e] <= gm
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_prefix[mid] <= gm) lo = mid; else hi = mid - 1;
+  }
+  Tile tl;
+  tl.e = lo;
+  tl.m0 = s_off[lo] + (gm - s_prefix[lo]) * kBM;
+  tl.row_end = s_off[lo + 1];
+  tl.n0 = nb * kBN;
+  tl.b_row = lo * a.N + tl.n0;
+  return tl;
+}
+
+// Bounded wait by one thread.  Returns false on abort (another role gave up) or timeout.
+__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        record_error(6 /* FP8Q_ERR_TIMEOUT */);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait by a whole warp with a warp-uniform outcome.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  const int lane = threadIdx.x & 31;
+  uint64_t t0 = 0;
+  for (uint32_t n = 0;; ++n) {
+    const bool ok = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    if ((n & 63u) == 63u) {
+      int stop = 0;
+      if (lane == 0) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        if (*abort_flag) {
+          stop = 1;
+        } else if (now - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          record_error(6 /* FP8Q_ERR_TIMEOUT */);
+          stop = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+    }
+  }
+}
+
+// Wait that ignores the abort flag (teardown drains); still bounded.
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(6 /* FP8Q_ERR_TIMEOUT */);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ float load_sw(const GemmArgs &a, const uint8_t *sw_row, int kb) {
+  if (a.sw_fmt == 0) return __ldg(reinterpret_cast<const float *>(sw_row) + kb);
+  const int b = __ldg(sw_row + kb);
+  return b >= 1 ? __uint_as_float(static_cast<uint32_t>(b) << 23) : __uint_as_float(0x00400000u);
+}
+
+template <bool GROUPED>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm_w8a8_block(const __grid_constant__ CUtensorMap tm_a,
+                      const __grid_constant__ CUtensorMap tm_b, const GemmArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + kOffBar;              // [kStages]
+  const uint32_t bar_empty = bar_full + 8 * kStages;      // [kStages]
+  const uint32_t bar_tfull = bar_empty + 8 * kStages;     // [2]
+  const uint32_t bar_tempty = bar_tfull + 16;             // [2]
+  const uint32_t bar_done = bar_tempty + 16;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+  int *s_off = reinterpret_cast<int *>(smem + kOffGroups);
+  int *s_prefix = s_off + (kMaxExperts + 1);
+
+  const int KB = args.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_tfull + 8 * i, 1);
+      mbar_init(bar_tempty + 8 * i, 8);
+    }
+    mbar_init(bar_done, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), 512);
+    tmem_relinquish();
+  }
+  int total_tiles;
+  if (GROUPED) {
+    // Clamp the offsets into [previous, M] and count m-tiles per expert.
+    for (int i = threadIdx.x; i <= args.E; i += blockDim.x) s_off[i] = args.group_offsets[i];
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int prev = 0, acc = 0;
+      for (int e = 0; e <= args.E; ++e) {
+        int v = s_off[e];
+        v = v < prev ? prev : (v > args.M ? args.M : v);
+        if (e == 0) v = v < 0 ? 0 : v;
+        s_off[e] = v;
+        prev = v;
+      }
+      for (int e = 0; e < args.E; ++e) {
+        s_prefix[e] = acc;
+        acc += (s_off[e + 1] - s_off[e] + kBM - 1) / kBM;
+      }
+      s_prefix[args.E] = acc;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  total_tiles = GROUPED ? s_prefix[args.E] * args.num_n : args.num_m * args.num_n;
+
+  if (warp < 4) {
+    reg_dealloc<kProducerRegs>();
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_b);
+        uint32_t it = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+          const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, t) : dense_tile(args, t);
+          bool ok = true;
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            if (!wait_one(bar_empty + 8 * s, ph ^ 1u, s_abort)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar_full + 8 * s, kStageBytes);
+            tma_load_2d(sbase + kOffA + s * kTileABytes, &tm_a, kb * kBK, tl.m0, bar_full + 8 * s);
+            tma_load_2d(sbase + kOffB + s * kTileBBytes, &tm_b, kb * kBK, tl.b_row,
+                        bar_full + 8 * s);
+          }
+          if (!ok) break;
+        }
+        // Drain: every issued load has landed before the CTA can exit.
+        for (uint32_t s = 0; s < kStages && s < it; ++s) {
+          const uint32_t last = s + ((it - 1 - s) / kStages) * kStages;  // last fill of stage s
+          wait_drain(bar_full + 8 * s, (last / kStages) & 1u);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        uint32_t it = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+          bool ok = true;
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            const uint32_t b = it & 1u, bph = (it >> 1) & 1u;
+            if (!wait_one(bar_tempty + 8 * b, bph ^ 1u, s_abort)) { ok = false; break; }
+            if (!wait_one(bar_full + 8 * s, ph, s_abort)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t ad = sdesc_k128(sbase + kOffA + s * kTileABytes);
+            const uint64_t bd = sdesc_k128(sbase + kOffB + s * kTileBBytes);
+            const uint32_t d = tmem_base + b * kBN;
+#pragma unroll
+            for (int kk = 0; kk < kBK / 32; ++kk)  // 32-byte steps inside the 128-byte row
+              mma_f8f6f4(d, ad + 2 * kk, bd + 2 * kk, kIdesc, kk > 0 ? 1u : 0u);
+            mma_commit(bar_empty + 8 * s);
+            mma_commit(bar_tfull + 8 * b);
+          }
+          if (!ok) break;
+        }
+        // Every MMA has completed before TMEM is released.
+        mma_commit(bar_done);
+        wait_drain(bar_done, 0);
+      }
+      __syncwarp();
+    }
+  } else {
+    reg_alloc<kEpilogueRegs>();
+    // ------------------------------------------------------------------ epilogue / promotion
+    const int q = warp & 3;         // TMEM lane quarter = rows 32q .. 32q + 31 of the tile
+    const int h = (warp - 4) >> 2;  // column half of the 256-wide tile
+    const int NB = args.N / 128;
+    uint8_t *stage = smem + kOffStaging + (warp - 4) * kStagingBytesPerWarp;
+    const uint32_t stage_u32 = smem_u32(stage);
+    const size_t sw_elem = args.sw_fmt == 0 ? 4 : 1;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+      const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, t) : dense_tile(args, t);
+      const int row = tl.m0 + 32 * q + lane;
+      const bool row_ok = row < tl.row_end;
+      const int nbh = tl.n0 / 128 + h;
+      const bool col_ok = nbh < NB;
+      const uint8_t *sw_row = static_cast<const uint8_t *>(args.sw) +
+                              (static_cast<size_t>(tl.e) * NB + (col_ok ? nbh : 0)) * KB * sw_elem;
+      const float *sa_col = args.sa + row;
+      // scales for K-blocks kb and kb + 1 are loaded ahead of use
+      float sa0 = (row_ok) ? __ldg(sa_col) : 0.0f;
+      float sa1 = (row_ok && KB > 1) ? __ldg(sa_col + args.lds) : 0.0f;
+      float sw0 = col_ok ? load_sw(args, sw_row, 0) : 0.0f;
+      float sw1 = (col_ok && KB > 1) ? load_sw(args, sw_row, 1) : 0.0f;
+      float acc[128];
+#pragma unroll
+      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t b = it & 1u, bph = (it >> 1) & 1u;
+        if (!wait_warp(bar_tfull + 8 * b, bph, s_abort)) { ok = false; break; }
+        tc_fence_after();
+        const float sc = __fmul_rn(sa0, sw0);
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * kBN + h * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + 32 * c, r);
+          tmem_ld_wait(r);
+          if (c == 3) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) acc[32 * c + j] = fmaf(__uint_as_float(r[j]), sc, acc[32 * c + j]);
+        }
+        sa0 = sa1;
+        sw0 = sw1;
+        if (kb + 2 < KB) {
+          sa1 = row_ok ? __ldg(sa_col + static_cast<int64_t>(kb + 2) * args.lds) : 0.0f;
+          sw1 = col_ok ? load_sw(args, sw_row, kb + 2) : 0.0f;
+        }
+      }
+      if (!ok) break;
+      // bf16 conversion and store, 32 columns at a time through a swizzled staging buffer so
+      // that each global store instruction writes 64-byte row segments.
+      uint16_t *out_base = args.out + static_cast<int64_t>(tl.n0 + 128 * h);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const __nv_bfloat162 v2 =
+                __floats2bfloat162_rn(acc[32 * c4 + 8 * j + 2 * u], acc[32 * c4 + 8 * j + 2 * u + 1]);
+            pk[u] = *reinterpret_cast<const uint32_t *>(&v2);
+          }
+          const int phys = j ^ ((lane >> 1) & 3);
+          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stage_u32 + lane * 64 + phys * 16),
+                       "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                       : "memory");
+        }
+        __syncwarp();
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const int r = p * 8 + (lane >> 2), c = lane & 3;
+          const int phys = c ^ ((r >> 1) & 3);
+          uint4 v;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(stage_u32 + r * 64 + phys * 16)
+                       : "memory");
+          const int grow = tl.m0 + 32 * q + r;
+          if (col_ok && grow < tl.row_end)
+            *reinterpret_cast<uint4 *>(out_base + static_cast<int64_t>(grow) * args.ldo + 32 * c4 + 8 * c) = v;
+        }
+        __syncwarp();
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+}  // namespace fp8q

@@ -1,0 +1,144 @@
+/*
+ * fp8q.h -- C ABI of libfp8q.so, the blockwise FP8 (E4M3) W8A8 linear layer on B200 (sm_100a).
+ *
+ * Four operations make up the hot path of an FP8 linear layer whose bf16 weights change every
+ * step ("FP8-RL: A Practical and Stable Low-Precision Stack for LLM Reinforcement Learning",
+ * abstract, item (i): W8A8 linear layers with blockwise FP8 quantization, weights requantized
+ * after every policy update):
+ *
+ *   fp8q_quant_weight_block       bf16 W -> E4M3 codes + one scale per 128x128 block
+ *   fp8q_rmsnorm_quant_token      bf16 X -> [RMSNorm] -> E4M3 codes + one scale per 1x128 group
+ *   fp8q_gemm_w8a8_block          codes x codes -> bf16, per-K-block fp32 promotion
+ *   fp8q_grouped_gemm_w8a8_block  the same GEMM per expert over row groups (MoE)
+ *
+ * Numerics (shared by all entry points):
+ *   - E4M3 is the OCP FP8 E4M3 format (bias 7, max 448, no infinities, 0x7F/0xFF NaN).
+ *   - A block scale is s = amax / 448 in fp32 (IEEE division), or 1 for an all-zero block; the
+ *     codes are q = RNE-saturating-E4M3(x / s), x / s an IEEE fp32 division.  The sign of zero
+ *     is kept (a negative value that rounds to zero gives 0x80).
+ *   - E8M0 scales (FP8Q_SCALE_E8M0): one byte b, value 2^(b - 127); the quantizer picks the
+ *     smallest power of two >= fp32(amax / 448), exponent clamped to [-127, 127], so every
+ *     scale it writes is exactly representable ("DeepSeek V4 performance: FP8 WO_A output
+ *     projection (vLLM PR 54894 analysis)", section 1: unsigned exponent, bias 127, lossless
+ *     only for exact powers of two).
+ *   - Outputs of the two quantizers are bit-exact against the CPU oracle; GEMM outputs satisfy
+ *     |out - ref| <= 8e-3 * sum_k |dec(a) sa dec(w) sw| + 1 bf16 ulp of |ref|.
+ *
+ * Conventions:
+ *   - Every pointer argument is a DEVICE pointer on the current CUDA device, except where a
+ *     comment says otherwise.  The caller owns all buffers; the library never allocates device
+ *     memory and never synchronizes, except fp8q_check_device_error.  Work is enqueued on
+ *     `stream` (0 = legacy default stream).
+ *   - Leading dimensions are in ELEMENTS of the buffer's type.  Matrices are row-major.
+ *   - Shapes: K and N must be multiples of 128 ("... vLLM PR 54894 analysis", section 2: the
+ *     FP8 path requires out % 128 == 0 and in % 128 == 0).  Unlike the page, which falls back
+ *     to bf16, this library returns FP8Q_ERR_SHAPE.  M may be any value >= 0; M == 0 is a
+ *     successful no-op.
+ *   - Activation scales sa are fp32 in K-block-major layout: the scale of row m, K-block kb is
+ *     sa[kb * lds + m], lds >= M, lds % 4 == 0.  Weight scales sw are a row-major
+ *     [N/128][K/128] grid ("... vLLM PR 54894 analysis", section 2: scale viewed as
+ *     [groups, out/128, in/128]); the grouped GEMM takes [E][N/128][K/128].
+ *   - Alignment: every base pointer 16-byte aligned; leading dimensions such that each row
+ *     starts 16-byte aligned (bf16: ld % 8 == 0; u8: ld % 16 == 0; fp32: ld % 4 == 0).
+ *     Otherwise FP8Q_ERR_ALIGN.
+ *   - The current device must be sm_100 (B200); otherwise FP8Q_ERR_ARCH.
+ *   - Return value: an fp8q_status.  Only argument and launch errors are returned; a kernel
+ *     that gives up on a bounded internal wait records FP8Q_ERR_TIMEOUT in a device-side
+ *     error word, read (and cleared) by fp8q_check_device_error.
+ *   - Thread safety: the entry points keep no host state apart from per-device caches filled
+ *     on first use; concurrent calls on different streams are safe.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP8Q_OK = 0,
+  FP8Q_ERR_NULL = 1,    /* a required pointer is NULL */
+  FP8Q_ERR_SHAPE = 2,   /* K or N not a multiple of 128, negative size, ld too small, K too large */
+  FP8Q_ERR_ALIGN = 3,   /* a pointer or leading dimension breaks the 16-byte rule */
+  FP8Q_ERR_ARCH = 4,    /* current device is not sm_100, or no device */
+  FP8Q_ERR_LAUNCH = 5,  /* a CUDA runtime call or kernel launch failed */
+  FP8Q_ERR_TIMEOUT = 6, /* (device error word) a kernel gave up on a bounded wait */
+  FP8Q_ERR_ARG = 7      /* an enum argument is out of range */
+} fp8q_status;
+
+typedef enum {
+  FP8Q_SCALE_F32 = 0,   /* fp32 scales */
+  FP8Q_SCALE_E8M0 = 1   /* one unsigned-exponent byte per scale, value 2^(b - 127) */
+} fp8q_scale_fmt;
+
+/* Requantize a bf16 weight into 128x128-block FP8 (a1 with fp32 scales, a2 with E8M0 scales).
+ *   w_bf16   [N][ldw] bf16, read                        (N, K multiples of 128; ldw >= K)
+ *   wq_e4m3  [N][ldq] uint8 E4M3 codes, written         (ldq >= K)
+ *   sw       [N/128][K/128] fp32 (sw_fmt = FP8Q_SCALE_F32) or uint8 (FP8Q_SCALE_E8M0), written
+ * Source: FP8-RL abstract (i) (per-step requantization of changed policy weights);
+ * vLLM PR 54894 analysis, sections 1 and 2 (E8M0 bytes, the [out/128, in/128] scale grid). */
+int fp8q_quant_weight_block(const void *w_bf16, int64_t N, int64_t K, int64_t ldw,
+                            void *wq_e4m3, int64_t ldq, void *sw, int sw_fmt,
+                            cudaStream_t stream);
+
+/* Per-token 1x128 activation quantization, optionally fused with RMSNorm (a3 / a4).
+ *   x_bf16      [M][ldx] bf16, read
+ *   gamma_bf16  [K] bf16 RMSNorm weight, or NULL for plain token quant (no normalisation)
+ *   eps         RMSNorm epsilon (fp32; ignored when gamma_bf16 is NULL)
+ *   xq_e4m3     [M][ldq] uint8 codes, written
+ *   sa          fp32 scales, sa[kb * lds + m], written for m < M only
+ * With gamma: r = fp32(1 / sqrt(S / K + eps)) where S is the fp64 sum of x^2 taken in ascending
+ * k within each 128-block and then over blocks in ascending order; y = bf16_RNE((x * r) * gamma)
+ * with two fp32 roundings; the 1x128 quant then runs on y, which is never written to memory.
+ * K <= 16384.  Source: SGLang PR 21403 analysis, section 1 (RMSNorm with weight and epsilon
+ * fused with FP8 quant so the normalised tensor makes no round trip through memory); vLLM PR
+ * 54894 analysis, section 3 (quant_group_size = 128). */
+int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
+                             int64_t K, int64_t ldx, void *xq_e4m3, int64_t ldq, float *sa,
+                             int64_t lds, cudaStream_t stream);
+
+/* Block-scaled W8A8 GEMM (a5): out[m, n] = bf16( sum_kb sa[m, kb] * sw[n/128, kb] * P_kb[m, n] )
+ * where P_kb is the fp32 tensor-core dot product of the E4M3 codes over K-block kb and each
+ * K-block partial is promoted (scaled and accumulated) in fp32.
+ *   aq   [M][lda] uint8 activation codes     sa  fp32, sa[kb * lds + m]
+ *   wq   [N][ldw] uint8 weight codes         sw  [N/128][K/128], fp32 or E8M0 per sw_fmt
+ *   out  [M][ldo] bf16, written (rows < M, columns < N)
+ * Source: SGLang PR 21403 analysis, section 3 (the GEMM consumes the pre-quantized (codes,
+ * scale) pair and writes bf16); FP8-RL abstract (i). */
+int fp8q_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                         const void *wq, int64_t ldw, const void *sw, int sw_fmt, int64_t M,
+                         int64_t N, int64_t K, void *out_bf16, int64_t ldo, cudaStream_t stream);
+
+/* Grouped W8A8 GEMM for MoE experts (a6): for each expert e the rows
+ * [group_offsets[e], group_offsets[e+1]) of aq/sa/out are multiplied by expert e's weight.
+ *   wq             [E][N][ldw] uint8 codes (expert stride N * ldw)
+ *   sw             [E][N/128][K/128] fp32 or E8M0
+ *   group_offsets  [E + 1] int32, DEVICE memory, nondecreasing, [0] = 0, [E] = M.  The kernel
+ *                  clamps each offset into [previous offset, M]; rows not covered by any
+ *                  expert are left unwritten.
+ * E <= 1024.  Source: vLLM PR 54894 analysis, section 3 (batched FP8 GEMM over [groups, out,
+ * in] weights with per-group block scales); FP8-RL abstract (dense and MoE models). */
+int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                                 const void *wq, int64_t ldw, const void *sw, int sw_fmt,
+                                 const int32_t *group_offsets, int64_t E, int64_t M, int64_t N,
+                                 int64_t K, void *out_bf16, int64_t ldo, cudaStream_t stream);
+
+/* Synchronize `stream`, then read and clear the device error word of the current device.
+ * Returns FP8Q_OK, FP8Q_ERR_TIMEOUT (a kernel gave up on a bounded wait since the last call;
+ * its outputs are incomplete) or FP8Q_ERR_LAUNCH (the synchronize failed). */
+int fp8q_check_device_error(cudaStream_t stream);
+
+/* Static, NUL-terminated description of a status code.  Never NULL. */
+const char *fp8q_status_string(int status);
+
+/* ABI version: (major << 16) | minor. */
+int fp8q_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -1,0 +1,98 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU, exports exactly what include/fp8q.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_blockwise_w8a8_b200 import _lib, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "fp8q.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(fp8q_\w+)\s*\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _lib.lib()
+
+
+def test_exports_match_header(L):
+    names = declared_functions()
+    assert names == sorted(_lib.SIGNATURES), names
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.fp8q_abi_version() >> 16 == 1
+
+
+def test_status_strings(L):
+    for s in range(8):
+        assert len(_lib.status_string(s)) >= 2
+    assert _lib.status_string(99) == "unknown status"
+
+
+P = ctypes.c_void_p
+FAKE = 1 << 20          # a 16-byte aligned non-null address; never dereferenced on these paths
+
+
+def test_weight_quant_host_checks(L):
+    f = L.fp8q_quant_weight_block
+    assert f(FAKE, 128, 200, 200, FAKE, 208, FAKE, 0, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, 100, 128, 128, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, 128, 128, 64, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, 128, 128, 128, FAKE, 128, FAKE, 2, None) == _lib.FP8Q_ERR_ARG
+    assert f(None, 128, 128, 128, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_ERR_NULL
+    assert f(FAKE + 2, 128, 128, 128, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_ERR_ALIGN
+    assert f(FAKE, 128, 128, 132, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_ERR_ALIGN
+    assert f(FAKE, 0, 128, 128, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_OK      # empty: no-op
+
+
+def test_token_quant_host_checks(L):
+    f = L.fp8q_rmsnorm_quant_token
+    assert f(FAKE, None, 1e-6, 4, 100, 100, FAKE, 112, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, None, 1e-6, 4, 32768, 32768, FAKE, 32768, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, None, 1e-6, 8, 128, 128, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, None, 1e-6, 4, 128, 128, FAKE, 128, FAKE, 6, None) == _lib.FP8Q_ERR_ALIGN
+    assert f(FAKE, FAKE + 8, 1e-6, 4, 128, 128, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_ALIGN
+    assert f(None, None, 1e-6, 4, 128, 128, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_NULL
+    assert f(None, None, 1e-6, 0, 128, 128, None, 128, None, 4, None) == _lib.FP8Q_OK
+
+
+def test_gemm_host_checks(L):
+    g = L.fp8q_gemm_w8a8_block
+    ok = dict(aq=FAKE, lda=256, sa=FAKE, lds=64, wq=FAKE, ldw=256, sw=FAKE, fmt=0, M=64, N=128,
+              K=256, out=FAKE, ldo=128)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["aq"], a["lda"], a["sa"], a["lds"], a["wq"], a["ldw"], a["sw"], a["fmt"],
+                 a["M"], a["N"], a["K"], a["out"], a["ldo"], None)
+    assert call(N=100) == _lib.FP8Q_ERR_SHAPE
+    assert call(K=200, lda=208, ldw=208) == _lib.FP8Q_ERR_SHAPE
+    assert call(lds=32) == _lib.FP8Q_ERR_SHAPE
+    assert call(M=-1) == _lib.FP8Q_ERR_SHAPE
+    assert call(fmt=5) == _lib.FP8Q_ERR_ARG
+    assert call(sa=None) == _lib.FP8Q_ERR_NULL
+    assert call(lda=264) == _lib.FP8Q_ERR_ALIGN
+    assert call(out=FAKE + 4) == _lib.FP8Q_ERR_ALIGN
+    assert call(M=0, aq=None, sa=None, out=None) == _lib.FP8Q_OK
+    gg = L.fp8q_grouped_gemm_w8a8_block
+    assert gg(FAKE, 256, FAKE, 64, FAKE, 256, FAKE, 0, FAKE, 0, 64, 128, 256, FAKE, 128,
+              None) == _lib.FP8Q_ERR_SHAPE
+    assert gg(FAKE, 256, FAKE, 64, FAKE, 256, FAKE, 0, None, 4, 64, 128, 256, FAKE, 128,
+              None) == _lib.FP8Q_ERR_NULL
+
+
+def test_valid_call_without_gpu_reports_arch(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    f = L.fp8q_quant_weight_block
+    assert f(FAKE, 128, 128, 128, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_ERR_ARCH

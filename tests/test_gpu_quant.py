@@ -1,0 +1,160 @@
+"""GPU parity of the two quantizers against the oracle: bit-exact codes and scales.
+
+Weight blocks: "FP8-RL ..." abstract (i), "DeepSeek V4 ... (vLLM PR 54894 analysis)" sections 1-2.
+Token groups / RMSNorm: "... (vLLM PR 54894 analysis)" section 3, "SGLang ... (PR 21403
+analysis)" section 1.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import fp8_blockwise_w8a8_b200 as fq
+from fp8_blockwise_w8a8_b200 import inputs
+
+from helpers import dev_bf16, host_bf16_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def _weight_case(w_bits, fmt):
+    wq_ref, sw_ref = oracle.quant_weight_block(w_bits, fmt)
+    q, s = fq.quant_weight_block(dev_bf16(w_bits), fmt)
+    assert fq.check_device_error() == 0
+    q = q.cpu().numpy()
+    s = s.cpu().numpy()
+    assert np.array_equal(s.view(np.uint8) if fmt else s.view(np.uint32),
+                          sw_ref.view(np.uint8) if fmt else sw_ref.view(np.uint32))
+    assert np.array_equal(q, wq_ref)
+
+
+@pytest.mark.parametrize("fmt", [oracle.SCALE_F32, oracle.SCALE_E8M0])
+def test_weight_tiny_and_decode(fmt):
+    _weight_case(inputs.tiny_linear()["W"], fmt)
+    _weight_case(inputs.decode_linear(M=8)["W"], fmt)
+
+
+@pytest.mark.parametrize("fmt", [oracle.SCALE_F32, oracle.SCALE_E8M0])
+def test_weight_special_values(fmt):
+    rng = np.random.default_rng(5)
+    w = inputs.randn_bf16((384, 640), 0.02, 77, 0)
+    w[:128, :128] = 0                                            # all-zero block
+    w[:128, 128:256] = 0x8000                                    # all -0 block
+    w[128:256, :128] = inputs.to_bf16_bits(                      # huge magnitudes
+        rng.standard_normal((128, 128)).astype(np.float32) * np.float32(1e37))
+    w[256:384, :128] = rng.integers(1, 0x80, (128, 128)).astype(np.uint16) | \
+        (rng.integers(0, 2, (128, 128)).astype(np.uint16) << 15)  # bf16 subnormals
+    w[128:256, 128:256] = inputs.to_bf16_bits(                   # tiny block: subnormal scale
+        rng.standard_normal((128, 128)).astype(np.float32) * np.float32(1e-38))
+    w[256:384, 256:384] = 0x8001                                 # negatives that quantize to 0
+    w[256, 256] = 0x3F80                                          # ... next to a 1.0
+    # exact E4M3 midpoints relative to the block maximum 448 (x/s ties)
+    mids = np.array([432, 416 + 8, 1.0625, 2 ** -10, 3 * 2 ** -10, 17, 19], np.float32)
+    blk = np.zeros((128, 128), np.float32)
+    blk[0, 0] = 448
+    blk[1, :mids.size] = mids
+    blk[2, :mids.size] = -mids
+    w[0:128, 512:640] = inputs.to_bf16_bits(blk)
+    _weight_case(w, fmt)
+
+
+@pytest.mark.parametrize("fmt", [oracle.SCALE_F32, oracle.SCALE_E8M0])
+def test_weight_strided(fmt):
+    w = inputs.randn_bf16((256, 384), 0.05, 78, 0)
+    wd = torch.zeros((256, 520), dtype=torch.bfloat16, device="cuda")
+    wd[:, :384] = dev_bf16(w)
+    qd = torch.full((256, 400), 0xAB, dtype=torch.uint8, device="cuda")
+    q, s = fq.quant_weight_block(wd[:, :384], fmt, out_q=qd[:, :384])
+    wq_ref, sw_ref = oracle.quant_weight_block(w, fmt)
+    assert np.array_equal(qd[:, :384].cpu().numpy(), wq_ref)
+    assert (qd[:, 384:].cpu().numpy() == 0xAB).all()                # padding untouched
+    assert np.array_equal(s.cpu().numpy(), sw_ref)
+
+
+def test_weight_sweep_layer0_and_sampled_layers():
+    """Per-step requant of the 36-layer dense model: layer 0 in full, plus sampled blocks of
+    three later layers, in both scale formats (same launch configuration the bench times)."""
+    rng = np.random.default_rng(0)
+    for layer in (0, 17, 35):
+        for idx in range(len(inputs.SWEEP_MATRICES)):
+            w = inputs.sweep_matrix(layer, idx, "cuda")
+            for fmt in (oracle.SCALE_F32, oracle.SCALE_E8M0):
+                q, s = fq.quant_weight_block(w, fmt)
+                if layer == 0:
+                    wq_ref, sw_ref = oracle.quant_weight_block(host_bf16_bits(w), fmt)
+                    assert np.array_equal(s.cpu().numpy(), sw_ref)
+                    assert np.array_equal(q.cpu().numpy(), wq_ref)
+                else:
+                    N, K = w.shape
+                    for _ in range(8):
+                        nb = int(rng.integers(0, N // 128))
+                        kb = int(rng.integers(0, K // 128))
+                        blk = host_bf16_bits(w[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128])
+                        bq, bs = oracle.quant_weight_block(blk, fmt)
+                        assert s[nb, kb].item() == bs[0, 0].item()
+                        assert np.array_equal(
+                            q[nb * 128:(nb + 1) * 128, kb * 128:(kb + 1) * 128].cpu().numpy(), bq)
+    assert fq.check_device_error() == 0
+
+
+# --- token groups ------------------------------------------------------------------------------
+
+def _token_case(x_bits, gamma_bits=None, eps=1e-6, lds=None):
+    M, K = x_bits.shape
+    lds = lds if lds is not None else max(4, (M + 3) // 4 * 4)
+    q_ref, sa_ref = oracle.rmsnorm_quant_token(x_bits, gamma_bits, eps, lds=lds)
+    g = None if gamma_bits is None else dev_bf16(gamma_bits)
+    sa_dev = torch.zeros((K // 128, lds), dtype=torch.float32, device="cuda")
+    q, sa = fq.rmsnorm_quant_token(dev_bf16(x_bits), g, eps, out_sa=sa_dev)
+    assert fq.check_device_error() == 0
+    assert np.array_equal(sa.cpu().numpy()[:, :M].view(np.uint32), sa_ref[:, :M].view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("M", [1, 3, 64, 127, 129, 600])
+def test_token_plain_shapes(M):
+    x = inputs.randn_bf16((M, 512), 1.0, 90, M)
+    _token_case(x)
+
+
+def test_token_tiny_decode_and_moe_inputs():
+    _token_case(inputs.tiny_linear()["A"])
+    _token_case(inputs.decode_linear(N=128)["A"])
+    d = inputs.moe(with_weights=False)
+    _token_case(d["A_gateup"])
+    _token_case(d["A_down"])
+
+
+@pytest.mark.parametrize("K", [128, 384, 4096, 16384])
+def test_rmsnorm_shapes(K):
+    x = inputs.randn_bf16((37, K), 1.0, 91, K)
+    g = inputs.to_bf16_bits(np.random.default_rng(K).uniform(0.5, 1.5, K).astype(np.float32))
+    _token_case(x, g, 1e-6)
+    _token_case(x, None)
+
+
+def test_rmsnorm_prefill_full():
+    d = inputs.prefill_linear(with_weight=False)
+    _token_case(d["X"], d["gamma"], d["eps"])
+
+
+def test_rmsnorm_wide_dynamic_range_rows():
+    """Rows whose per-block fp64 sums of squares are inexact, so the summation order matters."""
+    rng = np.random.default_rng(92)
+    x = rng.standard_normal((16, 1024)).astype(np.float32)
+    x *= np.float32(2.0) ** rng.integers(-30, 30, size=(16, 1024)).astype(np.float32)
+    xb = inputs.to_bf16_bits(x)
+    g = inputs.to_bf16_bits(rng.uniform(0.5, 1.5, 1024).astype(np.float32))
+    _token_case(xb, g, 1e-6)
+    _token_case(xb, g, 0.0)
+
+
+def test_token_zero_rows_and_sign_of_zero():
+    x = np.zeros((4, 256), np.uint16)
+    x[1] = 0x8000
+    x[2, :128] = 0x8001
+    x[2, 5] = 0x4000
+    x[3, :] = inputs.to_bf16_bits(np.linspace(-1, 1, 256).astype(np.float32))
+    _token_case(x)
+    g = np.full(256, 0x3F80, np.uint16)
+    _token_case(x, g, 1e-6)
