@@ -19,6 +19,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _quantize(a_bits, w_bits, fmt, lds=None):
+    lds = (a_bits.shape[0] + 3) // 4 * 4 if lds is None else lds
     aq, sa = oracle.quant_token_1x128(a_bits, lds=lds)
     wq, sw = oracle.quant_weight_block(w_bits, fmt)
     return aq, sa, wq, sw
@@ -61,7 +62,7 @@ def test_identity_blocks_exact():
     """W = identity 128x128 blocks with per-block scales: out = bf16(sa * sw * dec(a))."""
     M, K = 70, 256
     a = inputs.randn_bf16((M, K), 1.0, 42, 0)
-    aq, sa = oracle.quant_token_1x128(a)
+    aq, sa = oracle.quant_token_1x128(a, lds=72)
     wq = np.zeros((K, K), np.uint8)
     wq[np.arange(K), np.arange(K)] = 0x38
     sw = np.array([[0.5, 1e9], [1e9, 0.25]], np.float32)
