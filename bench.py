@@ -65,7 +65,7 @@ class ClockSampler:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.bus, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -132,23 +132,30 @@ class LinearStep:
             ev[3].record()
 
 
+def hold_gpu():
+    """Keep the GPU busy for ~25 ms so that the host can enqueue a timed batch ahead of it; the
+    events then time device work only, never host launch overhead."""
+    torch.cuda._sleep(50_000_000)
+
+
 def timed_loop(fn, steps, warmup, flush=None):
-    """Mean device time (ms) of fn over `steps` calls after `warmup`, events on the current
-    stream; `flush` (if given) runs between calls, outside the timed spans."""
+    """Mean device time (ms) of fn over `steps` calls after `warmup`, with an event pair around
+    each call on the current stream; `flush` (if given) runs between calls, outside the timed
+    spans.  All calls are enqueued behind hold_gpu() and synchronized once at the end."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
-    times = []
-    for _ in range(steps):
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    hold_gpu()
+    for a, b in ev:
         if flush is not None:
             flush()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
         a.record()
         fn()
         b.record()
-        b.synchronize()
-        times.append(a.elapsed_time(b))
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in ev]
     return statistics.mean(times), times
 
 
@@ -305,6 +312,7 @@ def run_ours(args):
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
+    hold_gpu()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record()
@@ -454,14 +462,74 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_ncu_case(name):
+    """A few launches of one kernel on a case sized for an Nsight Compute capture (inputs larger
+    than L2, a few hundred MB on the device): 2 warm-up launches, then 3 more."""
+    import fp8_blockwise_w8a8_b200 as fq
+    from fp8_blockwise_w8a8_b200 import inputs
+    fq._lib.lib()
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+
+    def randn(shape, std):
+        return (torch.randn(shape, generator=g, device=dev) * std).to(torch.bfloat16)
+    if name == "gemm_prefill":           # M=4096 of the prefill GEMM: A 16 MB, W 100 MB, out 201 MB
+        aq, sa = fq.rmsnorm_quant_token(randn((4096, K_), 1.0))
+        wq, sw = fq.quant_weight_block(randn((N_, K_), 0.02), "f32")
+        out = torch.empty((4096, N_), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm_w8a8_block(aq, sa, wq, sw, out=out)
+    elif name == "gemm_decode":
+        aq, sa = fq.rmsnorm_quant_token(randn((128, K_), 1.0))
+        wq, sw = fq.quant_weight_block(randn((12288, K_), 0.02), "f32")
+        out = torch.empty((128, 12288), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm_w8a8_block(aq, sa, wq, sw, out=out)
+    elif name == "rmsnorm_prefill":      # X [8192, 4096]: 67 MB in, 35 MB out
+        x = randn((M_, K_), 1.0)
+        gam = randn((K_,), 0.5) + 1.0
+        fn = lambda: fq.rmsnorm_quant_token(x, gam, 1e-6)
+    elif name == "token_prefill":        # plain 1x128 token quant of X [8192, 4096]
+        x = randn((M_, K_), 1.0)
+        fn = lambda: fq.rmsnorm_quant_token(x)
+    elif name == "requant_prefill":      # W [24576, 4096]: 201 MB in, 101 MB out
+        w = randn((N_, K_), 0.02)
+        fn = lambda: fq.quant_weight_block(w, "f32")
+    elif name == "requant_prefill_e8m0":
+        w = randn((N_, K_), 0.02)
+        fn = lambda: fq.quant_weight_block(w, "e8m0")
+    elif name == "grouped_gateup":
+        tok, off = inputs.moe_routing()
+        R = int(off[-1])
+        aq, sa = fq.rmsnorm_quant_token(randn((R, 2048), 1.0))
+        wq, sw = fq.quant_weight_block(randn((128 * 1536, 2048), 0.02), "f32")
+        offd = torch.from_numpy(off).to(dev)
+        out = torch.empty((R, 1536), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.grouped_gemm_w8a8_block(aq, sa, wq.view(128, 1536, 2048),
+                                                sw.view(128, 12, 16), offd, out=out)
+    else:
+        raise SystemExit(f"unknown --ncu-case {name}")
+    torch.cuda.synchronize()
+    for _ in range(5):
+        fn()
+    torch.cuda.synchronize()
+    if fq.check_device_error() != 0:
+        raise SystemExit("device error")
+    print(f"ncu case {name}: ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", dest="rows", action="store_false")
+    ap.add_argument("--ncu-case", default=None,
+                    help="run a few launches of one kernel on a small case (for ncu) and exit")
     args = ap.parse_args()
+    if args.ncu_case:
+        run_ncu_case(args.ncu_case)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":

@@ -104,7 +104,7 @@ int check_gemm_common(const void *aq, int64_t lda, const float *sa, int64_t lds,
                       const void *out, int64_t ldo) {
   if (sw_fmt != FP8Q_SCALE_F32 && sw_fmt != FP8Q_SCALE_E8M0) return FP8Q_ERR_ARG;
   if (M < 0 || N <= 0 || K <= 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
-  if (M > INT32_MAX - 256 || N > (1 << 30) || K > (1 << 30)) return FP8Q_ERR_SHAPE;
+  if (M > INT32_MAX - 256 || N > (1 << 30) || K > 128 * fp8q::kMaxKB) return FP8Q_ERR_SHAPE;
   if (lda < K || ldw < K || ldo < N || lds < M) return FP8Q_ERR_SHAPE;
   if (M == 0) return FP8Q_OK;
   if (!aq || !sa || !wq || !sw || !out) return FP8Q_ERR_NULL;
@@ -215,22 +215,30 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   const bool norm = gamma_bf16 != nullptr;
   const int KB = static_cast<int>(K / 128);
   const int row_bytes = KB * fp8q::kRowBlockStride;
-  const int gamma_bytes = norm ? row_bytes : 0;
+  const int gamma_bytes = norm ? static_cast<int>(K) * 4 : 0;
   const int budget = 227 * 1024;
-  int wpc = (budget - gamma_bytes) / (2 * row_bytes);
-  if (wpc > 4) wpc = 4;
-  if (wpc < 1) return FP8Q_ERR_SHAPE;
-  const int smem = gamma_bytes + wpc * 2 * row_bytes;
-  int per_sm = 1;
-  if (norm)
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_rmsnorm_quant_token<true>,
-                                                  32 * wpc, smem);
-  else
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_rmsnorm_quant_token<false>,
-                                                  32 * wpc, smem);
-  if (per_sm < 1) per_sm = 1;
+  // Warps per CTA: the choice that keeps the most warps resident per SM.
+  int best_wpc = 0, best_ctas = 0, best_smem = 0;
+  for (int wpc : {16, 12, 8, 4, 2, 1}) {
+    const int smem = norm ? gamma_bytes + wpc * row_bytes : 0;
+    if (smem > budget) continue;
+    int per_sm = 0;
+    if (norm)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_rmsnorm_quant_token<true>,
+                                                    32 * wpc, smem);
+    else
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_rmsnorm_quant_token<false>,
+                                                    32 * wpc, smem);
+    if (per_sm * wpc > best_ctas * best_wpc) {
+      best_wpc = wpc;
+      best_ctas = per_sm;
+      best_smem = smem;
+    }
+  }
+  if (best_wpc == 0) return FP8Q_ERR_SHAPE;
+  const int wpc = best_wpc, smem = best_smem;
   const int64_t need = (M + wpc - 1) / wpc;
-  const int64_t cap = static_cast<int64_t>(st->sms) * per_sm;
+  const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
   const int grid = static_cast<int>(need < cap ? need : cap);
   const auto *x = static_cast<const uint16_t *>(x_bf16);
   const auto *g = static_cast<const uint16_t *>(gamma_bf16);

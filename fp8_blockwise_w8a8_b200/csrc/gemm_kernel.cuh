@@ -12,11 +12,14 @@
 //   warp 1      TMEM allocator (whole warp) and MMA issuer (lane 0): 4 MMAs (K = 32 each) per
 //               K-block into one of two 256-column TMEM buffers, so the MMAs of K-block kb + 1
 //               run while the epilogue promotes K-block kb
-//   warps 2-3   idle (they complete warpgroup 0 for the register hand-off)
+//   warp 2      scale producer: streams the activation scales sa of each K-block into a shared
+//               ring with cp.async (8 K-blocks ahead) and stages the weight scales of each tile
+//   warp 3      idle (it completes warpgroup 0 for the register hand-off)
 //   warps 4-11  epilogue/promotion: warp w reads TMEM lanes 32 * (w % 4) (its 32 rows of the
 //               tile) and column half (w - 4) / 4; each thread keeps 128 fp32 accumulators
-// Registers: launched at 168 per thread (384 x 168 = 64512); warpgroup 0 drops to 40 and the two
-// epilogue warpgroups rise to 232 (128 x 40 + 256 x 232 = 64512, per sub-partition 16128).
+// Registers: launched at 168 per thread (384 x 168 = 64512); warpgroup 0 drops to 64 and the two
+// epilogue warpgroups rise to 216 (128 x 64 + 256 x 216 = 63488 <= 64512; per sub-partition
+// 64 x 32 + 2 x 216 x 32 = 15872 <= 16128).
 // Every wait is bounded: on expiry a kernel records FP8Q_ERR_TIMEOUT in the device error word,
 // all roles leave their loops, in-flight copies and MMAs are drained, and TMEM is released.
 #pragma once
@@ -28,7 +31,7 @@ namespace fp8q {
 constexpr int kBM = 128, kBN = 256, kBK = 128;
 constexpr int kStages = 4;
 constexpr int kGemmThreads = 384;
-constexpr int kProducerRegs = 40, kEpilogueRegs = 232;
+constexpr int kProducerRegs = 64, kEpilogueRegs = 216;
 constexpr int kTileABytes = kBM * kBK;            // 16 KB
 constexpr int kTileBBytes = kBN * kBK;            // 32 KB
 constexpr int kStageBytes = kTileABytes + kTileBBytes;
@@ -41,8 +44,13 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kTileABytes;
 constexpr int kOffStaging = kOffB + kStages * kTileBBytes;
-constexpr int kOffBar = kOffStaging + 8 * kStagingBytesPerWarp;
-constexpr int kNumBars = 2 * kStages + 4 + 1;     // full, empty, tmem_full[2], tmem_empty[2], done
+constexpr int kSaStages = 8;                      // K-blocks of activation scales in flight
+constexpr int kMaxKB = 256;                       // K <= 32768
+constexpr int kOffSa = kOffStaging + 8 * kStagingBytesPerWarp;      // [kSaStages][128] fp32
+constexpr int kOffSw = kOffSa + kSaStages * kBM * 4;                // [2 tiles][2 halves][kMaxKB]
+constexpr int kOffBar = kOffSw + 2 * 2 * kMaxKB * 4;
+// full, empty, tmem_full[2], tmem_empty[2], done, sa_full/empty[kSaStages], sw_full/empty[2]
+constexpr int kNumBars = 2 * kStages + 4 + 1 + 2 * kSaStages + 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
 constexpr int kOffGroups = kOffMisc + 16;          // grouped: offsets[E+1], tile prefix[E+1]
 constexpr int kGemmSmemDense = kOffGroups + 1024;  // + alignment slack
@@ -180,6 +188,23 @@ __device__ __forceinline__ float load_sw(const GemmArgs &a, const uint8_t *sw_ro
   return b >= 1 ? __uint_as_float(static_cast<uint32_t>(b) << 23) : __uint_as_float(0x00400000u);
 }
 
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void *src,
+                                                  uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed (no count increment).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 template <bool GROUPED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm_w8a8_block(const __grid_constant__ CUtensorMap tm_a,
@@ -194,6 +219,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t bar_tfull = bar_empty + 8 * kStages;     // [2]
   const uint32_t bar_tempty = bar_tfull + 16;             // [2]
   const uint32_t bar_done = bar_tempty + 16;
+  const uint32_t bar_safull = bar_done + 8;                   // [kSaStages]
+  const uint32_t bar_saempty = bar_safull + 8 * kSaStages;    // [kSaStages]
+  const uint32_t bar_swfull = bar_saempty + 8 * kSaStages;    // [2]
+  const uint32_t bar_swempty = bar_swfull + 16;               // [2]
+  float *s_sa = reinterpret_cast<float *>(smem + kOffSa);
+  float *s_sw = reinterpret_cast<float *>(smem + kOffSw);
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + kOffMisc);
   volatile int *s_abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
   int *s_off = reinterpret_cast<int *>(smem + kOffGroups);
@@ -211,6 +242,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(bar_tempty + 8 * i, 8);
     }
     mbar_init(bar_done, 1);
+    for (int i = 0; i < kSaStages; ++i) {
+      mbar_init(bar_safull + 8 * i, 32);
+      mbar_init(bar_saempty + 8 * i, 8);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_swfull + 8 * i, 32);
+      mbar_init(bar_swempty + 8 * i, 8);
+    }
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -273,6 +312,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       }
       __syncwarp();
+    } else if (warp == 2) {
+      // ---------------------------------------------------------------- scale producer
+      const int NB = args.N / 128;
+      const size_t sw_elem = args.sw_fmt == 0 ? 4 : 1;
+      uint32_t it = 0, tile_it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tile_it) {
+        const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, t) : dense_tile(args, t);
+        // weight scales of the tile's two 128-column halves, all K-blocks, as fp32
+        const uint32_t tp = tile_it & 1u;
+        if (!wait_warp(bar_swempty + 8 * tp, ((tile_it >> 1) & 1u) ^ 1u, s_abort)) break;
+        for (int j = lane; j < 2 * KB; j += 32) {
+          const int hh = j >= KB ? 1 : 0, kb = j - hh * KB;
+          const int nb = tl.n0 / 128 + hh;
+          float v = 0.0f;
+          if (nb < NB) {
+            const uint8_t *row = static_cast<const uint8_t *>(args.sw) +
+                                 (static_cast<size_t>(tl.e) * NB + nb) * KB * sw_elem;
+            v = load_sw(args, row, kb);
+          }
+          s_sw[(tp * 2 + hh) * kMaxKB + kb] = v;
+        }
+        mbar_arrive(bar_swfull + 8 * tp);
+        // activation scales: one 128-row column of sa per K-block, zero-filled past row_end
+        const int rows_here = tl.row_end - tl.m0;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const uint32_t s2 = it % kSaStages, ph2 = (it / kSaStages) & 1u;
+          if (!wait_warp(bar_saempty + 8 * s2, ph2 ^ 1u, s_abort)) { ok = false; break; }
+          const float *src = args.sa + static_cast<int64_t>(kb) * args.lds + tl.m0 + 4 * lane;
+          const uint32_t dst = smem_u32(s_sa + s2 * kBM + 4 * lane);
+          const int valid = max(0, min(4, rows_here - 4 * lane));
+          if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+            cp_async_16_zfill(dst, valid > 0 ? src : args.sa, 4u * valid);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              cp_async_4(dst + 4 * i, i < valid ? src + i : args.sa, i < valid ? 4u : 0u);
+          }
+          cp_async_arrive_noinc(bar_safull + 8 * s2);
+        }
+      }
+      cp_async_wait_all();
+      __syncwarp();
     } else if (warp == 1) {
       // ------------------------------------------------------------------ MMA issuer
       if (lane == 0) {
@@ -310,53 +392,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int NB = args.N / 128;
     uint8_t *stage = smem + kOffStaging + (warp - 4) * kStagingBytesPerWarp;
     const uint32_t stage_u32 = smem_u32(stage);
-    const size_t sw_elem = args.sw_fmt == 0 ? 4 : 1;
-    uint32_t it = 0;
+    uint32_t it = 0, tile_it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tile_it) {
       const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, t) : dense_tile(args, t);
-      const int row = tl.m0 + 32 * q + lane;
-      const bool row_ok = row < tl.row_end;
       const int nbh = tl.n0 / 128 + h;
       const bool col_ok = nbh < NB;
-      const uint8_t *sw_row = static_cast<const uint8_t *>(args.sw) +
-                              (static_cast<size_t>(tl.e) * NB + (col_ok ? nbh : 0)) * KB * sw_elem;
-      const float *sa_col = args.sa + row;
-      // scales for K-blocks kb and kb + 1 are loaded ahead of use
-      float sa0 = (row_ok) ? __ldg(sa_col) : 0.0f;
-      float sa1 = (row_ok && KB > 1) ? __ldg(sa_col + args.lds) : 0.0f;
-      float sw0 = col_ok ? load_sw(args, sw_row, 0) : 0.0f;
-      float sw1 = (col_ok && KB > 1) ? load_sw(args, sw_row, 1) : 0.0f;
-      float acc[128];
+      const uint32_t tp = tile_it & 1u;
+      if (!wait_warp(bar_swfull + 8 * tp, (tile_it >> 1) & 1u, s_abort)) { ok = false; break; }
+      const float *sw_tile = s_sw + (tp * 2 + h) * kMaxKB;
+      float2 acc[64];  // columns 2j, 2j + 1 of this thread's row
 #pragma unroll
-      for (int j = 0; j < 128; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
       for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t s2 = it % kSaStages, ph2 = (it / kSaStages) & 1u;
+        if (!wait_warp(bar_safull + 8 * s2, ph2, s_abort)) { ok = false; break; }
+        const float sc = __fmul_rn(s_sa[s2 * kBM + 32 * q + lane], sw_tile[kb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_saempty + 8 * s2);
         const uint32_t b = it & 1u, bph = (it >> 1) & 1u;
         if (!wait_warp(bar_tfull + 8 * b, bph, s_abort)) { ok = false; break; }
         tc_fence_after();
-        const float sc = __fmul_rn(sa0, sw0);
+        const float2 sc2 = make_float2(sc, sc);
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * kBN + h * 128;
+        // Two 64-column chunks: load, wait, promote.  The buffer is handed back to the MMA as
+        // soon as the second chunk is in registers.
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + 32 * c, r);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[64];
+          tmem_ld_32x32b_x64(taddr + 64 * c, r);
           tmem_ld_wait(r);
-          if (c == 3) {
+          if (c == 1) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
           }
 #pragma unroll
-          for (int j = 0; j < 32; ++j) acc[32 * c + j] = fmaf(__uint_as_float(r[j]), sc, acc[32 * c + j]);
-        }
-        sa0 = sa1;
-        sw0 = sw1;
-        if (kb + 2 < KB) {
-          sa1 = row_ok ? __ldg(sa_col + static_cast<int64_t>(kb + 2) * args.lds) : 0.0f;
-          sw1 = col_ok ? load_sw(args, sw_row, kb + 2) : 0.0f;
+          for (int j = 0; j < 32; ++j)
+            acc[32 * c + j] = __ffma2_rn(make_float2(__uint_as_float(r[2 * j]),
+                                                     __uint_as_float(r[2 * j + 1])),
+                                         sc2, acc[32 * c + j]);
         }
       }
       if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_swempty + 8 * tp);
       // bf16 conversion and store, 32 columns at a time through a swizzled staging buffer so
       // that each global store instruction writes 64-byte row segments.
       uint16_t *out_base = args.out + static_cast<int64_t>(tl.n0 + 128 * h);
@@ -367,8 +447,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint32_t pk[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const __nv_bfloat162 v2 =
-                __floats2bfloat162_rn(acc[32 * c4 + 8 * j + 2 * u], acc[32 * c4 + 8 * j + 2 * u + 1]);
+            const float2 a2 = acc[16 * c4 + 4 * j + u];
+            const __nv_bfloat162 v2 = __floats2bfloat162_rn(a2.x, a2.y);
             pk[u] = *reinterpret_cast<const uint32_t *>(&v2);
           }
           const int phys = j ^ ((lane >> 1) & 3);

@@ -22,8 +22,21 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
   return v;
 }
 
-__device__ __forceinline__ float amax_word(float m, uint32_t w) {
-  return fmaxf(m, fmaxf(fabsf(bf16_lo(w)), fabsf(bf16_hi(w))));
+// Running maximum of |x| over packed bf16 pairs: max.xorsign.abs compares magnitudes, so the
+// magnitude bits of the result are max(|a|, |b|) per half (the sign bit is not used).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Both halves of an absmax_bf16x2 accumulator reduced to one fp32 magnitude.
+__device__ __forceinline__ float absmax_finish(uint32_t m) {
+  return fmaxf(bf16_lo(m & 0x7FFF7FFFu), bf16_hi(m & 0x7FFF7FFFu));
+}
+
+__device__ __forceinline__ uint32_t absmax_uint4(uint32_t m, const uint4 &v) {
+  return absmax_bf16x2(absmax_bf16x2(m, v.x), absmax_bf16x2(absmax_bf16x2(v.y, v.z), v.w));
 }
 
 // Exponent e of the E8M0 scale for a block maximum: the smallest e with 2^e >= fp32(amax/448),
@@ -45,56 +58,79 @@ __device__ __forceinline__ float pow2_f32(int e) {
                    : __uint_as_float(0x00400000u);
 }
 
-// Per-block quantization parameters.  mode 0: codes = cvt(x * inv) exactly (power-of-two
-// scale); mode 1: fast path x * rcp with a bracket check, exact division when the bracket
-// straddles a rounding boundary; mode 2: exact division for every element.
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Per-block parameters of the fp32-scale quantizer.
+//   fast = true : bracket fast path (see quant8_f32), exact division when it is ambiguous.
+//   fast = false: exact IEEE division for every element (tiny scales, where 1/s would overflow).
 struct QParams {
-  float s;     // the scale (divisor)
-  float mul;   // 1/s: exact for powers of two, RN(1/s) otherwise
-  int mode;
+  float s;       // the scale (divisor)
+  float2 lo2;    // RN(r * (1 - 2^-19)) in both lanes, r ~ 1/s
+  float2 hi2;    // RN(r * (1 + 2^-19)) in both lanes
+  bool fast;
 };
 
 __device__ __forceinline__ QParams qparams_f32(float amax) {
   QParams p;
   p.s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-  p.mul = __fdiv_rn(1.0f, p.s);
-  // The bracket argument needs 1/s finite and products far from the subnormal range.
-  p.mode = (p.s >= 0x1.0p-100f) ? 1 : 2;
+  p.fast = p.s >= 0x1.0p-100f;
+  // r approximates 1/s within one ulp (2^-23 relative, the documented bound of rcp.approx).
+  const float r = rcp_approx(p.fast ? p.s : 1.0f);
+  const float lo = __fmul_rn(r, 0x1.ffffc0p-1f), hi = __fmul_rn(r, 0x1.000020p+0f);
+  p.lo2 = make_float2(lo, lo);
+  p.hi2 = make_float2(hi, hi);
   return p;
 }
 
-__device__ __forceinline__ QParams qparams_pow2(int e) {
-  QParams p;
-  p.s = pow2_f32(e);
-  p.mul = pow2_f32(-e);  // exact: x * 2^-e == x / 2^e, each rounded once
-  p.mode = 0;
-  return p;
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
+  return make_float2(bf16_lo(w), bf16_hi(w));
 }
 
-// Two E4M3 codes for RN_fp32(x0 / s), RN_fp32(x1 / s) (low byte = x0).
+// Eight E4M3 codes of RN_fp32(x / s) for the eight bf16 values of one uint4 (byte i = element i).
 //
-// Fast path: t = RN(x * RN(1/s)) is within (1 + 2^-24)^2 of x/s; t * (1 -+ 2^-20) (rounded)
-// then bracket x/s strictly, and RN_fp32 and the E4M3 conversion are both monotone, so when
-// both bracket ends give the same code that code is the exact one.  Otherwise (x/s within about
-// 2^-20 of an E4M3 rounding boundary) the pair is redone with IEEE divisions.
-__device__ __forceinline__ uint16_t quant_pair(float x0, float x1, const QParams &p) {
-  if (p.mode == 0) return cvt_e4m3x2(__fmul_rn(x0, p.mul), __fmul_rn(x1, p.mul));
-  if (p.mode == 1) {
-    const float t0 = __fmul_rn(x0, p.mul), t1 = __fmul_rn(x1, p.mul);
-    const uint16_t lo = cvt_e4m3x2(__fmul_rn(t0, 0x1.ffffe0p-1f), __fmul_rn(t1, 0x1.ffffe0p-1f));
-    const uint16_t hi = cvt_e4m3x2(__fmul_rn(t0, 0x1.000010p+0f), __fmul_rn(t1, 0x1.000010p+0f));
-    if (lo == hi) return lo;
+// Bracket: with r = 1/s (1 + e_r), |e_r| <= 2^-23, the rounded products x * RN(r (1 -+ 2^-19))
+// are within a relative 2^-23 + 3 * 2^-24 of x/s (1 -+ 2^-19), so they bracket x/s strictly.
+// RN_fp32 and the E4M3 conversion are both monotone, hence when the two bracket ends give the
+// same code, that code is the code of RN_fp32(x/s).  Otherwise (some x/s within ~2^-19 of an
+// E4M3 rounding boundary, exact ties included) the eight values are redone with IEEE divisions.
+__device__ __forceinline__ uint2 quant8_f32(const uint4 v, const QParams &p) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  if (p.fast) {
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 x = unpack_bf16x2(w[j]);
+      const float2 a = __fmul2_rn(x, p.lo2), b = __fmul2_rn(x, p.hi2);
+      lo[j] = cvt_e4m3x2(a.x, a.y);
+      hi[j] = cvt_e4m3x2(b.x, b.y);
+    }
+    const uint32_t l0 = lo[0] | (lo[1] << 16), l1 = lo[2] | (lo[3] << 16);
+    const uint32_t h0 = hi[0] | (hi[1] << 16), h1 = hi[2] | (hi[3] << 16);
+    if (((l0 ^ h0) | (l1 ^ h1)) == 0u) return make_uint2(l0, l1);
   }
-  return cvt_e4m3x2(__fdiv_rn(x0, p.s), __fdiv_rn(x1, p.s));
+  uint32_t c[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 x = unpack_bf16x2(w[j]);
+    c[j] = cvt_e4m3x2(__fdiv_rn(x.x, p.s), __fdiv_rn(x.y, p.s));
+  }
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
-// 8 bf16 values (one uint4) -> 8 codes (one uint2).
-__device__ __forceinline__ uint2 quant8_bf16(const uint4 v, const QParams &p) {
-  const uint32_t c0 = quant_pair(bf16_lo(v.x), bf16_hi(v.x), p);
-  const uint32_t c1 = quant_pair(bf16_lo(v.y), bf16_hi(v.y), p);
-  const uint32_t c2 = quant_pair(bf16_lo(v.z), bf16_hi(v.z), p);
-  const uint32_t c3 = quant_pair(bf16_lo(v.w), bf16_hi(v.w), p);
-  return make_uint2(c0 | (c1 << 16), c2 | (c3 << 16));
+// Eight codes for a power-of-two scale 2^e: x * 2^-e is exact (inv2 = {2^-e, 2^-e}).
+__device__ __forceinline__ uint2 quant8_pow2(const uint4 v, const float2 inv2) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 t = __fmul2_rn(unpack_bf16x2(w[j]), inv2);
+    c[j] = cvt_e4m3x2(t.x, t.y);
+  }
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -103,7 +139,7 @@ __device__ __forceinline__ uint2 quant8_bf16(const uint4 v, const QParams &p) {
 // warp covers two full 256-byte (load) / 128-byte (store) row segments.
 // ---------------------------------------------------------------------------------------------
 template <int FMT>
-__global__ void __launch_bounds__(256) k_quant_weight_block(const uint16_t *__restrict__ w,
+__global__ void __launch_bounds__(256, 4) k_quant_weight_block(const uint16_t *__restrict__ w,
                                                             int64_t ldw, uint8_t *__restrict__ q,
                                                             int64_t ldq, void *__restrict__ sw,
                                                             int KB, int64_t nblocks) {
@@ -117,14 +153,10 @@ __global__ void __launch_bounds__(256) k_quant_weight_block(const uint16_t *__re
     uint4 v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = ld_stream_v4(src + static_cast<int64_t>(i) * 16 * ldw);
-    float amax = 0.0f;
+    uint32_t m2 = 0u;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      amax = amax_word(amax, v[i].x);
-      amax = amax_word(amax, v[i].y);
-      amax = amax_word(amax, v[i].z);
-      amax = amax_word(amax, v[i].w);
-    }
+    for (int i = 0; i < 8; ++i) m2 = absmax_uint4(m2, v[i]);
+    float amax = absmax_finish(m2);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if (lane == 0) red[warp] = amax;
@@ -133,50 +165,72 @@ __global__ void __launch_bounds__(256) k_quant_weight_block(const uint16_t *__re
 #pragma unroll
     for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
     __syncthreads();  // red[] is rewritten by the next block
-    QParams p;
+    uint8_t *dst = q + (nb * 128 + r0) * ldq + kb * 128 + c8;
     if (FMT == kScaleF32) {
-      p = qparams_f32(amax);
+      const QParams p = qparams_f32(amax);
       if (tid == 0) static_cast<float *>(sw)[blk] = p.s;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<uint2 *>(dst + static_cast<int64_t>(i) * 16 * ldq) = quant8_f32(v[i], p);
     } else {
       const int e = e8m0_exponent(amax);
-      p = qparams_pow2(e);
       if (tid == 0) static_cast<uint8_t *>(sw)[blk] = static_cast<uint8_t>(e + 127);
-    }
-    uint8_t *dst = q + (nb * 128 + r0) * ldq + kb * 128 + c8;
+      const float inv = pow2_f32(-e);
+      const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      *reinterpret_cast<uint2 *>(dst + static_cast<int64_t>(i) * 16 * ldq) = quant8_bf16(v[i], p);
+      for (int i = 0; i < 8; ++i)
+        *reinterpret_cast<uint2 *>(dst + static_cast<int64_t>(i) * 16 * ldq) = quant8_pow2(v[i], inv2);
+    }
   }
 }
 
 // ---------------------------------------------------------------------------------------------
-// 1x128 token groups, optionally preceded by RMSNorm.  One warp per row at a time; rows are
-// double-buffered in shared memory with cp.async so the next row streams in while the current
-// one is processed.  Shared layout of a row: 128-element blocks at a 272-byte stride (256 bytes
-// of data + 16 bytes of padding), so that lane b reading its own block b sequentially (the RMS
-// sum of squares) hits distinct banks.  gamma uses the same layout, once per CTA.
+// 1x128 token groups, optionally preceded by RMSNorm.  One warp per row at a time.
+//
+// With RMSNorm the row is staged in shared memory (cp.async) in a padded layout -- 128-element
+// blocks at a 272-byte stride -- so that lane b can walk its own block b in ascending k for the
+// fp64 sum of squares without bank conflicts.  gamma is held once per CTA as fp32.  Without
+// RMSNorm nothing is staged: each step reads the row straight from global memory.  In both
+// cases the next row of the warp is prefetched into L2 while the current one is processed.
+//
+// Quantization step: lanes 0-15 take block 2j, lanes 16-31 block 2j + 1, each lane 8 elements.
 // ---------------------------------------------------------------------------------------------
 constexpr int kRowBlockStride = 272;
 
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
-__device__ __forceinline__ void cp_async_wait_1() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-__device__ __forceinline__ void load_row_async(uint32_t dst, const uint16_t *src, int K,
-                                               int lane) {
-  const int chunks = K >> 3;  // 16-byte chunks
-  for (int j = lane; j < chunks; j += 32)
-    cp_async_16(dst + (j >> 4) * kRowBlockStride + (j & 15) * 16, src + j * 8);
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+// y = bf16( (x * r) * gamma ), two fp32 roundings, for the 8 elements of one uint4; ga and gb
+// hold gamma of those elements as fp32.
+__device__ __forceinline__ uint4 rms_apply8(const uint4 v, float r, const float4 ga,
+                                            const float4 gb) {
+  const float2 r2 = make_float2(r, r);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const float2 gg[4] = {make_float2(ga.x, ga.y), make_float2(ga.z, ga.w), make_float2(gb.x, gb.y),
+                        make_float2(gb.z, gb.w)};
+  uint32_t y[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 u = __fmul2_rn(__fmul2_rn(unpack_bf16x2(w[j]), r2), gg[j]);
+    y[j] = pack_bf16x2(u.x, u.y);
+  }
+  return make_uint4(y[0], y[1], y[2], y[3]);
 }
 
 template <bool NORM>
-__global__ void __launch_bounds__(128) k_rmsnorm_quant_token(
+__global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
     int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ sa, int64_t lds) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -184,34 +238,38 @@ __global__ void __launch_bounds__(128) k_rmsnorm_quant_token(
   const int wpc = blockDim.x >> 5;
   const int KB = K >> 7;
   const int row_bytes = KB * kRowBlockStride;
-  uint8_t *g_s = smem;                                     // gamma (NORM only)
-  uint8_t *buf0 = smem + (NORM ? row_bytes : 0) + warp * 2 * row_bytes;
-  const uint32_t buf_u32[2] = {smem_u32(buf0), smem_u32(buf0 + row_bytes)};
+  // gamma as fp32, split per 16-byte chunk j of the row into gA[j] (elements 8j..8j+3) and
+  // gB[j] (8j+4..8j+7), so that eight lanes reading eight consecutive chunks hit distinct banks.
+  float4 *gA = reinterpret_cast<float4 *>(smem);
+  float4 *gB = gA + (K >> 3);
+  uint8_t *row = smem + (NORM ? K * 4 : 0) + warp * row_bytes;
+  const uint32_t row_u32 = smem_u32(row);
+  const int grp = lane >> 3, sub = lane & 7;   // 8 lanes per 128-block, 4 blocks per step
 
   if (NORM) {
-    const int chunks = K >> 3;
-    for (int j = threadIdx.x; j < chunks; j += blockDim.x)
-      *reinterpret_cast<uint4 *>(g_s + (j >> 4) * kRowBlockStride + (j & 15) * 16) =
-          *reinterpret_cast<const uint4 *>(gamma + j * 8);
+    for (int j = threadIdx.x; j < (K >> 3); j += blockDim.x) {
+      const uint4 g = *reinterpret_cast<const uint4 *>(gamma + j * 8);
+      gA[j] = make_float4(bf16_lo(g.x), bf16_hi(g.x), bf16_lo(g.y), bf16_hi(g.y));
+      gB[j] = make_float4(bf16_lo(g.z), bf16_hi(g.z), bf16_lo(g.w), bf16_hi(g.w));
+    }
     __syncthreads();
   }
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
-  int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp;
-  if (m < M) load_row_async(buf_u32[0], x + m * ldx, K, lane);
-  cp_async_commit();
-  const int half = lane >> 4, hl = lane & 15;
-  for (int it = 0; m < M; m += stride, ++it) {
-    const int cur = it & 1;
+  for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < M; m += stride) {
+    const uint16_t *xr = x + m * ldx;
     const int64_t next = m + stride;
-    if (next < M) load_row_async(buf_u32[cur ^ 1], x + next * ldx, K, lane);
-    cp_async_commit();
-    cp_async_wait_1();
-    __syncwarp();
-    const uint8_t *row = cur ? buf0 + row_bytes : buf0;
+    if (next < M) {
+      const char *nr = reinterpret_cast<const char *>(x + next * ldx);
+      for (int off = lane * 128; off < K * 2; off += 32 * 128) prefetch_l2(nr + off);
+    }
 
     float r = 1.0f;
     if (NORM) {
+      for (int j = lane; j < (K >> 3); j += 32)
+        cp_async_16(row_u32 + (j >> 4) * kRowBlockStride + (j & 15) * 16, xr + j * 8);
+      cp_async_commit_wait_all();
+      __syncwarp();
       // Sum of squares in fp64: each lane walks its own 128-blocks in ascending k ...
       double P[4];
 #pragma unroll
@@ -241,6 +299,7 @@ __global__ void __launch_bounds__(128) k_rmsnorm_quant_token(
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (32 * i >= KB) break;
+#pragma unroll 8
         for (int j = 0; j < 32; ++j) {
           const double pj = __shfl_sync(0xffffffffu, P[i], j);
           if (32 * i + j < KB) S = __dadd_rn(S, pj);
@@ -250,42 +309,38 @@ __global__ void __launch_bounds__(128) k_rmsnorm_quant_token(
       r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(var)));
     }
 
-    // Quantize two 128-blocks per step: lanes 0-15 take block 2j, lanes 16-31 block 2j + 1;
-    // each lane owns 8 consecutive elements.
-    for (int b0 = 0; b0 < KB; b0 += 2) {
-      const int b = b0 + half;
+    // Quantize: lanes 8g .. 8g+7 take block b0 + g; lane `sub` owns 16-byte chunks sub and
+    // sub + 8 of the block (elements 8 sub .. 8 sub + 7 and 64 + 8 sub .. 64 + 8 sub + 7).
+#pragma unroll 2
+    for (int b0 = 0; b0 < KB; b0 += 4) {
+      const int b = b0 + grp;
       const bool active = b < KB;
       const int bb = active ? b : b0;
-      uint4 v = *reinterpret_cast<const uint4 *>(row + bb * kRowBlockStride + hl * 16);
+      uint4 v0, v1;
       if (NORM) {
-        const uint4 g = *reinterpret_cast<const uint4 *>(g_s + bb * kRowBlockStride + hl * 16);
-        const uint32_t xv[4] = {v.x, v.y, v.z, v.w};
-        const uint32_t gv[4] = {g.x, g.y, g.z, g.w};
-        uint32_t yv[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float y0 = __fmul_rn(__fmul_rn(bf16_lo(xv[j]), r), bf16_lo(gv[j]));
-          const float y1 = __fmul_rn(__fmul_rn(bf16_hi(xv[j]), r), bf16_hi(gv[j]));
-          const __nv_bfloat162 yy = __floats2bfloat162_rn(y0, y1);
-          yv[j] = *reinterpret_cast<const uint32_t *>(&yy);
-        }
-        v = make_uint4(yv[0], yv[1], yv[2], yv[3]);
+        const uint8_t *rb = row + bb * kRowBlockStride;
+        v0 = *reinterpret_cast<const uint4 *>(rb + sub * 16);
+        v1 = *reinterpret_cast<const uint4 *>(rb + (sub + 8) * 16);
+        const int j0 = bb * 16 + sub, j1 = j0 + 8;
+        v0 = rms_apply8(v0, r, gA[j0], gB[j0]);
+        v1 = rms_apply8(v1, r, gA[j1], gB[j1]);
+      } else {
+        v0 = ld_stream_v4(xr + bb * 128 + sub * 8);
+        v1 = ld_stream_v4(xr + bb * 128 + 64 + sub * 8);
       }
-      float amax = 0.0f;
-      amax = amax_word(amax, v.x);
-      amax = amax_word(amax, v.y);
-      amax = amax_word(amax, v.z);
-      amax = amax_word(amax, v.w);
+      uint32_t m2 = absmax_bf16x2(absmax_uint4(0u, v0), absmax_uint4(0u, v1));
 #pragma unroll
-      for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const QParams p = qparams_f32(amax);
-      const uint2 codes = quant8_bf16(v, p);
+      for (int o = 4; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+      const QParams p = qparams_f32(absmax_finish(m2));
+      const uint2 c0 = quant8_f32(v0, p), c1 = quant8_f32(v1, p);
       if (active) {
-        *reinterpret_cast<uint2 *>(q + m * ldq + b * 128 + hl * 8) = codes;
-        if (hl == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
+        uint8_t *qb = q + m * ldq + b * 128;
+        *reinterpret_cast<uint2 *>(qb + sub * 8) = c0;
+        *reinterpret_cast<uint2 *>(qb + 64 + sub * 8) = c1;
+        if (sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
       }
     }
-    __syncwarp();  // every lane is done with this buffer before it is refilled
+    __syncwarp();  // every lane is done with the staged row before it is refilled
   }
 }
 

@@ -102,7 +102,7 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
 
 /* Block-scaled W8A8 GEMM (a5): out[m, n] = bf16( sum_kb sa[m, kb] * sw[n/128, kb] * P_kb[m, n] )
  * where P_kb is the fp32 tensor-core dot product of the E4M3 codes over K-block kb and each
- * K-block partial is promoted (scaled and accumulated) in fp32.
+ * K-block partial is promoted (scaled and accumulated) in fp32.  K <= 32768.
  *   aq   [M][lda] uint8 activation codes     sa  fp32, sa[kb * lds + m]
  *   wq   [N][ldw] uint8 weight codes         sw  [N/128][K/128], fp32 or E8M0 per sw_fmt
  *   out  [M][ldo] bf16, written (rows < M, columns < N)
