@@ -213,14 +213,11 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   const int rc = device_state(&st);
   if (rc != FP8Q_OK) return rc;
   const bool norm = gamma_bf16 != nullptr;
-  const int KB = static_cast<int>(K / 128);
-  const int row_bytes = KB * fp8q::kRowBlockStride;
-  const int gamma_bytes = norm ? static_cast<int>(K) * 4 : 0;
   const int budget = 227 * 1024;
   // Warps per CTA: the choice that keeps the most warps resident per SM.
   int best_wpc = 0, best_ctas = 0, best_smem = 0;
   for (int wpc : {16, 12, 8, 4, 2, 1}) {
-    const int smem = norm ? gamma_bytes + wpc * row_bytes : 0;
+    const int smem = fp8q::token_smem_bytes(static_cast<int>(K), norm, wpc);
     if (smem > budget) continue;
     int per_sm = 0;
     if (norm)

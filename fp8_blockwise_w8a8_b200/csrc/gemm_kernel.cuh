@@ -38,7 +38,6 @@ constexpr int kStageBytes = kTileABytes + kTileBBytes;
 constexpr int kStagingBytesPerWarp = 32 * 64;     // 32 rows x 32 bf16 columns
 constexpr int kMaxExperts = 1024;
 constexpr int kGroupM = 16;                       // rasterization: m-blocks per group
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
 constexpr int kOffA = 0;
@@ -127,59 +126,6 @@ __device__ __forceinline__ Tile grouped_tile(const GemmArgs &a, const int *s_off
   tl.n0 = nb * kBN;
   tl.b_row = lo * a.N + tl.n0;
   return tl;
-}
-
-// Bounded wait by one thread.  Returns false on abort (another role gave up) or timeout.
-__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort_flag = 1;
-        record_error(6 /* FP8Q_ERR_TIMEOUT */);
-        return false;
-      }
-    }
-  }
-}
-
-// Bounded wait by a whole warp with a warp-uniform outcome.
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
-  const int lane = threadIdx.x & 31;
-  uint64_t t0 = 0;
-  for (uint32_t n = 0;; ++n) {
-    const bool ok = mbar_try_wait(bar, parity);
-    if (__all_sync(0xffffffffu, ok)) return true;
-    if ((n & 63u) == 63u) {
-      int stop = 0;
-      if (lane == 0) {
-        const uint64_t now = globaltimer_ns();
-        if (t0 == 0) t0 = now;
-        if (*abort_flag) {
-          stop = 1;
-        } else if (now - t0 > kWaitLimitNs) {
-          *abort_flag = 1;
-          record_error(6 /* FP8Q_ERR_TIMEOUT */);
-          stop = 1;
-        }
-      }
-      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
-    }
-  }
-}
-
-// Wait that ignores the abort flag (teardown drains); still bounded.
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      record_error(6 /* FP8Q_ERR_TIMEOUT */);
-      return;
-    }
-  }
 }
 
 __device__ __forceinline__ float load_sw(const GemmArgs &a, const uint8_t *sw_row, int kb) {

@@ -87,6 +87,26 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
+                                            int32_t z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16), completion
+// counted on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------------------------
 // tcgen05: TMEM allocation, MMA, commit, loads, fences
 // ---------------------------------------------------------------------------------------------
@@ -189,6 +209,66 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[64]) {
   tmem_ld_wait(*reinterpret_cast<uint32_t (*)[32]>(&r[0]));
   tmem_ld_wait(*reinterpret_cast<uint32_t (*)[32]>(&r[32]));
+}
+
+// ---------------------------------------------------------------------------------------------
+// Bounded mbarrier waits.  A wait that has not completed after kWaitLimitNs records
+// FP8Q_ERR_TIMEOUT (6) in the device error word, raises the CTA's abort flag and returns false;
+// every other waiter of the CTA then returns false at its next check.
+// ---------------------------------------------------------------------------------------------
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+
+// Bounded wait by one thread.  Returns false on abort (another role gave up) or timeout.
+__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        record_error(6 /* FP8Q_ERR_TIMEOUT */);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait by a whole warp with a warp-uniform outcome.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+  const int lane = threadIdx.x & 31;
+  uint64_t t0 = 0;
+  for (uint32_t n = 0;; ++n) {
+    const bool ok = mbar_try_wait(bar, parity);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    if ((n & 63u) == 63u) {
+      int stop = 0;
+      if (lane == 0) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        if (*abort_flag) {
+          stop = 1;
+        } else if (now - t0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          record_error(6 /* FP8Q_ERR_TIMEOUT */);
+          stop = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+    }
+  }
+}
+
+// Wait that ignores the abort flag (teardown drains); still bounded.
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(6 /* FP8Q_ERR_TIMEOUT */);
+      return;
+    }
+  }
 }
 
 // Register budget hand-off between warpgroups (all four warps of a warpgroup execute it).  The

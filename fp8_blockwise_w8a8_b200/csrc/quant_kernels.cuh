@@ -65,19 +65,25 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 
 // Per-block parameters of the fp32-scale quantizer.
-//   fast = true : bracket fast path (see quant8_f32), exact division when it is ambiguous.
-//   fast = false: exact IEEE division for every element (tiny scales, where 1/s would overflow).
+//   fast = true : bracket fast path (see quant8_f32), exact fallback where it is ambiguous.
+//   fast = false: the exact fp64 quotient for every element (tiny scales, s < 2^-60).
 struct QParams {
   float s;       // the scale (divisor)
   float2 lo2;    // RN(r * (1 - 2^-19)) in both lanes, r ~ 1/s
   float2 hi2;    // RN(r * (1 + 2^-19)) in both lanes
   bool fast;
+  bool tie;      // amax / 448 is exact (see quant8_f32)
 };
 
 __device__ __forceinline__ QParams qparams_f32(float amax) {
   QParams p;
   p.s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-  p.fast = p.s >= 0x1.0p-100f;
+  // amax is a bf16 value a * 2^E with an integer significand a <= 255; amax / 448 =
+  // (a / 7) * 2^(E - 6) is exact iff 7 divides a.
+  const uint32_t ab = __float_as_uint(amax);
+  const uint32_t a = ((ab >> 16) & 0x7Fu) | (((ab >> 23) & 0xFFu) != 0u ? 0x80u : 0u);
+  p.tie = (a % 7u) == 0u;
+  p.fast = p.s >= 0x1.0p-60f;
   // r approximates 1/s within one ulp (2^-23 relative, the documented bound of rcp.approx).
   const float r = rcp_approx(p.fast ? p.s : 1.0f);
   const float lo = __fmul_rn(r, 0x1.ffffc0p-1f), hi = __fmul_rn(r, 0x1.000020p+0f);
@@ -92,11 +98,36 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
 
 // Eight E4M3 codes of RN_fp32(x / s) for the eight bf16 values of one uint4 (byte i = element i).
 //
+// Where the bracket ends disagree there are two cases.  If amax/448 is exact, s = b 2^k with
+// b = a/7 <= 36 (at most 6 significant bits), so mid * s has at most 11 significant bits for every
+// E4M3 midpoint mid (5 bits): a quotient x/s that is not exactly a midpoint then lies at least
+// ~2^-11 (relative) away from it, far outside the bracket -- a disagreement is an exact tie and
+// the code is the even one of the two.  Otherwise the eight codes are recomputed through the
+// exact fp64 quotient (quant8_fp64).
+//
 // Bracket: with r = 1/s (1 + e_r), |e_r| <= 2^-23, the rounded products x * RN(r (1 -+ 2^-19))
 // are within a relative 2^-23 + 3 * 2^-24 of x/s (1 -+ 2^-19), so they bracket x/s strictly.
 // RN_fp32 and the E4M3 conversion are both monotone, hence when the two bracket ends give the
 // same code, that code is the code of RN_fp32(x/s).  Otherwise (some x/s within ~2^-19 of an
 // E4M3 rounding boundary, exact ties included) the eight values are redone with IEEE divisions.
+// Eight codes through an fp64 quotient, exact for every element: with r64 = RN64(1/s) the product
+// q64 = RN64(x * r64) is within 2^-52 (relative) of x/s.  If x/s is an fp32 number, RN32(q64) is
+// that number.  Otherwise x/s is at least ~2^-49 (relative) away from every fp32 rounding
+// boundary B -- B has 25 significant bits ending in a one, so B * s has at least 24 and can never
+// equal the 8-bit x -- and RN32(q64) = RN32(x/s).  Used only where the fp32 bracket is ambiguous.
+__device__ __forceinline__ uint2 quant8_fp64(const uint4 v, float s) {
+  const double r64 = __drcp_rn(static_cast<double>(s));
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t c[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 x = unpack_bf16x2(w[j]);
+    c[j] = cvt_e4m3x2(__double2float_rn(__dmul_rn(static_cast<double>(x.x), r64)),
+                      __double2float_rn(__dmul_rn(static_cast<double>(x.y), r64)));
+  }
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
 __device__ __forceinline__ uint2 quant8_f32(const uint4 v, const QParams &p) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
   if (p.fast) {
@@ -110,15 +141,16 @@ __device__ __forceinline__ uint2 quant8_f32(const uint4 v, const QParams &p) {
     }
     const uint32_t l0 = lo[0] | (lo[1] << 16), l1 = lo[2] | (lo[3] << 16);
     const uint32_t h0 = hi[0] | (hi[1] << 16), h1 = hi[2] | (hi[3] << 16);
-    if (((l0 ^ h0) | (l1 ^ h1)) == 0u) return make_uint2(l0, l1);
+    const uint32_t d0 = l0 ^ h0, d1 = l1 ^ h1;
+    if (__builtin_expect((d0 | d1) == 0u, 1)) return make_uint2(l0, l1);
+    if (p.tie) {
+      // exact ties: per byte, keep the lower end's code if it is even, else take the other
+      // (the two magnitudes are adjacent and share the sign)
+      return make_uint2(l0 ^ (d0 & ((l0 & 0x01010101u) * 0xFFu)),
+                        l1 ^ (d1 & ((l1 & 0x01010101u) * 0xFFu)));
+    }
   }
-  uint32_t c[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float2 x = unpack_bf16x2(w[j]);
-    c[j] = cvt_e4m3x2(__fdiv_rn(x.x, p.s), __fdiv_rn(x.y, p.s));
-  }
-  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+  return quant8_fp64(v, p.s);  // ambiguous bracket, or a tiny scale (s < 2^-60)
 }
 
 // Eight codes for a power-of-two scale 2^e: x * 2^-e is exact (inv2 = {2^-e, 2^-e}).
@@ -185,15 +217,60 @@ __global__ void __launch_bounds__(256, 4) k_quant_weight_block(const uint16_t *_
 }
 
 // ---------------------------------------------------------------------------------------------
+// Scale parameters from a table, for the token kernel (one scale per 128 elements, so the
+// per-block arithmetic matters).  amax = a * 2^(ef - 134) with a = 128 + (7 mantissa bits) the
+// bf16 significand; s = RN(amax / 448) = RN(a / 7) * 2^(ef - 140) exactly while the result is a
+// normal number, and 1/s ~ RN(7 / a) * 2^(140 - ef) within 2^-23 (two roundings of 2^-24).
+// The table holds, per a: RN(a/7), RN(RN(7/a) (1 - 2^-19)), RN(RN(7/a) (1 + 2^-19)); it is
+// built with IEEE divisions when the kernel starts.
+// ---------------------------------------------------------------------------------------------
+struct ScaleTab {
+  float s[128], lo[128], hi[128];
+};
+
+__device__ __forceinline__ void build_scale_tab(ScaleTab *t, int tid, int nthreads) {
+  for (int i = tid; i < 128; i += nthreads) {
+    const float a = static_cast<float>(128 + i);
+    t->s[i] = __fdiv_rn(a, 7.0f);
+    const float r = __fdiv_rn(7.0f, a);
+    t->lo[i] = __fmul_rn(r, 0x1.ffffc0p-1f);
+    t->hi[i] = __fmul_rn(r, 0x1.000020p+0f);
+  }
+}
+
+// x * 2^k for a normal x and a result in the normal range (exact: exponent arithmetic).
+__device__ __forceinline__ float scale_pow2(float x, int k) {
+  return __uint_as_float(__float_as_uint(x) + (static_cast<uint32_t>(k) << 23));
+}
+
+__device__ __forceinline__ QParams qparams_tab(float amax, const ScaleTab *t) {
+  const uint32_t ab = __float_as_uint(amax);
+  const int ef = static_cast<int>(ab >> 23);
+  if (ef < 75) return qparams_f32(amax);  // zero or tiny blocks: s < 2^-60
+  const int i = static_cast<int>((ab >> 16) & 0x7Fu);
+  QParams p;
+  p.s = scale_pow2(t->s[i], ef - 140);
+  const float lo = scale_pow2(t->lo[i], 140 - ef), hi = scale_pow2(t->hi[i], 140 - ef);
+  p.lo2 = make_float2(lo, lo);
+  p.hi2 = make_float2(hi, hi);
+  p.fast = true;
+  p.tie = ((128u + static_cast<uint32_t>(i)) % 7u) == 0u;
+  return p;
+}
+
+// ---------------------------------------------------------------------------------------------
 // 1x128 token groups, optionally preceded by RMSNorm.  One warp per row at a time.
 //
 // With RMSNorm the row is staged in shared memory (cp.async) in a padded layout -- 128-element
 // blocks at a 272-byte stride -- so that lane b can walk its own block b in ascending k for the
-// fp64 sum of squares without bank conflicts.  gamma is held once per CTA as fp32.  Without
-// RMSNorm nothing is staged: each step reads the row straight from global memory.  In both
+// fp64 sum of squares without bank conflicts.  gamma is held once per CTA as fp32, split per
+// 16-byte chunk j into gA[j] (elements 8j..8j+3) and gB[j] (8j+4..8j+7).  Without RMSNorm
+// nothing is staged: the quantization reads the row straight from global memory.  In both
 // cases the next row of the warp is prefetched into L2 while the current one is processed.
 //
-// Quantization step: lanes 0-15 take block 2j, lanes 16-31 block 2j + 1, each lane 8 elements.
+// Quantization: LPB lanes per 128-block (8 with RMSNorm, reading the staged row without bank
+// conflicts; 4 without, reading global memory), 32 / LPB blocks per warp step; lane `sub` of a
+// block owns the 16-byte chunks sub + LPB c, c = 0 .. 16 / LPB - 1.
 // ---------------------------------------------------------------------------------------------
 constexpr int kRowBlockStride = 272;
 
@@ -229,31 +306,40 @@ __device__ __forceinline__ uint4 rms_apply8(const uint4 v, float r, const float4
   return make_uint4(y[0], y[1], y[2], y[3]);
 }
 
+// Shared-memory bytes of the token kernel.
+__host__ __device__ constexpr int token_smem_bytes(int K, bool norm, int wpc) {
+  return static_cast<int>(sizeof(ScaleTab)) +
+         (norm ? K * 4 + wpc * (K / 128) * kRowBlockStride : 0);
+}
+
 template <bool NORM>
 __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
     int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ sa, int64_t lds) {
+  constexpr int LPB = NORM ? 8 : 4;        // lanes per 128-block
+  constexpr int CPL = 16 / LPB;            // 16-byte chunks per lane
+  constexpr int BPS = 32 / LPB;            // blocks per warp step
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int wpc = blockDim.x >> 5;
   const int KB = K >> 7;
   const int row_bytes = KB * kRowBlockStride;
-  // gamma as fp32, split per 16-byte chunk j of the row into gA[j] (elements 8j..8j+3) and
-  // gB[j] (8j+4..8j+7), so that eight lanes reading eight consecutive chunks hit distinct banks.
-  float4 *gA = reinterpret_cast<float4 *>(smem);
+  ScaleTab *tab = reinterpret_cast<ScaleTab *>(smem);
+  float4 *gA = reinterpret_cast<float4 *>(smem + sizeof(ScaleTab));
   float4 *gB = gA + (K >> 3);
-  uint8_t *row = smem + (NORM ? K * 4 : 0) + warp * row_bytes;
+  uint8_t *row = smem + sizeof(ScaleTab) + K * 4 + warp * row_bytes;  // NORM only
   const uint32_t row_u32 = smem_u32(row);
-  const int grp = lane >> 3, sub = lane & 7;   // 8 lanes per 128-block, 4 blocks per step
+  const int grp = lane / LPB, sub = lane % LPB;
 
+  build_scale_tab(tab, threadIdx.x, blockDim.x);
   if (NORM) {
     for (int j = threadIdx.x; j < (K >> 3); j += blockDim.x) {
       const uint4 g = *reinterpret_cast<const uint4 *>(gamma + j * 8);
       gA[j] = make_float4(bf16_lo(g.x), bf16_hi(g.x), bf16_lo(g.y), bf16_hi(g.y));
       gB[j] = make_float4(bf16_lo(g.z), bf16_hi(g.z), bf16_lo(g.w), bf16_hi(g.w));
     }
-    __syncthreads();
   }
+  __syncthreads();
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
   for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < M; m += stride) {
@@ -273,9 +359,9 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
       // Sum of squares in fp64: each lane walks its own 128-blocks in ascending k ...
       double P[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        P[i] = 0.0;
-        const int b = lane + 32 * i;
+      for (int t = 0; t < 4; ++t) {
+        P[t] = 0.0;
+        const int b = lane + 32 * t;
         if (b < KB) {
           const uint4 *blk = reinterpret_cast<const uint4 *>(row + b * kRowBlockStride);
           double acc = 0.0;
@@ -291,54 +377,65 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
               acc = __fma_rn(b2, b2, acc);
             }
           }
-          P[i] = acc;
+          P[t] = acc;
         }
       }
       // ... then the block sums are added in ascending block order.
       double S = 0.0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (32 * i >= KB) break;
+      for (int t = 0; t < 4; ++t) {
+        if (32 * t >= KB) break;
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) {
-          const double pj = __shfl_sync(0xffffffffu, P[i], j);
-          if (32 * i + j < KB) S = __dadd_rn(S, pj);
+          const double pj = __shfl_sync(0xffffffffu, P[t], j);
+          if (32 * t + j < KB) S = __dadd_rn(S, pj);
         }
       }
       const double var = __dadd_rn(__ddiv_rn(S, static_cast<double>(K)), static_cast<double>(eps));
       r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(var)));
     }
 
-    // Quantize: lanes 8g .. 8g+7 take block b0 + g; lane `sub` owns 16-byte chunks sub and
-    // sub + 8 of the block (elements 8 sub .. 8 sub + 7 and 64 + 8 sub .. 64 + 8 sub + 7).
+    // Without RMSNorm the loads of the next step are issued before this step is processed.
+    uint4 vn[CPL];
+    if (!NORM) {
+      const int bb = grp < KB ? grp : 0;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) vn[c] = ld_stream_v4(xr + bb * 128 + (sub + LPB * c) * 8);
+    }
 #pragma unroll 2
-    for (int b0 = 0; b0 < KB; b0 += 4) {
+    for (int b0 = 0; b0 < KB; b0 += BPS) {
       const int b = b0 + grp;
       const bool active = b < KB;
       const int bb = active ? b : b0;
-      uint4 v0, v1;
-      if (NORM) {
-        const uint8_t *rb = row + bb * kRowBlockStride;
-        v0 = *reinterpret_cast<const uint4 *>(rb + sub * 16);
-        v1 = *reinterpret_cast<const uint4 *>(rb + (sub + 8) * 16);
-        const int j0 = bb * 16 + sub, j1 = j0 + 8;
-        v0 = rms_apply8(v0, r, gA[j0], gB[j0]);
-        v1 = rms_apply8(v1, r, gA[j1], gB[j1]);
-      } else {
-        v0 = ld_stream_v4(xr + bb * 128 + sub * 8);
-        v1 = ld_stream_v4(xr + bb * 128 + 64 + sub * 8);
-      }
-      uint32_t m2 = absmax_bf16x2(absmax_uint4(0u, v0), absmax_uint4(0u, v1));
+      uint4 v[CPL];
 #pragma unroll
-      for (int o = 4; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-      const QParams p = qparams_f32(absmax_finish(m2));
-      const uint2 c0 = quant8_f32(v0, p), c1 = quant8_f32(v1, p);
-      if (active) {
-        uint8_t *qb = q + m * ldq + b * 128;
-        *reinterpret_cast<uint2 *>(qb + sub * 8) = c0;
-        *reinterpret_cast<uint2 *>(qb + 64 + sub * 8) = c1;
-        if (sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
+      for (int c = 0; c < CPL; ++c) {
+        const int chunk = sub + LPB * c;
+        if (NORM) {
+          v[c] = *reinterpret_cast<const uint4 *>(row + bb * kRowBlockStride + chunk * 16);
+          v[c] = rms_apply8(v[c], r, gA[bb * 16 + chunk], gB[bb * 16 + chunk]);
+        } else {
+          v[c] = vn[c];
+        }
       }
+      if (!NORM && b0 + BPS < KB) {
+        const int bn = b0 + BPS + grp < KB ? b0 + BPS + grp : b0 + BPS;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) vn[c] = ld_stream_v4(xr + bn * 128 + (sub + LPB * c) * 8);
+      }
+      uint32_t m2 = 0u;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) m2 = absmax_uint4(m2, v[c]);
+#pragma unroll
+      for (int o = LPB / 2; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+      const QParams p = qparams_tab(absmax_finish(m2), tab);
+      uint8_t *qb = q + m * ldq + b * 128;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        const uint2 codes = quant8_f32(v[c], p);
+        if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
+      }
+      if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
     }
     __syncwarp();  // every lane is done with the staged row before it is refilled
   }
