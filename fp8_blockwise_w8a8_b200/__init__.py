@@ -9,6 +9,7 @@ library or a non-sm_100 device raises.
     quant_weight_block(w, fmt)                 bf16 [N, K] -> (codes u8 [N, K], scales [N/128, K/128])
     rmsnorm_quant_token(x, gamma, eps)         bf16 [M, K] -> (codes u8 [M, K], sa f32 [K/128, lds])
     gemm_w8a8_block(aq, sa, wq, sw, fmt)       -> bf16 [M, N]
+    gemm_w8a8_block_splitk(aq, sa, wq, sw, ...) -> bf16 [M, N], K split over CTAs (small M)
     grouped_gemm_w8a8_block(aq, sa, wq, sw, offsets, fmt) -> bf16 [M, N]
 """
 import torch
@@ -18,7 +19,10 @@ from ._lib import (FP8Q_ERR_ALIGN, FP8Q_ERR_ARCH, FP8Q_ERR_ARG, FP8Q_ERR_LAUNCH,
                    FP8Q_ERR_SHAPE, FP8Q_ERR_TIMEOUT, FP8Q_OK, FP8Q_SCALE_E8M0, FP8Q_SCALE_F32,
                    Fp8qError)
 
+import ctypes
+
 __all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
+           "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -89,6 +93,41 @@ def gemm_w8a8_block(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, sw: to
                                          _ld(wq), _ptr(sw), f, M, N, K, _ptr(o), _ld(o),
                                          _stream(stream))
     _lib.check(st, "fp8q_gemm_w8a8_block")
+    return o
+
+
+def gemm_splitk_workspace_bytes(M: int, N: int, K: int, splits: int = 0) -> int:
+    """Bytes of split-K workspace for these sizes (splits=0: the library's choice)."""
+    b = ctypes.c_int64(0)
+    st = _lib.lib().fp8q_gemm_splitk_workspace_bytes(M, N, K, int(splits), ctypes.byref(b))
+    _lib.check(st, "fp8q_gemm_splitk_workspace_bytes")
+    return b.value
+
+
+def splitk_workspace(M: int, N: int, K: int, splits: int = 0, device=None) -> torch.Tensor:
+    """A zeroed workspace for gemm_w8a8_block_splitk; reusable by later calls in stream order."""
+    n = gemm_splitk_workspace_bytes(M, N, K, splits)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def gemm_w8a8_block_splitk(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor,
+                           sw: torch.Tensor, fmt=None, splits: int = 0, workspace=None, out=None,
+                           stream=None):
+    """gemm_w8a8_block with K split over several CTAs per output tile.  `workspace` is a zeroed
+    uint8 device tensor of gemm_splitk_workspace_bytes(M, N, K, splits) bytes, reused across
+    calls on one stream; None allocates a fresh one."""
+    f = scale_format(sw.dtype if fmt is None else fmt)
+    M, K = aq.shape
+    N = wq.shape[0]
+    if workspace is None:
+        workspace = splitk_workspace(M, N, K, splits, device=aq.device)
+    o = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device) if out is None else out
+    st = _lib.lib().fp8q_gemm_w8a8_block_splitk(_ptr(aq), _ld(aq), _ptr(sa), sa.stride(0),
+                                                _ptr(wq), _ld(wq), _ptr(sw), f, M, N, K, _ptr(o),
+                                                _ld(o), int(splits), _ptr(workspace),
+                                                workspace.numel() * workspace.element_size(),
+                                                _stream(stream))
+    _lib.check(st, "fp8q_gemm_w8a8_block_splitk")
     return o
 
 

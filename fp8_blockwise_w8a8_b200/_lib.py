@@ -30,6 +30,9 @@ SIGNATURES = {
                                       _I64, _P]),
     "fp8q_gemm_w8a8_block": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64, _I64, _P,
                                   _I64, _P]),
+    "fp8q_gemm_w8a8_block_splitk": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64, _I64,
+                                         _P, _I64, _I, _P, _I64, _P]),
+    "fp8q_gemm_splitk_workspace_bytes": (_I, [_I64, _I64, _I64, _I, ctypes.POINTER(_I64)]),
     "fp8q_grouped_gemm_w8a8_block": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _P, _I64, _I64,
                                           _I64, _I64, _P, _I64, _P]),
     "fp8q_check_device_error": (_I, [_P]),

@@ -114,10 +114,38 @@ int check_gemm_common(const void *aq, int64_t lda, const float *sa, int64_t lds,
   return FP8Q_OK;
 }
 
+// Split-K workspace: fp32 partials of one 128 x 256 tile per (tile, split), then one int32
+// arrival counter per tile.
+constexpr int64_t kSplitPartialBytes = int64_t{fp8q::kBM} * fp8q::kBN * 4;
+
+int64_t splitk_tiles(int64_t M, int64_t N) {
+  return ((M + fp8q::kBM - 1) / fp8q::kBM) * ((N + fp8q::kBN - 1) / fp8q::kBN);
+}
+
+int64_t splitk_workspace_bytes(int64_t M, int64_t N, int splits) {
+  if (splits <= 1) return 0;
+  const int64_t tiles = splitk_tiles(M, N);
+  return tiles * splits * kSplitPartialBytes + ((tiles * 4 + 15) / 16) * 16;
+}
+
+// splits = 0 picks the K-split count: 1 when the tiles alone fill the SMs, else as many splits as
+// fit the SMs, each keeping at least 4 K-blocks.  Returns a count in [1, K/128] or 0 on error.
+int resolve_splits(int64_t M, int64_t N, int64_t K, int splits, int sms) {
+  const int64_t KB = K / fp8q::kBK;
+  if (splits < 0 || splits > KB) return 0;
+  if (splits > 0) return splits;
+  const int64_t tiles = splitk_tiles(M, N);
+  if (tiles <= 0 || tiles * 2 > sms) return 1;
+  int64_t s = sms / tiles;
+  if (s > KB / 4) s = KB / 4;
+  return static_cast<int>(s < 1 ? 1 : s);
+}
+
 int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int64_t lds,
                 const void *wq, int64_t ldw, const void *sw, int sw_fmt,
                 const int32_t *group_offsets, int64_t E, int64_t M, int64_t N, int64_t K,
-                void *out, int64_t ldo, cudaStream_t stream) {
+                void *out, int64_t ldo, cudaStream_t stream, int splits = 1,
+                void *workspace = nullptr) {
   DeviceState *st = nullptr;
   int rc = device_state(&st);
   if (rc != FP8Q_OK) return rc;
@@ -140,9 +168,16 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
   a.ldo = ldo;
   a.num_n = static_cast<int>((N + fp8q::kBN - 1) / fp8q::kBN);
   a.num_m = static_cast<int>((M + fp8q::kBM - 1) / fp8q::kBM);
+  a.splits = splits;
+  a.ws = static_cast<float *>(workspace);
+  a.cnt = nullptr;
   // Upper bound of the tile count (grouped: every expert may add one partial m-tile).
   const int64_t tiles = (static_cast<int64_t>(a.num_m) + (grouped ? E : 0)) * a.num_n;
-  const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+  if (splits > 1)
+    a.cnt = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) +
+                                    tiles * splits * kSplitPartialBytes);
+  const int64_t units = tiles * splits;
+  const int grid = static_cast<int>(units < st->sms ? units : st->sms);
   if (grouped)
     fp8q::k_gemm_w8a8_block<true><<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemGrouped, stream>>>(
         tm_a, tm_b, a);
@@ -156,7 +191,7 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
 
 extern "C" {
 
-int fp8q_abi_version(void) { return (1 << 16) | 0; }
+int fp8q_abi_version(void) { return (1 << 16) | 1; }
 
 const char *fp8q_status_string(int status) {
   switch (status) {
@@ -258,6 +293,51 @@ int fp8q_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t l
   if (sw_fmt == FP8Q_SCALE_F32 && (reinterpret_cast<uintptr_t>(sw) & 3u)) return FP8Q_ERR_ALIGN;
   return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K, out_bf16,
                      ldo, stream);
+}
+
+int fp8q_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int splits,
+                                     int64_t *bytes) {
+  if (!bytes) return FP8Q_ERR_NULL;
+  *bytes = 0;
+  if (M < 0 || N <= 0 || K <= 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
+  if (M > INT32_MAX - 256 || N > (1 << 30) || K > 128 * fp8q::kMaxKB) return FP8Q_ERR_SHAPE;
+  if (splits < 0 || splits > K / 128) return FP8Q_ERR_ARG;
+  int sms = 0;
+  if (splits == 0) {
+    DeviceState *st = nullptr;
+    const int rc = device_state(&st);
+    if (rc != FP8Q_OK) return rc;
+    sms = st->sms;
+  }
+  const int s = resolve_splits(M, N, K, splits, sms);
+  if (s <= 0) return FP8Q_ERR_ARG;
+  if (splitk_tiles(M, N) * s > INT32_MAX) return FP8Q_ERR_SHAPE;
+  *bytes = splitk_workspace_bytes(M, N, s);
+  return FP8Q_OK;
+}
+
+int fp8q_gemm_w8a8_block_splitk(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                                const void *wq, int64_t ldw, const void *sw, int sw_fmt,
+                                int64_t M, int64_t N, int64_t K, void *out_bf16, int64_t ldo,
+                                int splits, void *workspace, int64_t workspace_bytes,
+                                cudaStream_t stream) {
+  int rc = check_gemm_common(aq, lda, sa, lds, wq, ldw, sw, sw_fmt, M, N, K, out_bf16, ldo);
+  if (rc != FP8Q_OK) return rc;
+  if (splits < 0 || splits > K / 128) return FP8Q_ERR_ARG;
+  if (M == 0) return FP8Q_OK;
+  if (sw_fmt == FP8Q_SCALE_F32 && (reinterpret_cast<uintptr_t>(sw) & 3u)) return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  if ((rc = device_state(&st)) != FP8Q_OK) return rc;
+  const int s = resolve_splits(M, N, K, splits, st->sms);
+  if (s <= 0) return FP8Q_ERR_ARG;
+  if (splitk_tiles(M, N) * s > INT32_MAX) return FP8Q_ERR_SHAPE;
+  if (s > 1) {
+    if (!workspace) return FP8Q_ERR_NULL;
+    if (!aligned16(workspace)) return FP8Q_ERR_ALIGN;
+    if (workspace_bytes < splitk_workspace_bytes(M, N, s)) return FP8Q_ERR_SHAPE;
+  }
+  return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K, out_bf16,
+                     ldo, stream, s, s > 1 ? workspace : nullptr);
 }
 
 int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t lds,

@@ -48,9 +48,10 @@ constexpr int kMaxKB = 256;                       // K <= 32768
 constexpr int kOffSa = kOffStaging + 8 * kStagingBytesPerWarp;      // [kSaStages][128] fp32
 constexpr int kOffSw = kOffSa + kSaStages * kBM * 4;                // [2 tiles][2 halves][kMaxKB]
 constexpr int kOffBar = kOffSw + 2 * 2 * kMaxKB * 4;
-// full, empty, tmem_full[2], tmem_empty[2], done, sa_full/empty[kSaStages], sw_full/empty[2]
-constexpr int kNumBars = 2 * kStages + 4 + 1 + 2 * kSaStages + 4;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
+// full, empty, tmem_full[2], tmem_empty[2], done, sa_full/empty[kSaStages], sw_full/empty[2],
+// split-K handshake ep1, ep2
+constexpr int kNumBars = 2 * kStages + 4 + 1 + 2 * kSaStages + 4 + 2;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag, split-K last flag
 constexpr int kOffGroups = kOffMisc + 16;          // grouped: offsets[E+1], tile prefix[E+1]
 constexpr int kGemmSmemDense = kOffGroups + 1024;  // + alignment slack
 constexpr int kGemmSmemGrouped = kOffGroups + 2 * (kMaxExperts + 1) * 4 + 1024;
@@ -81,7 +82,24 @@ struct GemmArgs {
   int64_t ldo;
   int num_n;            // ceil(N / 256)
   int num_m;            // dense: ceil(M / 128)
+  int splits;           // K-splits per tile (1: no split)
+  float *ws;            // splits > 1: fp32 partials, [tile][split][2][32][128] float4
+  int *cnt;             // splits > 1: one arrival counter per tile, zero between launches
 };
+
+// Work unit u covers tile u / splits and the K-blocks [kb0, kb1) of split u % splits.
+struct Unit {
+  int t, j, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit unit_of(const GemmArgs &a, int u, int KB) {
+  Unit w;
+  w.t = u / a.splits;
+  w.j = u - w.t * a.splits;
+  w.kb0 = (w.j * KB) / a.splits;
+  w.kb1 = ((w.j + 1) * KB) / a.splits;
+  return w;
+}
 
 struct Tile {
   int m0;        // first row of the tile in A / out
@@ -151,6 +169,42 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// bf16 conversion and store of 32 columns (v[j] = columns 2j, 2j + 1 of chunk c4) of this
+// thread's row, through the warp's swizzled staging buffer so that each global store
+// instruction writes 64-byte row segments.
+__device__ __forceinline__ void store_chunk32(const float2 (&v)[16], uint32_t stage_u32, int lane,
+                                              uint16_t *out_base, const Tile &tl, int q, int c4,
+                                              bool col_ok, int64_t ldo) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t pk[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat162 v2 = __floats2bfloat162_rn(v[4 * j + u].x, v[4 * j + u].y);
+      pk[u] = *reinterpret_cast<const uint32_t *>(&v2);
+    }
+    const int phys = j ^ ((lane >> 1) & 3);
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stage_u32 + lane * 64 + phys * 16),
+                 "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                 : "memory");
+  }
+  __syncwarp();
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const int r = p * 8 + (lane >> 2), c = lane & 3;
+    const int phys = c ^ ((r >> 1) & 3);
+    uint4 w;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                 : "r"(stage_u32 + r * 64 + phys * 16)
+                 : "memory");
+    const int grow = tl.m0 + 32 * q + r;
+    if (col_ok && grow < tl.row_end)
+      *reinterpret_cast<uint4 *>(out_base + static_cast<int64_t>(grow) * ldo + 32 * c4 + 8 * c) = w;
+  }
+  __syncwarp();
+}
+
 template <bool GROUPED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm_w8a8_block(const __grid_constant__ CUtensorMap tm_a,
@@ -169,6 +223,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t bar_saempty = bar_safull + 8 * kSaStages;    // [kSaStages]
   const uint32_t bar_swfull = bar_saempty + 8 * kSaStages;    // [2]
   const uint32_t bar_swempty = bar_swfull + 16;               // [2]
+  const uint32_t bar_ep1 = bar_swempty + 16;                  // epilogue warps -> leader
+  const uint32_t bar_ep2 = bar_ep1 + 8;                       // leader -> epilogue warps
+  volatile int *s_last = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
   float *s_sa = reinterpret_cast<float *>(smem + kOffSa);
   float *s_sw = reinterpret_cast<float *>(smem + kOffSw);
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + kOffMisc);
@@ -196,6 +253,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(bar_swfull + 8 * i, 32);
       mbar_init(bar_swempty + 8 * i, 8);
     }
+    mbar_init(bar_ep1, 8);
+    mbar_init(bar_ep2, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -203,7 +262,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tmem_alloc(smem_u32(s_tmem), 512);
     tmem_relinquish();
   }
-  int total_tiles;
+  int total_tiles, total_units;
   if (GROUPED) {
     // Clamp the offsets into [previous, M] and count m-tiles per expert.
     for (int i = threadIdx.x; i <= args.E; i += blockDim.x) s_off[i] = args.group_offsets[i];
@@ -229,6 +288,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   total_tiles = GROUPED ? s_prefix[args.E] * args.num_n : args.num_m * args.num_n;
+  total_units = total_tiles * args.splits;
 
   if (warp < 4) {
     reg_dealloc<kProducerRegs>();
@@ -238,10 +298,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_b);
         uint32_t it = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-          const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, t) : dense_tile(args, t);
+        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+          const Unit un = unit_of(args, u, KB);
+          const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, un.t) : dense_tile(args, un.t);
           bool ok = true;
-          for (int kb = 0; kb < KB; ++kb, ++it) {
+          for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
             const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
             if (!wait_one(bar_empty + 8 * s, ph ^ 1u, s_abort)) { ok = false; break; }
             mbar_arrive_expect_tx(bar_full + 8 * s, kStageBytes);
@@ -264,8 +325,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const size_t sw_elem = args.sw_fmt == 0 ? 4 : 1;
       uint32_t it = 0, tile_it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tile_it) {
-        const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, t) : dense_tile(args, t);
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++tile_it) {
+        const Unit un = unit_of(args, u, KB);
+        const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, un.t) : dense_tile(args, un.t);
         // weight scales of the tile's two 128-column halves, all K-blocks, as fp32
         const uint32_t tp = tile_it & 1u;
         if (!wait_warp(bar_swempty + 8 * tp, ((tile_it >> 1) & 1u) ^ 1u, s_abort)) break;
@@ -283,7 +345,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         mbar_arrive(bar_swfull + 8 * tp);
         // activation scales: one 128-row column of sa per K-block, zero-filled past row_end
         const int rows_here = tl.row_end - tl.m0;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
           const uint32_t s2 = it % kSaStages, ph2 = (it / kSaStages) & 1u;
           if (!wait_warp(bar_saempty + 8 * s2, ph2 ^ 1u, s_abort)) { ok = false; break; }
           const float *src = args.sa + static_cast<int64_t>(kb) * args.lds + tl.m0 + 4 * lane;
@@ -305,9 +367,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // ------------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         uint32_t it = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+        for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+          const Unit un = unit_of(args, u, KB);
           bool ok = true;
-          for (int kb = 0; kb < KB; ++kb, ++it) {
+          for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
             const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
             const uint32_t b = it & 1u, bph = (it >> 1) & 1u;
             if (!wait_one(bar_tempty + 8 * b, bph ^ 1u, s_abort)) { ok = false; break; }
@@ -340,8 +403,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t stage_u32 = smem_u32(stage);
     uint32_t it = 0, tile_it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tile_it) {
-      const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, t) : dense_tile(args, t);
+    for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x, ++tile_it) {
+      const Unit un = unit_of(args, u, KB);
+      const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, un.t) : dense_tile(args, un.t);
       const int nbh = tl.n0 / 128 + h;
       const bool col_ok = nbh < NB;
       const uint32_t tp = tile_it & 1u;
@@ -350,7 +414,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float2 acc[64];  // columns 2j, 2j + 1 of this thread's row
 #pragma unroll
       for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
         const uint32_t s2 = it % kSaStages, ph2 = (it / kSaStages) & 1u;
         if (!wait_warp(bar_safull + 8 * s2, ph2, s_abort)) { ok = false; break; }
         const float sc = __fmul_rn(s_sa[s2 * kBM + 32 * q + lane], sw_tile[kb]);
@@ -383,41 +447,61 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!ok) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_swempty + 8 * tp);
-      // bf16 conversion and store, 32 columns at a time through a swizzled staging buffer so
-      // that each global store instruction writes 64-byte row segments.
       uint16_t *out_base = args.out + static_cast<int64_t>(tl.n0 + 128 * h);
+      if (args.splits > 1) {
+        // Split K: publish this split's fp32 partial, count arrivals per tile; the last split to
+        // arrive adds all partials in split order (a fixed order: deterministic) and stores.
+        const int rl = 32 * q + lane;
+        float4 *ws_tile = reinterpret_cast<float4 *>(args.ws) +
+                          static_cast<size_t>(un.t) * args.splits * (2 * 32 * 128);
+        float4 *mine = ws_tile + static_cast<size_t>(un.j) * (2 * 32 * 128) + (h * 32) * 128 + rl;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float2 a2 = acc[16 * c4 + 4 * j + u];
-            const __nv_bfloat162 v2 = __floats2bfloat162_rn(a2.x, a2.y);
-            pk[u] = *reinterpret_cast<const uint32_t *>(&v2);
+        for (int c = 0; c < 32; ++c)
+          __stcg(mine + c * 128, make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x,
+                                             acc[2 * c + 1].y));
+        __threadfence();
+        __syncwarp();
+        const uint32_t pu = (tile_it & 1u);  // one handshake per unit: parity alternates
+        if (lane == 0) mbar_arrive(bar_ep1);
+        if (warp == 4) {
+          if (!wait_warp(bar_ep1, pu, s_abort)) { ok = false; break; }
+          if (lane == 0) {
+            const int prev = atomicAdd(args.cnt + un.t, 1);
+            __threadfence();
+            *s_last = (prev == args.splits - 1) ? 1 : 0;
+            mbar_arrive(bar_ep2);
           }
-          const int phys = j ^ ((lane >> 1) & 3);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stage_u32 + lane * 64 + phys * 16),
-                       "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
-                       : "memory");
+          __syncwarp();
         }
-        __syncwarp();
+        if (!wait_warp(bar_ep2, pu, s_abort)) { ok = false; break; }
+        if (!*s_last) continue;
+        // Sum the partials (this CTA's own included, re-read from L2) 32 columns at a time.
+        const float4 *col = ws_tile + (h * 32) * 128 + rl;
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float2 v[16];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const int r = p * 8 + (lane >> 2), c = lane & 3;
-          const int phys = c ^ ((r >> 1) & 3);
-          uint4 v;
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                       : "r"(stage_u32 + r * 64 + phys * 16)
-                       : "memory");
-          const int grow = tl.m0 + 32 * q + r;
-          if (col_ok && grow < tl.row_end)
-            *reinterpret_cast<uint4 *>(out_base + static_cast<int64_t>(grow) * args.ldo + 32 * c4 + 8 * c) = v;
+          for (int c = 0; c < 16; ++c) v[c] = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+          for (int i = 0; i < args.splits; ++i) {
+            const float4 *src = col + static_cast<size_t>(i) * (2 * 32 * 128) + (8 * c4) * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const float4 p = __ldcg(src + c * 128);
+              v[2 * c] = make_float2(__fadd_rn(v[2 * c].x, p.x), __fadd_rn(v[2 * c].y, p.y));
+              v[2 * c + 1] = make_float2(__fadd_rn(v[2 * c + 1].x, p.z),
+                                         __fadd_rn(v[2 * c + 1].y, p.w));
+            }
+          }
+          store_chunk32(v, stage_u32, lane, out_base, tl, q, c4, col_ok, args.ldo);
         }
-        __syncwarp();
+        if (warp == 4 && lane == 0) args.cnt[un.t] = 0;  // ready for the next launch
+        continue;
       }
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        store_chunk32(*reinterpret_cast<const float2(*)[16]>(acc + 16 * c4), stage_u32, lane,
+                      out_base, tl, q, c4, col_ok, args.ldo);
     }
     tc_fence_before();
   }

@@ -112,6 +112,37 @@ int fp8q_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t l
                          const void *wq, int64_t ldw, const void *sw, int sw_fmt, int64_t M,
                          int64_t N, int64_t K, void *out_bf16, int64_t ldo, cudaStream_t stream);
 
+/* The block-scaled GEMM above with its K dimension split over several CTAs per output tile, for
+ * shapes with too few 128 x 256 output tiles to occupy every SM (decode: M <= 128).  Split j of
+ * S takes the K-blocks [j * KB / S, (j + 1) * KB / S) (KB = K / 128), promotes them exactly as
+ * fp8q_gemm_w8a8_block does and writes its fp32 partial to `workspace`; the last split of a tile
+ * to finish adds the S partials in the order j = 0, 1, ..., S - 1 (deterministic, independent of
+ * which CTA finishes last) and writes bf16.  The result differs from fp8q_gemm_w8a8_block only
+ * in the fp32 summation order of the K-block terms and meets the same error bound.
+ *   splits           S in [1, K / 128]; 0 = chosen by the library (1 when the tiles already fill
+ *                    the SMs)
+ *   workspace        DEVICE memory of at least fp8q_gemm_splitk_workspace_bytes(M, N, K, splits)
+ *                    bytes, 16-byte aligned, owned by the caller; unused (may be NULL) when the
+ *                    resolved S is 1.  It must be ZEROED before its first use; every call that
+ *                    completes leaves it ready for the next call.  After FP8Q_ERR_TIMEOUT from
+ *                    fp8q_check_device_error it must be zeroed again.  Two calls that share a
+ *                    workspace must be ordered (same stream, or synchronized): concurrent calls
+ *                    on one workspace race.
+ * Other arguments, layouts and errors as fp8q_gemm_w8a8_block; splits out of range gives
+ * FP8Q_ERR_ARG, a workspace smaller than required FP8Q_ERR_SHAPE.  Source: the same passages as
+ * fp8q_gemm_w8a8_block (the split only reorders the fp32 promotion sum over K-blocks). */
+int fp8q_gemm_w8a8_block_splitk(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                                const void *wq, int64_t ldw, const void *sw, int sw_fmt,
+                                int64_t M, int64_t N, int64_t K, void *out_bf16, int64_t ldo,
+                                int splits, void *workspace, int64_t workspace_bytes,
+                                cudaStream_t stream);
+
+/* Workspace size in bytes for fp8q_gemm_w8a8_block_splitk with these sizes and `splits` (0 =
+ * the library's choice on the current device), written to *bytes (a HOST pointer); 0 when the
+ * resolved split count is 1. */
+int fp8q_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int splits,
+                                     int64_t *bytes);
+
 /* Grouped W8A8 GEMM for MoE experts (a6): for each expert e the rows
  * [group_offsets[e], group_offsets[e+1]) of aq/sa/out are multiplied by expert e's weight.
  *   wq             [E][N][ldw] uint8 codes (expert stride N * ldw)

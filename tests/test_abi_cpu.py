@@ -96,3 +96,29 @@ def test_valid_call_without_gpu_reports_arch(L):
         pytest.skip("a GPU is present")
     f = L.fp8q_quant_weight_block
     assert f(FAKE, 128, 128, 128, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_ERR_ARCH
+
+
+def test_splitk_host_checks(L):
+    g = L.fp8q_gemm_w8a8_block_splitk
+    ok = dict(aq=FAKE, lda=512, sa=FAKE, lds=64, wq=FAKE, ldw=512, sw=FAKE, fmt=0, M=64, N=256,
+              K=512, out=FAKE, ldo=256, splits=2, ws=FAKE, wsb=1 << 30)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["aq"], a["lda"], a["sa"], a["lds"], a["wq"], a["ldw"], a["sw"], a["fmt"],
+                 a["M"], a["N"], a["K"], a["out"], a["ldo"], a["splits"], a["ws"], a["wsb"], None)
+    assert call(splits=-1) == _lib.FP8Q_ERR_ARG
+    assert call(splits=5) == _lib.FP8Q_ERR_ARG          # more splits than K-blocks
+    assert call(N=100) == _lib.FP8Q_ERR_SHAPE
+    assert call(lda=520) == _lib.FP8Q_ERR_ALIGN
+    assert call(M=0, aq=None, sa=None, out=None, ws=None) == _lib.FP8Q_OK
+    q = L.fp8q_gemm_splitk_workspace_bytes
+    b = ctypes.c_int64(-1)
+    assert q(64, 256, 512, 2, ctypes.byref(b)) == _lib.FP8Q_OK
+    assert b.value == 2 * 128 * 256 * 4 + 16
+    assert q(300, 768, 4096, 3, ctypes.byref(b)) == _lib.FP8Q_OK
+    assert b.value == 9 * 3 * 128 * 256 * 4 + 48      # 9 tiles: counters padded to 16 B
+    assert q(64, 256, 512, 1, ctypes.byref(b)) == _lib.FP8Q_OK and b.value == 0
+    assert q(64, 256, 512, 5, ctypes.byref(b)) == _lib.FP8Q_ERR_ARG
+    assert q(64, 200, 512, 2, ctypes.byref(b)) == _lib.FP8Q_ERR_SHAPE
+    assert q(64, 256, 512, 2, None) == _lib.FP8Q_ERR_NULL
