@@ -16,6 +16,7 @@ FP8Q_ERR_ARCH = 4
 FP8Q_ERR_LAUNCH = 5
 FP8Q_ERR_TIMEOUT = 6
 FP8Q_ERR_ARG = 7
+FP8Q_ERR_TOO_LARGE = 8
 
 FP8Q_SCALE_F32 = 0
 FP8Q_SCALE_E8M0 = 1
@@ -32,6 +33,8 @@ SIGNATURES = {
                                   _I64, _P]),
     "fp8q_gemm_w8a8_block_splitk": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64, _I64,
                                          _P, _I64, _I, _P, _I64, _P]),
+    "fp8q_gemm_w8a8_block_splitk_noalloc": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64,
+                                                 _I64, _P, _I64, _I, _P]),
     "fp8q_gemm_splitk_workspace_bytes": (_I, [_I64, _I64, _I64, _I, ctypes.POINTER(_I64)]),
     "fp8q_grouped_gemm_w8a8_block": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _P, _I64, _I64,
                                           _I64, _I64, _P, _I64, _P]),

@@ -23,7 +23,14 @@ struct DeviceState {
   bool is_sm100 = false;
   int sms = 0;
   bool attrs_set = false;
+  void *static_scratch = nullptr;  // this device's address of g_splitk_static_scratch
 };
+
+// Split-K scratch owned by the library, for fp8q_gemm_w8a8_block_splitk_noalloc: 24 MiB of
+// fp32 partials (192 tile-splits of 128 x 256) plus one counter per tile (at most 192 tiles).
+constexpr int64_t kStaticPartialBytes = int64_t{24} << 20;
+constexpr int64_t kStaticScratchBytes = kStaticPartialBytes + 4096;
+__device__ __align__(256) uint8_t g_splitk_static_scratch[kStaticScratchBytes];
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
@@ -203,6 +210,7 @@ const char *fp8q_status_string(int status) {
     case FP8Q_ERR_LAUNCH: return "CUDA runtime or launch failure";
     case FP8Q_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (outputs incomplete)";
     case FP8Q_ERR_ARG: return "enum argument out of range";
+    case FP8Q_ERR_TOO_LARGE: return "problem needs more split-K scratch than the library's static 24 MiB buffer (use fp8q_gemm_w8a8_block_splitk with a workspace, or fewer splits)";
     default: return "unknown status";
   }
 }
@@ -338,6 +346,49 @@ int fp8q_gemm_w8a8_block_splitk(const void *aq, int64_t lda, const float *sa, in
   }
   return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K, out_bf16,
                      ldo, stream, s, s > 1 ? workspace : nullptr);
+}
+
+int fp8q_gemm_w8a8_block_splitk_noalloc(const void *aq, int64_t lda, const float *sa,
+                                        int64_t lds, const void *wq, int64_t ldw, const void *sw,
+                                        int sw_fmt, int64_t M, int64_t N, int64_t K,
+                                        void *out_bf16, int64_t ldo, int splits,
+                                        cudaStream_t stream) {
+  int rc = check_gemm_common(aq, lda, sa, lds, wq, ldw, sw, sw_fmt, M, N, K, out_bf16, ldo);
+  if (rc != FP8Q_OK) return rc;
+  if (splits < 0 || splits > K / 128) return FP8Q_ERR_ARG;
+  if (M == 0) return FP8Q_OK;
+  if (sw_fmt == FP8Q_SCALE_F32 && (reinterpret_cast<uintptr_t>(sw) & 3u)) return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  if ((rc = device_state(&st)) != FP8Q_OK) return rc;
+  const int s = resolve_splits(M, N, K, splits, st->sms);
+  if (s <= 0) return FP8Q_ERR_ARG;
+  const int64_t tiles = splitk_tiles(M, N);
+  if (tiles * s > INT32_MAX) return FP8Q_ERR_SHAPE;
+  if (s == 1)
+    return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K,
+                       out_bf16, ldo, stream);
+  if (tiles * s * kSplitPartialBytes > kStaticPartialBytes ||
+      tiles * 4 > kStaticScratchBytes - kStaticPartialBytes)
+    return FP8Q_ERR_TOO_LARGE;
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!st->static_scratch) {
+      // once per device, with that device current (device_state resolved the current device)
+      if (cudaGetSymbolAddress(&st->static_scratch, g_splitk_static_scratch) != cudaSuccess) {
+        st->static_scratch = nullptr;
+        return FP8Q_ERR_LAUNCH;
+      }
+    }
+    scratch = st->static_scratch;
+  }
+  // The kernel finds the partials at the start and the per-tile counters right after them;
+  // place the counters at the same offset and zero them on the stream before the launch.
+  uint8_t *counters = static_cast<uint8_t *>(scratch) + tiles * s * kSplitPartialBytes;
+  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(tiles) * 4, stream) != cudaSuccess)
+    return FP8Q_ERR_LAUNCH;
+  return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K, out_bf16,
+                     ldo, stream, s, scratch);
 }
 
 int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t lds,

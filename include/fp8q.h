@@ -66,7 +66,8 @@ typedef enum {
   FP8Q_ERR_ARCH = 4,    /* current device is not sm_100, or no device */
   FP8Q_ERR_LAUNCH = 5,  /* a CUDA runtime call or kernel launch failed */
   FP8Q_ERR_TIMEOUT = 6, /* (device error word) a kernel gave up on a bounded wait */
-  FP8Q_ERR_ARG = 7      /* an enum argument is out of range */
+  FP8Q_ERR_ARG = 7,     /* an enum argument is out of range */
+  FP8Q_ERR_TOO_LARGE = 8 /* the problem does not fit the library's static split-K scratch */
 } fp8q_status;
 
 typedef enum {
@@ -142,6 +143,31 @@ int fp8q_gemm_w8a8_block_splitk(const void *aq, int64_t lda, const float *sa, in
  * resolved split count is 1. */
 int fp8q_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int splits,
                                      int64_t *bytes);
+
+/* fp8q_gemm_w8a8_block_splitk without a caller workspace: the split-K partials and counters live
+ * in a fixed 24 MiB (+ 4 KiB) buffer that the library declares in its own device memory (reserved
+ * when the library's device code is loaded), so the call allocates nothing.  It serves callers
+ * that cannot allocate device memory at call time: an inference engine that hands all free HBM
+ * to its KV-cache pool at start-up and has no room left for per-call workspaces, or a caller that
+ * must not call cudaMalloc/cudaFree on its hot path because they can synchronize the device.
+ * The pages define no such variant; it computes exactly what fp8q_gemm_w8a8_block_splitk does
+ * (same kernel, same split order, bit-identical results for the same splits).
+ *   Limit: tiles * S <= 192 (tiles = ceil(M / 128) * ceil(N / 256), S the resolved split
+ *   count); beyond it FP8Q_ERR_TOO_LARGE.  Decode (M <= 128, N <= 12288) with
+ *   S <= 4 fits.  A resolved S of 1 runs fp8q_gemm_w8a8_block and touches no scratch.
+ *   The per-tile counters must start at zero: each call zeroes them on `stream`
+ *   (cudaMemsetAsync, no allocation) before its kernel.
+ *   The first call on each device looks the buffer's address up (cudaGetSymbolAddress, with
+ *   that device current); make that first call before any stream capture.
+ *   Each device has one such buffer (per process), shared by every caller: two calls on one
+ *   device that are not ordered with respect to each other (unsynchronized streams, host
+ *   threads) race on it and give wrong results.  Order them.
+ * Other arguments and errors as fp8q_gemm_w8a8_block_splitk. */
+int fp8q_gemm_w8a8_block_splitk_noalloc(const void *aq, int64_t lda, const float *sa,
+                                        int64_t lds, const void *wq, int64_t ldw, const void *sw,
+                                        int sw_fmt, int64_t M, int64_t N, int64_t K,
+                                        void *out_bf16, int64_t ldo, int splits,
+                                        cudaStream_t stream);
 
 /* Grouped W8A8 GEMM for MoE experts (a6): for each expert e the rows
  * [group_offsets[e], group_offsets[e+1]) of aq/sa/out are multiplied by expert e's weight.

@@ -33,7 +33,7 @@ def test_exports_match_header(L):
 
 
 def test_status_strings(L):
-    for s in range(8):
+    for s in range(9):
         assert len(_lib.status_string(s)) >= 2
     assert _lib.status_string(99) == "unknown status"
 
@@ -122,3 +122,12 @@ def test_splitk_host_checks(L):
     assert q(64, 256, 512, 5, ctypes.byref(b)) == _lib.FP8Q_ERR_ARG
     assert q(64, 200, 512, 2, ctypes.byref(b)) == _lib.FP8Q_ERR_SHAPE
     assert q(64, 256, 512, 2, None) == _lib.FP8Q_ERR_NULL
+
+
+def test_splitk_noalloc_host_checks(L):
+    g = L.fp8q_gemm_w8a8_block_splitk_noalloc
+    a = (FAKE, 512, FAKE, 64, FAKE, 512, FAKE, 0)
+    assert g(*a, 64, 256, 512, FAKE, 256, -1, None) == _lib.FP8Q_ERR_ARG
+    assert g(*a, 64, 256, 512, FAKE, 256, 5, None) == _lib.FP8Q_ERR_ARG
+    assert g(*a, 64, 200, 512, FAKE, 256, 2, None) == _lib.FP8Q_ERR_SHAPE
+    assert g(*a, 0, 256, 512, None, 256, 2, None) == _lib.FP8Q_OK
