@@ -12,11 +12,18 @@
 //   warp 1      TMEM allocator (whole warp) and MMA issuer (lane 0): 4 MMAs (K = 32 each) per
 //               K-block into one of two 256-column TMEM buffers, so the MMAs of K-block kb + 1
 //               run while the epilogue promotes K-block kb
-//   warp 2      scale producer: streams the activation scales sa of each K-block into a shared
-//               ring with cp.async (8 K-blocks ahead) and stages the weight scales of each tile
+//   warp 2      scale producer: stages the weight scales of each tile (both 128-column halves,
+//               all K-blocks) in shared memory, double-buffered across tiles; grouped: also
+//               streams the activation scales of each K-block into a shared ring with cp.async
+//               (8 K-blocks ahead)
 //   warp 3      idle (it completes warpgroup 0 for the register hand-off)
 //   warps 4-11  epilogue/promotion: warp w reads TMEM lanes 32 * (w % 4) (its 32 rows of the
-//               tile) and column half (w - 4) / 4; each thread keeps 128 fp32 accumulators
+//               tile) and column half (w - 4) / 4; each thread keeps 128 fp32 accumulators and
+//               (dense) loads its own row's activation scales from global memory two K-blocks
+//               ahead.
+//               Per K-block it reads its 128 columns as eight 16-column TMEM loads, promoting
+//               each chunk while the next load is in flight (the last chunk under the first load
+//               of the next K-block)
 // Registers: launched at 168 per thread (384 x 168 = 64512); warpgroup 0 drops to 64 and the two
 // epilogue warpgroups rise to 216 (128 x 64 + 256 x 216 = 63488 <= 64512; per sub-partition
 // 64 x 32 + 2 x 216 x 32 = 15872 <= 16128).
@@ -43,7 +50,7 @@ constexpr int kGroupM = 16;                       // rasterization: m-blocks per
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kTileABytes;
 constexpr int kOffStaging = kOffB + kStages * kTileBBytes;
-constexpr int kSaStages = 8;                      // K-blocks of activation scales in flight
+constexpr int kSaStages = 8;                      // grouped: K-blocks of activation scales in flight
 constexpr int kMaxKB = 256;                       // K <= 32768
 constexpr int kOffSa = kOffStaging + 8 * kStagingBytesPerWarp;      // [kSaStages][128] fp32
 constexpr int kOffSw = kOffSa + kSaStages * kBM * 4;                // [2 tiles][2 halves][kMaxKB]
@@ -167,6 +174,16 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// acc[j] += sc * (r[2j], r[2j + 1]) for j < 8: packed fp32x2 FMAs, round to nearest (the fp32
+// promotion of one 16-column chunk of a K-block partial).
+__device__ __forceinline__ void promote8(float2 *acc, const uint32_t (&r)[16], float sc) {
+  const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    acc[j] = __ffma2_rn(make_float2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1])), sc2,
+                        acc[j]);
 }
 
 // bf16 conversion and store of 32 columns (v[j] = columns 2j, 2j + 1 of chunk c4) of this
@@ -343,22 +360,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           s_sw[(tp * 2 + hh) * kMaxKB + kb] = v;
         }
         mbar_arrive(bar_swfull + 8 * tp);
-        // activation scales: one 128-row column of sa per K-block, zero-filled past row_end
-        const int rows_here = tl.row_end - tl.m0;
-        for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
-          const uint32_t s2 = it % kSaStages, ph2 = (it / kSaStages) & 1u;
-          if (!wait_warp(bar_saempty + 8 * s2, ph2 ^ 1u, s_abort)) { ok = false; break; }
-          const float *src = args.sa + static_cast<int64_t>(kb) * args.lds + tl.m0 + 4 * lane;
-          const uint32_t dst = smem_u32(s_sa + s2 * kBM + 4 * lane);
-          const int valid = max(0, min(4, rows_here - 4 * lane));
-          if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
-            cp_async_16_zfill(dst, valid > 0 ? src : args.sa, 4u * valid);
-          } else {
+        if constexpr (GROUPED) {
+          // activation scales: one 128-row column of sa per K-block, zero-filled past row_end
+          const int rows_here = tl.row_end - tl.m0;
+          for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
+            const uint32_t s2 = it % kSaStages, ph2 = (it / kSaStages) & 1u;
+            if (!wait_warp(bar_saempty + 8 * s2, ph2 ^ 1u, s_abort)) { ok = false; break; }
+            const float *src = args.sa + static_cast<int64_t>(kb) * args.lds + tl.m0 + 4 * lane;
+            const uint32_t dst = smem_u32(s_sa + s2 * kBM + 4 * lane);
+            const int valid = max(0, min(4, rows_here - 4 * lane));
+            if ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) {
+              cp_async_16_zfill(dst, valid > 0 ? src : args.sa, 4u * valid);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              cp_async_4(dst + 4 * i, i < valid ? src + i : args.sa, i < valid ? 4u : 0u);
+              for (int i = 0; i < 4; ++i)
+                cp_async_4(dst + 4 * i, i < valid ? src + i : args.sa, i < valid ? 4u : 0u);
+            }
+            cp_async_arrive_noinc(bar_safull + 8 * s2);
           }
-          cp_async_arrive_noinc(bar_safull + 8 * s2);
         }
       }
       cp_async_wait_all();
@@ -414,36 +433,66 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float2 acc[64];  // columns 2j, 2j + 1 of this thread's row
 #pragma unroll
       for (int j = 0; j < 64; ++j) acc[j] = make_float2(0.0f, 0.0f);
+      // Activation scales.  Dense: this thread loads its own row's scales from global memory
+      // two K-blocks ahead.  Grouped: the scale producer streams them through a shared ring
+      // (measured faster for the short, many-tile grouped problems).
+      const int row = tl.m0 + 32 * q + lane;
+      const bool row_ok = row < tl.row_end;
+      const float *sa_row = args.sa + row;
+      float sa0 = 0.0f, sa1 = 0.0f;
+      if constexpr (!GROUPED) {
+        sa0 = (row_ok && un.kb0 < un.kb1)
+                  ? __ldg(sa_row + static_cast<int64_t>(un.kb0) * args.lds) : 0.0f;
+        sa1 = (row_ok && un.kb0 + 1 < un.kb1)
+                  ? __ldg(sa_row + static_cast<int64_t>(un.kb0 + 1) * args.lds) : 0.0f;
+      }
+      uint32_t rb[16];  // the last chunk of the previous K-block, promoted under the next load
+      float sc_prev = 0.0f;
+      bool have_prev = false;
       for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
-        const uint32_t s2 = it % kSaStages, ph2 = (it / kSaStages) & 1u;
-        if (!wait_warp(bar_safull + 8 * s2, ph2, s_abort)) { ok = false; break; }
-        const float sc = __fmul_rn(s_sa[s2 * kBM + 32 * q + lane], sw_tile[kb]);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_saempty + 8 * s2);
+        float sa_cur;
+        if constexpr (GROUPED) {
+          const uint32_t s2 = it % kSaStages, ph2 = (it / kSaStages) & 1u;
+          if (!wait_warp(bar_safull + 8 * s2, ph2, s_abort)) { ok = false; break; }
+          sa_cur = s_sa[s2 * kBM + 32 * q + lane];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_saempty + 8 * s2);
+        } else {
+          sa_cur = sa0;
+          sa0 = sa1;
+          sa1 = (row_ok && kb + 2 < un.kb1)
+                    ? __ldg(sa_row + static_cast<int64_t>(kb + 2) * args.lds) : 0.0f;
+        }
+        const float sc = __fmul_rn(sa_cur, sw_tile[kb]);
         const uint32_t b = it & 1u, bph = (it >> 1) & 1u;
         if (!wait_warp(bar_tfull + 8 * b, bph, s_abort)) { ok = false; break; }
         tc_fence_after();
-        const float2 sc2 = make_float2(sc, sc);
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * kBN + h * 128;
-        // Two 64-column chunks: load, wait, promote.  The buffer is handed back to the MMA as
-        // soon as the second chunk is in registers.
+        // Eight 16-column chunks; the load of chunk c + 1 is in flight while chunk c is promoted.
+        // The buffer goes back to the MMA as soon as the last chunk is in registers.
+        uint32_t ra[16];
+        tmem_ld_32x32b_x16(taddr, ra);
+        if (have_prev) promote8(acc + 56, rb, sc_prev);
+        tmem_ld_wait(ra);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t r[64];
-          tmem_ld_32x32b_x64(taddr + 64 * c, r);
-          tmem_ld_wait(r);
-          if (c == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            acc[32 * c + j] = __ffma2_rn(make_float2(__uint_as_float(r[2 * j]),
-                                                     __uint_as_float(r[2 * j + 1])),
-                                         sc2, acc[32 * c + j]);
+        for (int c = 0; c < 3; ++c) {
+          tmem_ld_32x32b_x16(taddr + 32 * c + 16, rb);
+          promote8(acc + 16 * c, ra, sc);
+          tmem_ld_wait(rb);
+          tmem_ld_32x32b_x16(taddr + 32 * c + 32, ra);
+          promote8(acc + 16 * c + 8, rb, sc);
+          tmem_ld_wait(ra);
         }
+        tmem_ld_32x32b_x16(taddr + 112, rb);
+        promote8(acc + 48, ra, sc);
+        tmem_ld_wait(rb);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
+        sc_prev = sc;
+        have_prev = true;
       }
+      if (have_prev) promote8(acc + 56, rb, sc_prev);
       if (!ok) break;
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_swempty + 8 * tp);
