@@ -32,9 +32,30 @@ sys.path.insert(0, ROOT)
 
 M_, N_, K_ = 8192, 24576, 4096
 FLOPS = 2.0 * M_ * N_ * K_
+GEMM_BYTES = M_ * K_ + N_ * K_ + (K_ // 128) * M_ * 4 + (N_ // 128) * (K_ // 128) * 4 + M_ * N_ * 2
 METRIC = "blockwise W8A8 FP8 GEMM TFLOP/s (% FP8 peak); quant-kernel HBM GB/s (% peak)"
 WORKLOAD = "prefill linear: RMSNorm+1x128 quant of X[8192,4096] -> GEMM with W[24576,4096] requantized (128x128, fp32 scales) every step"
 L2_BYTES = 126 * 2 ** 20
+
+
+def gemm_traffic():
+    """DRAM bytes per launch of the dense GEMM on the bench's workload, as recorded from an ncu
+    capture in profiles/k_gemm_w8a8_block_prefill.md -- only while the kernel source is the one
+    that capture measured (else None)."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    src = os.path.join(here, "fp8_blockwise_w8a8_b200", "csrc", "gemm_kernel.cuh")
+    prof = os.path.join(here, "profiles", "k_gemm_w8a8_block_prefill.md")
+    try:
+        text = open(prof).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    except OSError:
+        return None
+    vals = dict(line.split(":", 1) for line in text.splitlines()
+                if line.startswith(("traffic_bytes_per_launch:", "source_sha256:")))
+    if vals.get("source_sha256", "").strip() != sha:
+        return None
+    return int(vals["traffic_bytes_per_launch"].strip())
 
 
 def peaks():
@@ -415,7 +436,10 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (step working set 0.8 GB > 126 MB)",
                        "rows_l2": "rows: between timed calls write 2 x L2 then read another 2 x L2 buffer (flush, no dirty lines left)"},
             "roofline": {"bound": "tensor", "achieved": gemm_tf, "peak": fp8_peak_sus,
-                         "unit": "TFLOP/s", "frac": gemm_tf / fp8_peak_sus, "traffic": None,
+                         "unit": "TFLOP/s", "frac": gemm_tf / fp8_peak_sus,
+                         "traffic": gemm_traffic(),
+                         "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
+                         "algorithmic_bytes": GEMM_BYTES,
                          "kernel": "k_gemm_w8a8_block<false>",
                          "peak_source": f"{pk['source']}: 2 x sustained cuBLAS bf16 "
                                         f"({pk['bf16_sustained']} TFLOP/s), the fp8/bf16 nominal ratio"},
@@ -492,6 +516,11 @@ def run_ncu_case(name):
         aq, sa = fq.rmsnorm_quant_token(randn((4096, K_), 1.0))
         wq, sw = fq.quant_weight_block(randn((N_, K_), 0.02), "f32")
         out = torch.empty((4096, N_), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm_w8a8_block(aq, sa, wq, sw, out=out)
+    elif name == "gemm_prefill_full":    # the bench's GEMM launch: M=8192 (A 34 MB, W 101 MB, out 403 MB)
+        aq, sa = fq.rmsnorm_quant_token(randn((M_, K_), 1.0))
+        wq, sw = fq.quant_weight_block(randn((N_, K_), 0.02), "f32")
+        out = torch.empty((M_, N_), dtype=torch.bfloat16, device=dev)
         fn = lambda: fq.gemm_w8a8_block(aq, sa, wq, sw, out=out)
     elif name == "gemm_decode":
         aq, sa = fq.rmsnorm_quant_token(randn((128, K_), 1.0))

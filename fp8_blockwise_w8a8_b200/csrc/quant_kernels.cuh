@@ -109,7 +109,7 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w) {
 // are within a relative 2^-23 + 3 * 2^-24 of x/s (1 -+ 2^-19), so they bracket x/s strictly.
 // RN_fp32 and the E4M3 conversion are both monotone, hence when the two bracket ends give the
 // same code, that code is the code of RN_fp32(x/s).  Otherwise (some x/s within ~2^-19 of an
-// E4M3 rounding boundary, exact ties included) the eight values are redone with IEEE divisions.
+// E4M3 rounding boundary, exact ties included) the tie rule or the fp64 quotient below decides.
 // Eight codes through an fp64 quotient, exact for every element: with r64 = RN64(1/s) the product
 // q64 = RN64(x * r64) is within 2^-52 (relative) of x/s.  If x/s is an fp32 number, RN32(q64) is
 // that number.  Otherwise x/s is at least ~2^-49 (relative) away from every fp32 rounding
