@@ -9,14 +9,15 @@
 // Structure (one persistent CTA per SM, 384 threads = 3 warpgroups):
 //   warp 0      TMA producer (lane 0): A tile 128 x 128 B and B tile 256 x 128 B per K-block into
 //               a 4-stage shared-memory ring, 128-byte swizzled
-//   warp 1      TMEM allocator (whole warp) and MMA issuer (lane 0): 4 MMAs (K = 32 each) per
-//               K-block into one of two 256-column TMEM buffers, so the MMAs of K-block kb + 1
-//               run while the epilogue promotes K-block kb
+//   warps 1, 3  MMA issuers (lane 0 of each): 4 MMAs (K = 32 each) per K-block into one of two
+//               256-column TMEM buffers, so the MMAs of K-block kb + 1 run while the epilogue
+//               promotes K-block kb.  Warp 1 issues the even K-blocks (buffer 0), warp 3 the odd
+//               ones (buffer 1): one thread's issue cost plus its barrier waits exceed the slack
+//               the tensor pipe leaves between K-blocks.  Warp 1 also allocates TMEM.
 //   warp 2      scale producer: stages the weight scales of each tile (both 128-column halves,
 //               all K-blocks) in shared memory, double-buffered across tiles; grouped: also
 //               streams the activation scales of each K-block into a shared ring with cp.async
 //               (8 K-blocks ahead)
-//   warp 3      idle (it completes warpgroup 0 for the register hand-off)
 //   warps 4-11  epilogue/promotion: warp w reads TMEM lanes 32 * (w % 4) (its 32 rows of the
 //               tile) and column half (w - 4) / 4; each thread keeps 128 fp32 accumulators and
 //               (dense) loads its own row's activation scales from global memory two K-blocks
@@ -261,7 +262,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(bar_tfull + 8 * i, 1);
       mbar_init(bar_tempty + 8 * i, 8);
     }
-    mbar_init(bar_done, 1);
+    mbar_init(bar_done, 2);
     for (int i = 0; i < kSaStages; ++i) {
       mbar_init(bar_safull + 8 * i, 32);
       mbar_init(bar_saempty + 8 * i, 8);
@@ -382,14 +383,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       cp_async_wait_all();
       __syncwarp();
-    } else if (warp == 1) {
-      // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 3) {
+      // ------------------------------------------------------------------ MMA issuers
+      // Two issuing threads: warp 1 takes the even K-blocks (TMEM buffer 0), warp 3 the odd ones
+      // (buffer 1), so each has two K-blocks of tensor-pipe time to cover its waits and issue.
       if (lane == 0) {
+        const uint32_t mine = warp == 3 ? 1u : 0u;
         uint32_t it = 0;
         for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
           const Unit un = unit_of(args, u, KB);
           bool ok = true;
           for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
+            if ((it & 1u) != mine) continue;
             const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
             const uint32_t b = it & 1u, bph = (it >> 1) & 1u;
             if (!wait_one(bar_tempty + 8 * b, bph ^ 1u, s_abort)) { ok = false; break; }
