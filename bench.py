@@ -38,6 +38,22 @@ WORKLOAD = "prefill linear: RMSNorm+1x128 quant of X[8192,4096] -> GEMM with W[2
 L2_BYTES = 126 * 2 ** 20
 
 
+def max_over_ranks(x, dist, device):
+    """The maximum of a per-rank float over all ranks (identity on one rank).  Every rank must call
+    it at the same point: it is a collective."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world, ms_per_step):
+    """Whole-job throughput: every rank runs one step of the workload (weak scaling), so the job
+    does world x FLOPS per step in the slowest rank's step time."""
+    return world * FLOPS / (ms_per_step / 1e3) / 1e12
+
+
 def gemm_traffic():
     """DRAM bytes per launch of the dense GEMM on the bench's workload, as recorded from an ncu
     capture in profiles/k_gemm_w8a8_block_prefill.md -- only while the kernel source is the one
@@ -357,11 +373,7 @@ def run_ours(args):
     clk = clocks.stop()
     if dist is not None:
         dist.barrier()
-    ms_total = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([ms_total], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dist, device)
     ms_step = ms_total / args.steps
     k_req = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     k_rms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
@@ -386,10 +398,7 @@ def run_ours(args):
         oh.copy_(step.out, non_blocking=True)
     e2e_steps = max(3, args.steps // 2)
     ms_e2e, _ = timed_loop(e2e_step, e2e_steps, max(1, args.warmup // 2))
-    if dist is not None:
-        t = torch.tensor([ms_e2e], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ms_e2e, dist, device)
     h2d = xh.numel() * 2 + wh.numel() * 2 + gh.numel() * 2
     d2h = oh.numel() * 2
 
@@ -419,7 +428,7 @@ def run_ours(args):
         gemm_tf = FLOPS / k_gemm / 1e9
         line = {
             "metric": METRIC,
-            "value": world * FLOPS / (ms_step / 1e3) / 1e12,
+            "value": whole_job_tflops(world, ms_step),
             "unit": "TFLOP/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -443,7 +452,7 @@ def run_ours(args):
                          "kernel": "k_gemm_w8a8_block<false>",
                          "peak_source": f"{pk['source']}: 2 x sustained cuBLAS bf16 "
                                         f"({pk['bf16_sustained']} TFLOP/s), the fp8/bf16 nominal ratio"},
-            "e2e": {"value": world * FLOPS / (ms_e2e / 1e3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": whole_job_tflops(world, ms_e2e), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": ms_e2e},
             "cpu_baseline": cpu,
