@@ -261,25 +261,18 @@ __device__ __forceinline__ QParams qparams_tab(float amax, const ScaleTab *t) {
 // ---------------------------------------------------------------------------------------------
 // 1x128 token groups, optionally preceded by RMSNorm.  One warp per row at a time.
 //
-// With RMSNorm the row is staged in shared memory (cp.async) in a padded layout -- 128-element
-// blocks at a 272-byte stride -- so that lane b can walk its own block b in ascending k for the
-// fp64 sum of squares without bank conflicts.  gamma is held once per CTA as fp32, split per
-// 16-byte chunk j into gA[j] (elements 8j..8j+3) and gB[j] (8j+4..8j+7).  Without RMSNorm
-// nothing is staged: the quantization reads the row straight from global memory.  In both
-// cases the next row of the warp is prefetched into L2 while the current one is processed.
+// RMSNorm, phase 1: lane l owns the 128-blocks l, l + 32, ... of the row and reads each one from
+// global memory (L1-cached; the row was prefetched into L2 while the previous row was processed)
+// to form the fp64 sum of squares of the block in ascending k.  The block sums go through a small
+// per-warp shared-memory area and lane 0 adds them in ascending block order, then forms r.
+// Phase 2 re-reads the row (now in L1/L2) for the quantization.  gamma is held once per CTA as
+// fp32, split per 16-byte chunk j into gA[j] (elements 8j..8j+3) and gB[j] (8j+4..8j+7).
 //
-// Quantization: LPB lanes per 128-block (8 with RMSNorm, reading the staged row without bank
-// conflicts; 4 without, reading global memory), 32 / LPB blocks per warp step; lane `sub` of a
-// block owns the 16-byte chunks sub + LPB c, c = 0 .. 16 / LPB - 1.
+// Quantization: LPB lanes per 128-block (8 with RMSNorm, so that the gamma reads are free of bank
+// conflicts; 4 without), 32 / LPB blocks per warp step; lane `sub` of a block owns the 16-byte
+// chunks sub + LPB c, c = 0 .. 16 / LPB - 1.  The loads of the next step are issued before the
+// current step is processed.
 // ---------------------------------------------------------------------------------------------
-constexpr int kRowBlockStride = 272;
-
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
 __device__ __forceinline__ void prefetch_l2(const void *p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
@@ -306,10 +299,30 @@ __device__ __forceinline__ uint4 rms_apply8(const uint4 v, float r, const float4
   return make_uint4(y[0], y[1], y[2], y[3]);
 }
 
+// fp64 sum of squares of one 128-element bf16 block, in ascending k.
+__device__ __forceinline__ double block_sumsq(const uint16_t *blk) {
+  const uint4 *p = reinterpret_cast<const uint4 *>(blk);
+  uint4 v[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) v[c] = p[c];
+  double acc = 0.0;
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const uint32_t wv[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const double a = static_cast<double>(bf16_lo(wv[j]));
+      acc = __fma_rn(a, a, acc);  // a*a is exact in fp64, so this is RN(acc + a*a)
+      const double b2 = static_cast<double>(bf16_hi(wv[j]));
+      acc = __fma_rn(b2, b2, acc);
+    }
+  }
+  return acc;
+}
+
 // Shared-memory bytes of the token kernel.
 __host__ __device__ constexpr int token_smem_bytes(int K, bool norm, int wpc) {
-  return static_cast<int>(sizeof(ScaleTab)) +
-         (norm ? K * 4 + wpc * (K / 128) * kRowBlockStride : 0);
+  return static_cast<int>(sizeof(ScaleTab)) + (norm ? K * 4 + wpc * (K / 128) * 8 : 0);
 }
 
 template <bool NORM>
@@ -323,12 +336,10 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int wpc = blockDim.x >> 5;
   const int KB = K >> 7;
-  const int row_bytes = KB * kRowBlockStride;
   ScaleTab *tab = reinterpret_cast<ScaleTab *>(smem);
   float4 *gA = reinterpret_cast<float4 *>(smem + sizeof(ScaleTab));
   float4 *gB = gA + (K >> 3);
-  uint8_t *row = smem + sizeof(ScaleTab) + K * 4 + warp * row_bytes;  // NORM only
-  const uint32_t row_u32 = smem_u32(row);
+  double *wsum = reinterpret_cast<double *>(smem + sizeof(ScaleTab) + K * 4) + warp * KB;  // NORM
   const int grp = lane / LPB, sub = lane % LPB;
 
   build_scale_tab(tab, threadIdx.x, blockDim.x);
@@ -352,55 +363,28 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
 
     float r = 1.0f;
     if (NORM) {
-      for (int j = lane; j < (K >> 3); j += 32)
-        cp_async_16(row_u32 + (j >> 4) * kRowBlockStride + (j & 15) * 16, xr + j * 8);
-      cp_async_commit_wait_all();
+      // Sum of squares in fp64: each lane takes its own 128-blocks in ascending k ...
+      for (int b = lane; b < KB; b += 32) wsum[b] = block_sumsq(xr + b * 128);
       __syncwarp();
-      // Sum of squares in fp64: each lane walks its own 128-blocks in ascending k ...
-      double P[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        P[t] = 0.0;
-        const int b = lane + 32 * t;
-        if (b < KB) {
-          const uint4 *blk = reinterpret_cast<const uint4 *>(row + b * kRowBlockStride);
-          double acc = 0.0;
-#pragma unroll 4
-          for (int c = 0; c < 16; ++c) {
-            const uint4 v = blk[c];
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const double a = static_cast<double>(bf16_lo(wv[j]));
-              acc = __fma_rn(a, a, acc);  // a*a is exact in fp64, so this is RN(acc + a*a)
-              const double b2 = static_cast<double>(bf16_hi(wv[j]));
-              acc = __fma_rn(b2, b2, acc);
-            }
-          }
-          P[t] = acc;
-        }
+      // ... then lane 0 adds the block sums in ascending block order.
+      if (lane == 0) {
+        double S = 0.0;
+        for (int b = 0; b < KB; ++b) S = __dadd_rn(S, wsum[b]);
+        const double var = __dadd_rn(__ddiv_rn(S, static_cast<double>(K)), static_cast<double>(eps));
+        r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(var)));
       }
-      // ... then the block sums are added in ascending block order.
-      double S = 0.0;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        if (32 * t >= KB) break;
-#pragma unroll 8
-        for (int j = 0; j < 32; ++j) {
-          const double pj = __shfl_sync(0xffffffffu, P[t], j);
-          if (32 * t + j < KB) S = __dadd_rn(S, pj);
-        }
-      }
-      const double var = __dadd_rn(__ddiv_rn(S, static_cast<double>(K)), static_cast<double>(eps));
-      r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(var)));
+      r = __shfl_sync(0xffffffffu, r, 0);
     }
 
-    // Without RMSNorm the loads of the next step are issued before this step is processed.
+    // The loads of the next step are issued before the current step is processed.
     uint4 vn[CPL];
-    if (!NORM) {
+    {
       const int bb = grp < KB ? grp : 0;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) vn[c] = ld_stream_v4(xr + bb * 128 + (sub + LPB * c) * 8);
+      for (int c = 0; c < CPL; ++c) {
+        const uint16_t *src = xr + bb * 128 + (sub + LPB * c) * 8;
+        vn[c] = NORM ? *reinterpret_cast<const uint4 *>(src) : ld_stream_v4(src);
+      }
     }
 #pragma unroll 2
     for (int b0 = 0; b0 < KB; b0 += BPS) {
@@ -411,17 +395,15 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
         const int chunk = sub + LPB * c;
-        if (NORM) {
-          v[c] = *reinterpret_cast<const uint4 *>(row + bb * kRowBlockStride + chunk * 16);
-          v[c] = rms_apply8(v[c], r, gA[bb * 16 + chunk], gB[bb * 16 + chunk]);
-        } else {
-          v[c] = vn[c];
-        }
+        v[c] = NORM ? rms_apply8(vn[c], r, gA[bb * 16 + chunk], gB[bb * 16 + chunk]) : vn[c];
       }
-      if (!NORM && b0 + BPS < KB) {
+      if (b0 + BPS < KB) {
         const int bn = b0 + BPS + grp < KB ? b0 + BPS + grp : b0 + BPS;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) vn[c] = ld_stream_v4(xr + bn * 128 + (sub + LPB * c) * 8);
+        for (int c = 0; c < CPL; ++c) {
+          const uint16_t *src = xr + bn * 128 + (sub + LPB * c) * 8;
+          vn[c] = NORM ? *reinterpret_cast<const uint4 *>(src) : ld_stream_v4(src);
+        }
       }
       uint32_t m2 = 0u;
 #pragma unroll
@@ -437,7 +419,7 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
       }
       if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
     }
-    __syncwarp();  // every lane is done with the staged row before it is refilled
+    __syncwarp();  // lane 0 has read every block sum before they are overwritten
   }
 }
 
