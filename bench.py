@@ -245,19 +245,31 @@ def measure_rows(fq, device, steps, warmup, pk):
     out = torch.empty((128, 12288), dtype=torch.bfloat16, device=device)
     byts = 12288 * 4096 + 128 * 4096 + 128 * 32 * 4 + 96 * 32 * 4 + 128 * 12288 * 2
     fl = 2.0 * 128 * 12288 * 4096
-    ws = fq.splitk_workspace(128, 12288, 4096, 0, device=device)
-    splits = max(1, ws.numel() // (48 * 128 * 256 * 4))
-    for name, fn in (("a5_gemm_decode",
-                      lambda: fq.gemm_w8a8_block_splitk(aq, sa, wq, sw, splits=0, workspace=ws,
-                                                        out=out)),
-                     ("a5_gemm_decode_unsplit",
-                      lambda: fq.gemm_w8a8_block(aq, sa, wq, sw, out=out))):
+    ms, _ = timed_loop(lambda: fq.gemm_w8a8_block(aq, sa, wq, sw, out=out), steps, warmup, flush)
+    rows["a5_gemm_decode"] = {"ms": ms, "TFLOP/s": fl / ms / 1e9, "GB/s": byts / ms / 1e6,
+                              "frac_hbm": byts / ms / 1e6 / hbm, "bound": "hbm", "splits": 1,
+                              "workload": "M=128 N=12288 K=4096"}
+    # decode down projection (long K, few tiles): split-K with the library's choice vs unsplit
+    Md, Nd, Kd = 128, 4096, 12288
+    ad = dev_bf16(inputs.randn_bf16((Md, Kd), 1.0, 90, 0), device)
+    wd = dev_bf16(inputs.randn_bf16((Nd, Kd), 0.02, 90, 1), device)
+    wqd, swd = fq.quant_weight_block(wd, "f32")
+    aqd, sad = fq.rmsnorm_quant_token(ad)
+    outd = torch.empty((Md, Nd), dtype=torch.bfloat16, device=device)
+    wsd = fq.splitk_workspace(Md, Nd, Kd, 0, device=device)
+    splits = max(1, wsd.numel() // (16 * 128 * 256 * 4))
+    bd = Nd * Kd + Md * Kd + Md * (Kd // 128) * 4 + (Nd // 128) * (Kd // 128) * 4 + Md * Nd * 2
+    fd = 2.0 * Md * Nd * Kd
+    for name, fn, sp in (("a5_gemm_decode_down_splitk",
+                          lambda: fq.gemm_w8a8_block_splitk(aqd, sad, wqd, swd, splits=0,
+                                                            workspace=wsd, out=outd), splits),
+                         ("a5_gemm_decode_down_unsplit",
+                          lambda: fq.gemm_w8a8_block(aqd, sad, wqd, swd, out=outd), 1)):
         ms, _ = timed_loop(fn, steps, warmup, flush)
-        rows[name] = {"ms": ms, "TFLOP/s": fl / ms / 1e9, "GB/s": byts / ms / 1e6,
-                      "frac_hbm": byts / ms / 1e6 / hbm, "bound": "hbm",
-                      "splits": splits if name == "a5_gemm_decode" else 1,
-                      "workload": "M=128 N=12288 K=4096"}
-    del ws
+        rows[name] = {"ms": ms, "TFLOP/s": fd / ms / 1e9, "GB/s": bd / ms / 1e6,
+                      "frac_hbm": bd / ms / 1e6 / hbm, "bound": "hbm", "splits": sp,
+                      "workload": f"M={Md} N={Nd} K={Kd}"}
+    del ad, wd, wqd, swd, aqd, sad, outd, wsd
     ms, _ = timed_loop(lambda: fq.rmsnorm_quant_token(a, out_q=aq, out_sa=sa), steps, warmup,
                        flush)
     byts = 128 * 4096 * 3 + 128 * 32 * 4

@@ -105,17 +105,18 @@ def gemm_splitk_workspace_bytes(M: int, N: int, K: int, splits: int = 0) -> int:
 
 
 def splitk_workspace(M: int, N: int, K: int, splits: int = 0, device=None) -> torch.Tensor:
-    """A zeroed workspace for gemm_w8a8_block_splitk; reusable by later calls in stream order."""
+    """A workspace for gemm_w8a8_block_splitk (no initialisation needed); reusable by later calls
+    in stream order."""
     n = gemm_splitk_workspace_bytes(M, N, K, splits)
-    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
 
 
 def gemm_w8a8_block_splitk(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor,
                            sw: torch.Tensor, fmt=None, splits: int = 0, workspace=None, out=None,
                            stream=None):
-    """gemm_w8a8_block with K split over several CTAs per output tile.  `workspace` is a zeroed
-    uint8 device tensor of gemm_splitk_workspace_bytes(M, N, K, splits) bytes, reused across
-    calls on one stream; None allocates a fresh one."""
+    """gemm_w8a8_block with K split over several CTAs per output tile.  `workspace` is a uint8
+    device tensor of gemm_splitk_workspace_bytes(M, N, K, splits) bytes, reused across calls on
+    one stream; None allocates a fresh one."""
     f = scale_format(sw.dtype if fmt is None else fmt)
     M, K = aq.shape
     N = wq.shape[0]

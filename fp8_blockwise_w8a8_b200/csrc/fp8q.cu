@@ -27,9 +27,8 @@ struct DeviceState {
 };
 
 // Split-K scratch owned by the library, for fp8q_gemm_w8a8_block_splitk_noalloc: 24 MiB of
-// fp32 partials (192 tile-splits of 128 x 256) plus one counter per tile (at most 192 tiles).
-constexpr int64_t kStaticPartialBytes = int64_t{24} << 20;
-constexpr int64_t kStaticScratchBytes = kStaticPartialBytes + 4096;
+// fp32 partials (192 tile-splits of 128 x 256).
+constexpr int64_t kStaticScratchBytes = int64_t{24} << 20;
 __device__ __align__(256) uint8_t g_splitk_static_scratch[kStaticScratchBytes];
 
 std::mutex g_mu;
@@ -121,8 +120,7 @@ int check_gemm_common(const void *aq, int64_t lda, const float *sa, int64_t lds,
   return FP8Q_OK;
 }
 
-// Split-K workspace: fp32 partials of one 128 x 256 tile per (tile, split), then one int32
-// arrival counter per tile.
+// Split-K workspace: fp32 partials of one 128 x 256 tile per (tile, split).
 constexpr int64_t kSplitPartialBytes = int64_t{fp8q::kBM} * fp8q::kBN * 4;
 
 int64_t splitk_tiles(int64_t M, int64_t N) {
@@ -131,21 +129,32 @@ int64_t splitk_tiles(int64_t M, int64_t N) {
 
 int64_t splitk_workspace_bytes(int64_t M, int64_t N, int splits) {
   if (splits <= 1) return 0;
-  const int64_t tiles = splitk_tiles(M, N);
-  return tiles * splits * kSplitPartialBytes + ((tiles * 4 + 15) / 16) * 16;
+  return splitk_tiles(M, N) * splits * kSplitPartialBytes;
 }
 
-// splits = 0 picks the K-split count: 1 when the tiles alone fill the SMs, else as many splits as
-// fit the SMs, each keeping at least 4 K-blocks.  Returns a count in [1, K/128] or 0 on error.
+// splits = 0 picks the K-split count from a cost model fitted to B200 measurements of this
+// kernel (decode-sized M): time(S) ~ KB / S * t_kb + (S > 1 ? t_red + t_part * tiles * S : 0),
+// with t_kb = 0.6 us per K-block of one CTA, t_red = 4.6 us for the reduction launch and
+// t_part = 0.064 us per 128 x 256 fp32 partial written and re-read.  S is limited to one wave
+// (tiles * S <= SMs).  Returns a count in [1, K/128] or 0 on error.
 int resolve_splits(int64_t M, int64_t N, int64_t K, int splits, int sms) {
   const int64_t KB = K / fp8q::kBK;
   if (splits < 0 || splits > KB) return 0;
   if (splits > 0) return splits;
   const int64_t tiles = splitk_tiles(M, N);
   if (tiles <= 0 || tiles * 2 > sms) return 1;
-  int64_t s = sms / tiles;
-  if (s > KB / 4) s = KB / 4;
-  return static_cast<int>(s < 1 ? 1 : s);
+  constexpr double t_kb = 0.6, t_red = 4.6, t_part = 0.064;
+  int best = 1;
+  double best_t = static_cast<double>(KB) * t_kb;
+  for (int64_t s = 2; s <= KB && tiles * s <= sms; ++s) {
+    const double t = static_cast<double>((KB + s - 1) / s) * t_kb + t_red +
+                     t_part * static_cast<double>(tiles * s);
+    if (t < best_t) {
+      best_t = t;
+      best = static_cast<int>(s);
+    }
+  }
+  return best;
 }
 
 int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int64_t lds,
@@ -177,12 +186,8 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
   a.num_m = static_cast<int>((M + fp8q::kBM - 1) / fp8q::kBM);
   a.splits = splits;
   a.ws = static_cast<float *>(workspace);
-  a.cnt = nullptr;
   // Upper bound of the tile count (grouped: every expert may add one partial m-tile).
   const int64_t tiles = (static_cast<int64_t>(a.num_m) + (grouped ? E : 0)) * a.num_n;
-  if (splits > 1)
-    a.cnt = reinterpret_cast<int *>(static_cast<uint8_t *>(workspace) +
-                                    tiles * splits * kSplitPartialBytes);
   const int64_t units = tiles * splits;
   const int grid = static_cast<int>(units < st->sms ? units : st->sms);
   if (grouped)
@@ -191,6 +196,11 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
   else
     fp8q::k_gemm_w8a8_block<false><<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemDense, stream>>>(
         tm_a, tm_b, a);
+  if (splits > 1 && !grouped) {
+    if ((rc = launch_status()) != FP8Q_OK) return rc;
+    fp8q::k_splitk_reduce<<<static_cast<unsigned>(tiles * 8), fp8q::kReduceThreads, 0, stream>>>(
+        static_cast<const float4 *>(workspace), splits, a.num_m, a.num_n, a.M, a.N, a.out, ldo);
+  }
   return launch_status();
 }
 
@@ -367,9 +377,7 @@ int fp8q_gemm_w8a8_block_splitk_noalloc(const void *aq, int64_t lda, const float
   if (s == 1)
     return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K,
                        out_bf16, ldo, stream);
-  if (tiles * s * kSplitPartialBytes > kStaticPartialBytes ||
-      tiles * 4 > kStaticScratchBytes - kStaticPartialBytes)
-    return FP8Q_ERR_TOO_LARGE;
+  if (tiles * s * kSplitPartialBytes > kStaticScratchBytes) return FP8Q_ERR_TOO_LARGE;
   void *scratch = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
@@ -382,11 +390,6 @@ int fp8q_gemm_w8a8_block_splitk_noalloc(const void *aq, int64_t lda, const float
     }
     scratch = st->static_scratch;
   }
-  // The kernel finds the partials at the start and the per-tile counters right after them;
-  // place the counters at the same offset and zero them on the stream before the launch.
-  uint8_t *counters = static_cast<uint8_t *>(scratch) + tiles * s * kSplitPartialBytes;
-  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(tiles) * 4, stream) != cudaSuccess)
-    return FP8Q_ERR_LAUNCH;
   return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K, out_bf16,
                      ldo, stream, s, scratch);
 }

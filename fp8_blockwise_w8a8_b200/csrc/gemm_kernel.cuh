@@ -56,10 +56,9 @@ constexpr int kMaxKB = 256;                       // K <= 32768
 constexpr int kOffSa = kOffStaging + 8 * kStagingBytesPerWarp;      // [kSaStages][128] fp32
 constexpr int kOffSw = kOffSa + kSaStages * kBM * 4;                // [2 tiles][2 halves][kMaxKB]
 constexpr int kOffBar = kOffSw + 2 * 2 * kMaxKB * 4;
-// full, empty, tmem_full[2], tmem_empty[2], done, sa_full/empty[kSaStages], sw_full/empty[2],
-// split-K handshake ep1, ep2
-constexpr int kNumBars = 2 * kStages + 4 + 1 + 2 * kSaStages + 4 + 2;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag, split-K last flag
+// full, empty, tmem_full[2], tmem_empty[2], done, sa_full/empty[kSaStages], sw_full/empty[2]
+constexpr int kNumBars = 2 * kStages + 4 + 1 + 2 * kSaStages + 4;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
 constexpr int kOffGroups = kOffMisc + 16;          // grouped: offsets[E+1], tile prefix[E+1]
 constexpr int kGemmSmemDense = kOffGroups + 1024;  // + alignment slack
 constexpr int kGemmSmemGrouped = kOffGroups + 2 * (kMaxExperts + 1) * 4 + 1024;
@@ -92,7 +91,6 @@ struct GemmArgs {
   int num_m;            // dense: ceil(M / 128)
   int splits;           // K-splits per tile (1: no split)
   float *ws;            // splits > 1: fp32 partials, [tile][split][2][32][128] float4
-  int *cnt;             // splits > 1: one arrival counter per tile, zero between launches
 };
 
 // Work unit u covers tile u / splits and the K-blocks [kb0, kb1) of split u % splits.
@@ -241,9 +239,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t bar_saempty = bar_safull + 8 * kSaStages;    // [kSaStages]
   const uint32_t bar_swfull = bar_saempty + 8 * kSaStages;    // [2]
   const uint32_t bar_swempty = bar_swfull + 16;               // [2]
-  const uint32_t bar_ep1 = bar_swempty + 16;                  // epilogue warps -> leader
-  const uint32_t bar_ep2 = bar_ep1 + 8;                       // leader -> epilogue warps
-  volatile int *s_last = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
   float *s_sa = reinterpret_cast<float *>(smem + kOffSa);
   float *s_sw = reinterpret_cast<float *>(smem + kOffSw);
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + kOffMisc);
@@ -271,8 +266,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(bar_swfull + 8 * i, 32);
       mbar_init(bar_swempty + 8 * i, 8);
     }
-    mbar_init(bar_ep1, 8);
-    mbar_init(bar_ep2, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -503,53 +496,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (lane == 0) mbar_arrive(bar_swempty + 8 * tp);
       uint16_t *out_base = args.out + static_cast<int64_t>(tl.n0 + 128 * h);
       if (args.splits > 1) {
-        // Split K: publish this split's fp32 partial, count arrivals per tile; the last split to
-        // arrive adds all partials in split order (a fixed order: deterministic) and stores.
+        // Split K: this unit's fp32 partial goes to the workspace (coalesced: lane = row); the
+        // partials of a tile are added in split order by k_splitk_reduce, launched next.
         const int rl = 32 * q + lane;
-        float4 *ws_tile = reinterpret_cast<float4 *>(args.ws) +
-                          static_cast<size_t>(un.t) * args.splits * (2 * 32 * 128);
-        float4 *mine = ws_tile + static_cast<size_t>(un.j) * (2 * 32 * 128) + (h * 32) * 128 + rl;
+        float4 *mine = reinterpret_cast<float4 *>(args.ws) +
+                       (static_cast<size_t>(un.t) * args.splits + un.j) * (2 * 32 * 128) +
+                       (h * 32) * 128 + rl;
 #pragma unroll
         for (int c = 0; c < 32; ++c)
           __stcg(mine + c * 128, make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x,
                                              acc[2 * c + 1].y));
-        __threadfence();
-        __syncwarp();
-        const uint32_t pu = (tile_it & 1u);  // one handshake per unit: parity alternates
-        if (lane == 0) mbar_arrive(bar_ep1);
-        if (warp == 4) {
-          if (!wait_warp(bar_ep1, pu, s_abort)) { ok = false; break; }
-          if (lane == 0) {
-            const int prev = atomicAdd(args.cnt + un.t, 1);
-            __threadfence();
-            *s_last = (prev == args.splits - 1) ? 1 : 0;
-            mbar_arrive(bar_ep2);
-          }
-          __syncwarp();
-        }
-        if (!wait_warp(bar_ep2, pu, s_abort)) { ok = false; break; }
-        if (!*s_last) continue;
-        // Sum the partials (this CTA's own included, re-read from L2) 32 columns at a time.
-        const float4 *col = ws_tile + (h * 32) * 128 + rl;
-#pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float2 v[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) v[c] = make_float2(0.0f, 0.0f);
-#pragma unroll 1
-          for (int i = 0; i < args.splits; ++i) {
-            const float4 *src = col + static_cast<size_t>(i) * (2 * 32 * 128) + (8 * c4) * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float4 p = __ldcg(src + c * 128);
-              v[2 * c] = make_float2(__fadd_rn(v[2 * c].x, p.x), __fadd_rn(v[2 * c].y, p.y));
-              v[2 * c + 1] = make_float2(__fadd_rn(v[2 * c + 1].x, p.z),
-                                         __fadd_rn(v[2 * c + 1].y, p.w));
-            }
-          }
-          store_chunk32(v, stage_u32, lane, out_base, tl, q, c4, col_ok, args.ldo);
-        }
-        if (warp == 4 && lane == 0) args.cnt[un.t] = 0;  // ready for the next launch
         continue;
       }
 #pragma unroll
@@ -565,6 +521,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }
+}
+
+// Split-K reduction: out[m, n] = bf16( sum over j = 0 .. S - 1, in that order, of partial_j ).
+// Partials: [tile][split][half h][chunk c][row r] float4 = columns 128 h + 4 c .. + 3 of row r.
+// Grid: 8 CTAs of 256 threads per dense tile; thread (r, g) adds row r, columns 16 g .. 16 g + 15
+// (4 float4 per split, read coalesced across rows) and writes 32 contiguous output bytes.
+constexpr int kReduceThreads = 256;
+__global__ void __launch_bounds__(kReduceThreads)
+    k_splitk_reduce(const float4 *__restrict__ ws, int splits, int num_m, int num_n, int M, int N,
+                    uint16_t *__restrict__ out, int64_t ldo) {
+  const int t = blockIdx.x >> 3;                  // dense tile, same order as dense_tile()
+  const int r = threadIdx.x & 127;
+  const int g = ((blockIdx.x & 7) << 1) | (threadIdx.x >> 7);  // 16-column group, 0 .. 15
+  GemmArgs a{};
+  a.num_m = num_m;
+  a.num_n = num_n;
+  a.M = M;
+  const Tile tl = dense_tile(a, t);
+  const int row = tl.m0 + r, col = tl.n0 + 16 * g;
+  if (row >= M || col >= N) return;
+  const int h = g >> 3, c0 = (g & 7) * 4;
+  const float4 *p = ws + static_cast<size_t>(t) * splits * (2 * 32 * 128) + (h * 32 + c0) * 128 + r;
+  float4 sum[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sum[i] = __ldcg(p + i * 128);
+  for (int j = 1; j < splits; ++j) {
+    const float4 *pj = p + static_cast<size_t>(j) * (2 * 32 * 128);
+    float4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = __ldcg(pj + i * 128);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      sum[i] = make_float4(__fadd_rn(sum[i].x, v[i].x), __fadd_rn(sum[i].y, v[i].y),
+                           __fadd_rn(sum[i].z, v[i].z), __fadd_rn(sum[i].w, v[i].w));
+  }
+  uint32_t pk[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(sum[i].x, sum[i].y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(sum[i].z, sum[i].w);
+    pk[2 * i] = *reinterpret_cast<const uint32_t *>(&lo);
+    pk[2 * i + 1] = *reinterpret_cast<const uint32_t *>(&hi);
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(out + static_cast<int64_t>(row) * ldo + col);
+  dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
 }  // namespace fp8q

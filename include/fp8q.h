@@ -116,19 +116,17 @@ int fp8q_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t l
 /* The block-scaled GEMM above with its K dimension split over several CTAs per output tile, for
  * shapes with too few 128 x 256 output tiles to occupy every SM (decode: M <= 128).  Split j of
  * S takes the K-blocks [j * KB / S, (j + 1) * KB / S) (KB = K / 128), promotes them exactly as
- * fp8q_gemm_w8a8_block does and writes its fp32 partial to `workspace`; the last split of a tile
- * to finish adds the S partials in the order j = 0, 1, ..., S - 1 (deterministic, independent of
- * which CTA finishes last) and writes bf16.  The result differs from fp8q_gemm_w8a8_block only
- * in the fp32 summation order of the K-block terms and meets the same error bound.
+ * fp8q_gemm_w8a8_block does and writes its fp32 partial to `workspace`; a second kernel on the
+ * same stream then adds the S partials of each tile in the order j = 0, 1, ..., S - 1
+ * (deterministic) and writes bf16.  The result differs from fp8q_gemm_w8a8_block only in the
+ * fp32 summation order of the K-block terms and meets the same error bound.
  *   splits           S in [1, K / 128]; 0 = chosen by the library (1 when the tiles already fill
  *                    the SMs)
  *   workspace        DEVICE memory of at least fp8q_gemm_splitk_workspace_bytes(M, N, K, splits)
  *                    bytes, 16-byte aligned, owned by the caller; unused (may be NULL) when the
- *                    resolved S is 1.  It must be ZEROED before its first use; every call that
- *                    completes leaves it ready for the next call.  After FP8Q_ERR_TIMEOUT from
- *                    fp8q_check_device_error it must be zeroed again.  Two calls that share a
- *                    workspace must be ordered (same stream, or synchronized): concurrent calls
- *                    on one workspace race.
+ *                    resolved S is 1.  Its contents need no initialisation.  Two calls that
+ *                    share a workspace must be ordered (same stream, or synchronized):
+ *                    concurrent calls on one workspace race.
  * Other arguments, layouts and errors as fp8q_gemm_w8a8_block; splits out of range gives
  * FP8Q_ERR_ARG, a workspace smaller than required FP8Q_ERR_SHAPE.  Source: the same passages as
  * fp8q_gemm_w8a8_block (the split only reorders the fp32 promotion sum over K-blocks). */
@@ -144,8 +142,8 @@ int fp8q_gemm_w8a8_block_splitk(const void *aq, int64_t lda, const float *sa, in
 int fp8q_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int splits,
                                      int64_t *bytes);
 
-/* fp8q_gemm_w8a8_block_splitk without a caller workspace: the split-K partials and counters live
- * in a fixed 24 MiB (+ 4 KiB) buffer that the library declares in its own device memory (reserved
+/* fp8q_gemm_w8a8_block_splitk without a caller workspace: the split-K partials live in a fixed
+ * 24 MiB buffer that the library declares in its own device memory (reserved
  * when the library's device code is loaded), so the call allocates nothing.  It serves callers
  * that cannot allocate device memory at call time: an inference engine that hands all free HBM
  * to its KV-cache pool at start-up and has no room left for per-call workspaces, or a caller that
@@ -155,8 +153,7 @@ int fp8q_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int splits
  *   Limit: tiles * S <= 192 (tiles = ceil(M / 128) * ceil(N / 256), S the resolved split
  *   count); beyond it FP8Q_ERR_TOO_LARGE.  Decode (M <= 128, N <= 12288) with
  *   S <= 4 fits.  A resolved S of 1 runs fp8q_gemm_w8a8_block and touches no scratch.
- *   The per-tile counters must start at zero: each call zeroes them on `stream`
- *   (cudaMemsetAsync, no allocation) before its kernel.
+ *   Nothing in the buffer needs to start at zero: each call writes every partial it reads.
  *   The first call on each device looks the buffer's address up (cudaGetSymbolAddress, with
  *   that device current); make that first call before any stream capture.
  *   Each device has one such buffer (per process), shared by every caller: two calls on one

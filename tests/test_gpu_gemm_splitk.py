@@ -42,14 +42,12 @@ def test_splitk_ragged(M, N, K, splits, fmt):
     assert torch.isnan(buf[:, N:].float()).all()
     ref, absref = oracle.gemm_w8a8_block(aq, sa, wq, sw, fmt)
     assert_within_gemm_tolerance(host_bf16_f64(o), ref, absref)
-    # counters are back at zero, so the same workspace serves the next call; the fixed summation
-    # order makes the second result bit-identical
+    # the same workspace serves the next call, even filled with garbage (every partial is written
+    # before it is read); the fixed summation order makes the second result bit-identical
+    ws.fill_(0xFF)
     o2 = fq.gemm_w8a8_block_splitk(*d, fmt, splits=splits, workspace=ws)
     assert fq.check_device_error() == 0
     assert torch.equal(o.view(torch.int16), o2.view(torch.int16))
-    tiles = -(-M // 128) * -(-N // 256)
-    cnt = ws[tiles * splits * 128 * 256 * 4:].view(torch.int32)[:tiles]
-    assert int(cnt.abs().sum()) == 0
 
 
 def test_splits_equal_k_blocks_and_single_split():
@@ -68,13 +66,13 @@ def test_splits_equal_k_blocks_and_single_split():
     assert torch.equal(o1.view(torch.int16), o0.view(torch.int16))
 
 
-def test_decode_full_size_auto_splits_sampled_rows():
-    """Decode shape (128 x 12288 x 4096) with the library's split choice, as the bench runs it."""
-    d = inputs.decode_linear()
-    aq, sa, wq, sw = _quantize(d["A"], d["W"], 0)
-    M, K = aq.shape
-    N = wq.shape[0]
-    assert fq.gemm_splitk_workspace_bytes(M, N, K, 0) > 0       # decode does split on 148 SMs
+def test_decode_long_k_auto_splits_sampled_rows():
+    """Decode down projection (128 x 4096 x 12288) with the library's split choice, as the bench
+    runs it: long K with few tiles is where splitting pays."""
+    M, N, K = 128, 4096, 12288
+    assert fq.gemm_splitk_workspace_bytes(M, N, K, 0) > 0       # splits on 148 SMs
+    aq, sa, wq, sw = _quantize(inputs.randn_bf16((M, K), 1.0, 64, 0),
+                               inputs.randn_bf16((N, K), 0.02, 64, 1), 0)
     dv = _dev(aq, sa, wq, sw, 0)
     ws = fq.splitk_workspace(M, N, K, 0, device="cuda")
     for _ in range(3):   # repeated calls reuse the workspace
@@ -85,10 +83,15 @@ def test_decode_full_size_auto_splits_sampled_rows():
     assert_within_gemm_tolerance(host_bf16_f64(o)[rows], ref, absref)
 
 
+def test_decode_auto_choice_does_not_split_short_k():
+    """128 x 12288 x 4096: splitting was measured not to pay; the library picks one split."""
+    assert fq.gemm_splitk_workspace_bytes(128, 12288, 4096, 0) == 0
+
+
 def test_workspace_too_small_is_rejected():
     M, N, K = 64, 256, 512
     need = fq.gemm_splitk_workspace_bytes(M, N, K, 2)
-    assert need == 2 * 128 * 256 * 4 + 16
+    assert need == 2 * 128 * 256 * 4
     aq = torch.zeros((M, K), dtype=torch.uint8, device="cuda")
     sa = torch.ones((K // 128, M), dtype=torch.float32, device="cuda")
     wq = torch.zeros((N, K), dtype=torch.uint8, device="cuda")

@@ -41,7 +41,7 @@ def _call_workspace(L, d, M, N, K, out, splits):
     aq, sa, wq, sw = d
     nbytes = ctypes.c_int64(0)
     assert L.fp8q_gemm_splitk_workspace_bytes(M, N, K, splits, ctypes.byref(nbytes)) == 0
-    ws = torch.zeros(max(16, nbytes.value), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(max(16, nbytes.value), dtype=torch.uint8, device="cuda")
     st = L.fp8q_gemm_w8a8_block_splitk(
         aq.data_ptr(), aq.stride(0), sa.data_ptr(), sa.stride(0), wq.data_ptr(), wq.stride(0),
         sw.data_ptr(), _lib.FP8Q_SCALE_F32, M, N, K, out.data_ptr(), out.stride(0), splits,
@@ -52,7 +52,7 @@ def _call_workspace(L, d, M, N, K, out, splits):
 @pytest.mark.parametrize("M,N,K,splits,rows", [
     (100, 2048, 1024, 4, None),                              # 8 tiles x 4 splits, all rows
     (128, 12288, 4096, 3, [0, 1, 63, 64, 126, 127]),         # decode shape, 48 tiles x 3
-    (128, 12288, 4096, 0, [0, 77, 127]),                     # the library's split choice
+    (128, 4096, 12288, 0, [0, 77, 127]),                     # the library's choice: 8 splits
 ])
 def test_noalloc_matches_workspace_entry_twice(M, N, K, splits, rows):
     L = _lib.lib()
