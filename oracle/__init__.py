@@ -53,6 +53,10 @@ def lib():
                                                           ctypes.c_int, P, I64, I64, I64, P,
                                                           I64, P, P]
         L.oracle_e4m3_encode_array.restype = None
+        L.oracle_quant_rowwise.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64, P]
+        L.oracle_quant_rowwise.restype = None
+        L.oracle_gemm_w8a8_rowwise_rows.argtypes = [P, I64, P, P, I64, P, I64, I64, P, I64, P, P]
+        L.oracle_gemm_w8a8_rowwise_rows.restype = None
         L.oracle_e4m3_encode_array.argtypes = [P, I64, P]
         L.oracle_f32_to_bf16_array.restype = None
         L.oracle_f32_to_bf16_array.argtypes = [P, I64, P]
@@ -216,6 +220,35 @@ def grouped_gemm_w8a8_block(aq, sa, wq, sw, group_offsets, sw_fmt: int = SCALE_F
     lib().oracle_grouped_gemm_w8a8_block_rows(_ptr(aq), K, _ptr(sa), sa.shape[1], _ptr(wq), K,
                                               _ptr(sw), int(sw_fmt), _ptr(off), E, N, K,
                                               _ptr(rows), rows.size, _ptr(ref), _ptr(absref))
+    return ref, absref
+
+
+def quant_rowwise(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6):
+    """Per-token (or per-channel) quantization, reading R7: codes uint8 [R, K] and one fp32 scale
+    per row; with gamma, each row is RMS-normalised first (reading R4)."""
+    x = _c(x_bf16, np.uint16)
+    R, K = x.shape
+    q = np.empty((R, K), np.uint8)
+    s = np.empty(R, np.float32)
+    g = None if gamma_bf16 is None else _c(gamma_bf16, np.uint16)
+    lib().oracle_quant_rowwise(_ptr(x), None if g is None else _ptr(g), float(eps), R, K, K,
+                               _ptr(q), K, _ptr(s))
+    return q, s
+
+
+def gemm_w8a8_rowwise(aq, sa, wq, sw, rows=None):
+    """Per-channel GEMM reference (reading R7) in fp64 on the selected rows: (ref, absref)."""
+    aq = _c(aq, np.uint8)
+    wq = _c(wq, np.uint8)
+    sa = _c(sa, np.float32)
+    sw = _c(sw, np.float32)
+    M, K = aq.shape
+    N = wq.shape[0]
+    r = np.arange(M, dtype=np.int64) if rows is None else _c(np.asarray(rows), np.int64)
+    ref = np.empty((len(r), N), np.float64)
+    absref = np.empty((len(r), N), np.float64)
+    lib().oracle_gemm_w8a8_rowwise_rows(_ptr(aq), K, _ptr(sa), _ptr(wq), K, _ptr(sw), N, K,
+                                        _ptr(r), len(r), _ptr(ref), _ptr(absref))
     return ref, absref
 
 

@@ -41,6 +41,12 @@
  *   R5  activation scales sa are fp32, stored K-block-major: sa[kb * lds + m].
  *   R6  GEMM reference: out[m,n] = sum_kb (sa[m,kb] * sw[nb,kb]) * P_kb[m,n], P_kb the exact
  *       dot product of the decoded codes over K-block kb; all in fp64.
+ *   R7  per-token / per-channel ("PTPC") variant [SGL-RMSQ sections 1-3: group_size 0 means
+ *       per token; CHANNEL weight strategy; the GEMM takes (codes, x_scale) and weight_scale]:
+ *       one scale per full row of K, s = amax / 448 as in R1 (0 -> 1), codes as in R1; the
+ *       same rule quantizes a weight per output channel (one row of W).  With gamma, the row
+ *       is first normalised as in R4.  GEMM reference: out[m,n] = sa[m] * sw[n] * P[m,n], P the
+ *       exact dot product of the decoded codes over all of K, in fp64.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math -fopenmp.
  * fp32 arithmetic below relies on FLT_EVAL_METHOD == 0 (SSE on x86-64), so every float
@@ -299,6 +305,57 @@ void oracle_rmsnorm_quant_token(const uint16_t *x, const uint16_t *gamma, float 
             sa[kb * lds + m] = quant_group_1x128(y, q + m * ldq + kb * 128);
         }
     }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Per-token / per-channel quantization [SGL-RMSQ section 1, group_size 0], reading R7          */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Rows of bf16 x [R, K] (leading dimension ldx) -> codes [R, K] (ldq) and one fp32 scale per row
+ * in s[R].  gamma == NULL: plain; otherwise each row is the bf16 RMSNorm of reading R4 first. */
+void oracle_quant_rowwise(const uint16_t *x, const uint16_t *gamma, float eps, int64_t R,
+                          int64_t K, int64_t ldx, uint8_t *q, int64_t ldq, float *s) {
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t m = 0; m < R; ++m) {
+        const uint16_t *xr = x + m * ldx;
+        float r = (gamma != NULL) ? rms_inverse(xr, K, eps) : 1.0f;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float y = bf16_to_f32(xr[k]);
+            if (gamma != NULL) y = bf16_to_f32(f32_to_bf16_rne((y * r) * bf16_to_f32(gamma[k])));
+            float a = fabsf(y);
+            if (a > amax) amax = a;
+        }
+        float sc = scale_f32_from_amax(amax);
+        for (int64_t k = 0; k < K; ++k) {
+            float y = bf16_to_f32(xr[k]);
+            if (gamma != NULL) y = bf16_to_f32(f32_to_bf16_rne((y * r) * bf16_to_f32(gamma[k])));
+            q[m * ldq + k] = oracle_e4m3_encode(y / sc);
+        }
+        s[m] = sc;
+    }
+}
+
+/* Per-channel GEMM reference on a subset of rows, reading R7: ref = sa[m] * sw[n] * P and
+ * absref = sa[m] * sw[n] * sum_k |dec(a) * dec(w)|, in fp64 (P is exact: 8-bit products). */
+void oracle_gemm_w8a8_rowwise_rows(const uint8_t *aq, int64_t lda, const float *sa,
+                                   const uint8_t *wq, int64_t ldw, const float *sw, int64_t N,
+                                   int64_t K, const int64_t *rows, int64_t nrows, double *ref,
+                                   double *absref) {
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t i = 0; i < nrows; ++i)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t m = rows[i];
+            double P = 0.0, PA = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double prod = oracle_e4m3_decode(aq[m * lda + k]) * oracle_e4m3_decode(wq[n * ldw + k]);
+                P += prod;
+                PA += fabs(prod);
+            }
+            double sc = (double)sa[m] * (double)sw[n];
+            ref[i * N + n] = sc * P;
+            absref[i * N + n] = fabs(sc) * PA;
+        }
 }
 
 /* ------------------------------------------------------------------------------------------ */
