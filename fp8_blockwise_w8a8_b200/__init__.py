@@ -23,6 +23,7 @@ import ctypes
 
 __all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
+           "quant_rowwise", "gemm_w8a8_rowwise",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -152,6 +153,32 @@ def grouped_gemm_w8a8_block(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor
                                                  _ptr(group_offsets), E, M, N, K, _ptr(o),
                                                  _ld(o), _stream(stream))
     _lib.check(st, "fp8q_grouped_gemm_w8a8_block")
+    return o
+
+
+def quant_rowwise(x: torch.Tensor, gamma=None, eps: float = 1e-6, out_q=None, out_s=None,
+                  stream=None):
+    """bf16 [R, K] -> (codes uint8 [R, K], scales fp32 [R]): one scale per row (per token, or per
+    output channel for a weight); gamma: RMSNorm first."""
+    R, K = x.shape
+    q = torch.empty((R, K), dtype=torch.uint8, device=x.device) if out_q is None else out_q
+    s = torch.empty((R,), dtype=torch.float32, device=x.device) if out_s is None else out_s
+    st = _lib.lib().fp8q_quant_rowwise(_ptr(x), _ptr(gamma), float(eps), R, K, _ld(x), _ptr(q),
+                                       _ld(q), _ptr(s), _stream(stream))
+    _lib.check(st, "fp8q_quant_rowwise")
+    return q, s
+
+
+def gemm_w8a8_rowwise(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                      out=None, stream=None):
+    """Per-token x per-channel GEMM: codes aq [M, K] (scales sa [M]) x codes wq [N, K] (scales
+    sw [N]) -> bf16 [M, N]."""
+    M, K = aq.shape
+    N = wq.shape[0]
+    o = torch.empty((M, N), dtype=torch.bfloat16, device=aq.device) if out is None else out
+    st = _lib.lib().fp8q_gemm_w8a8_rowwise(_ptr(aq), _ld(aq), _ptr(sa), _ptr(wq), _ld(wq),
+                                           _ptr(sw), M, N, K, _ptr(o), _ld(o), _stream(stream))
+    _lib.check(st, "fp8q_gemm_w8a8_rowwise")
     return o
 
 

@@ -63,7 +63,16 @@ int device_state(DeviceState **out) {
             cudaSuccess ||
         cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
-            cudaSuccess)
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_quant_rowwise<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_quant_rowwise<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_gemm_w8a8_rowwise,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fp8q::kGemmSmemDense) != cudaSuccess)
       return FP8Q_ERR_LAUNCH;
     st.attrs_set = true;
   }
@@ -208,7 +217,7 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
 
 extern "C" {
 
-int fp8q_abi_version(void) { return (1 << 16) | 1; }
+int fp8q_abi_version(void) { return (1 << 16) | 2; }
 
 const char *fp8q_status_string(int status) {
   switch (status) {
@@ -405,6 +414,91 @@ int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, i
   if (E * N > INT32_MAX) return FP8Q_ERR_SHAPE;
   return launch_gemm(true, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, group_offsets, E, M, N, K,
                      out_bf16, ldo, stream);
+}
+
+int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
+                       int64_t K, int64_t ldx, void *q_e4m3, int64_t ldq, float *s,
+                       cudaStream_t stream) {
+  if (M < 0 || K <= 0 || K % 128 || K > kMaxTokenK) return FP8Q_ERR_SHAPE;
+  if (ldx < K || ldq < K) return FP8Q_ERR_SHAPE;
+  if (M == 0) return FP8Q_OK;
+  if (!x_bf16 || !q_e4m3 || !s) return FP8Q_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(q_e4m3) || (reinterpret_cast<uintptr_t>(s) & 3u) ||
+      ldx % 8 || ldq % 16 || (gamma_bf16 && !aligned16(gamma_bf16)))
+    return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  const bool norm = gamma_bf16 != nullptr;
+  const int budget = 227 * 1024;
+  int best_wpc = 0, best_ctas = 0, best_smem = 0;
+  for (int wpc : {16, 12, 8, 4, 2, 1}) {
+    const int smem = fp8q::token_smem_bytes(static_cast<int>(K), norm, wpc);
+    if (smem > budget) continue;
+    int per_sm = 0;
+    if (norm)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_quant_rowwise<true>,
+                                                    32 * wpc, smem);
+    else
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_quant_rowwise<false>,
+                                                    32 * wpc, smem);
+    if (per_sm * wpc > best_ctas * best_wpc) {
+      best_wpc = wpc;
+      best_ctas = per_sm;
+      best_smem = smem;
+    }
+  }
+  if (best_wpc == 0) return FP8Q_ERR_SHAPE;
+  const int wpc = best_wpc, smem = best_smem;
+  const int64_t need = (M + wpc - 1) / wpc;
+  const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  const auto *x = static_cast<const uint16_t *>(x_bf16);
+  const auto *g = static_cast<const uint16_t *>(gamma_bf16);
+  auto *q = static_cast<uint8_t *>(q_e4m3);
+  if (norm)
+    fp8q::k_quant_rowwise<true><<<grid, 32 * wpc, smem, stream>>>(x, ldx, g, eps, M,
+                                                                   static_cast<int>(K), q, ldq, s);
+  else
+    fp8q::k_quant_rowwise<false><<<grid, 32 * wpc, smem, stream>>>(x, ldx, nullptr, eps, M,
+                                                                    static_cast<int>(K), q, ldq, s);
+  return launch_status();
+}
+
+int fp8q_gemm_w8a8_rowwise(const void *aq, int64_t lda, const float *sa, const void *wq,
+                           int64_t ldw, const float *sw, int64_t M, int64_t N, int64_t K,
+                           void *out_bf16, int64_t ldo, cudaStream_t stream) {
+  if (M < 0 || N <= 0 || K <= 0 || N % 128 || K % 128) return FP8Q_ERR_SHAPE;
+  if (M > INT32_MAX - 256 || N > (1 << 30) || K > (1 << 30)) return FP8Q_ERR_SHAPE;
+  if (lda < K || ldw < K || ldo < N) return FP8Q_ERR_SHAPE;
+  if (M == 0) return FP8Q_OK;
+  if (!aq || !sa || !wq || !sw || !out_bf16) return FP8Q_ERR_NULL;
+  if (!aligned16(aq) || !aligned16(wq) || !aligned16(out_bf16) ||
+      (reinterpret_cast<uintptr_t>(sa) & 3u) || (reinterpret_cast<uintptr_t>(sw) & 3u) ||
+      lda % 16 || ldw % 16 || ldo % 8)
+    return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  if ((rc = get_encoder()) != FP8Q_OK) return rc;
+  CUtensorMap tm_a, tm_b;
+  if ((rc = make_u8_map(&tm_a, aq, M, K, lda, fp8q::kBM)) != FP8Q_OK) return rc;
+  if ((rc = make_u8_map(&tm_b, wq, N, K, ldw, fp8q::kBN)) != FP8Q_OK) return rc;
+  fp8q::RowwiseArgs a;
+  a.sa = sa;
+  a.sw = sw;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K);
+  a.out = static_cast<uint16_t *>(out_bf16);
+  a.ldo = ldo;
+  a.num_n = static_cast<int>((N + fp8q::kBN - 1) / fp8q::kBN);
+  a.num_m = static_cast<int>((M + fp8q::kBM - 1) / fp8q::kBM);
+  const int64_t tiles = static_cast<int64_t>(a.num_m) * a.num_n;
+  const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+  fp8q::k_gemm_w8a8_rowwise<<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemDense, stream>>>(tm_a,
+                                                                                       tm_b, a);
+  return launch_status();
 }
 
 int fp8q_check_device_error(cudaStream_t stream) {

@@ -523,7 +523,206 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// Split-K reduction: out[m, n] = bf16( sum over j = 0 .. S - 1, in that order, of partial_j ).
+// ---------------------------------------------------------------------------------------------
+// Per-token x per-channel ("PTPC") W8A8 GEMM: out[m, n] = bf16( P[m, n] * fp32(sa[m] * sw[n]) )
+// with P the fp32 tensor-core dot product over all of K.  With no per-K-block promotion the MMA
+// accumulates a whole tile in one TMEM buffer; the epilogue drains a buffer once per tile while
+// the MMA fills the other.  Same persistent structure, shared-memory layout and barriers as
+// k_gemm_w8a8_block:
+//   warp 0      TMA producer (A 128 x 128 B, B 256 x 128 B per K-block, 4-stage ring)
+//   warp 1      TMEM allocator and MMA issuer: per tile, all K-blocks into buffer tile % 2
+//   warp 2      scale producer: the tile's 256 weight scales, double-buffered across tiles
+//   warps 4-11  epilogue: warp w reads TMEM lanes 32 (w % 4), column half (w - 4) / 4
+// ---------------------------------------------------------------------------------------------
+struct RowwiseArgs {
+  const float *sa;      // [M] per-token scales
+  const float *sw;      // [N] per-channel scales
+  int M, N, K;
+  uint16_t *out;
+  int64_t ldo;
+  int num_n, num_m;
+};
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm_w8a8_rowwise(const __grid_constant__ CUtensorMap tm_a,
+                        const __grid_constant__ CUtensorMap tm_b, const RowwiseArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + kOffBar;              // [kStages]
+  const uint32_t bar_empty = bar_full + 8 * kStages;      // [kStages]
+  const uint32_t bar_tfull = bar_empty + 8 * kStages;     // [2]
+  const uint32_t bar_tempty = bar_tfull + 16;             // [2]
+  const uint32_t bar_done = bar_tempty + 16;
+  const uint32_t bar_swfull = bar_done + 8;               // [2]
+  const uint32_t bar_swempty = bar_swfull + 16;           // [2]
+  float *s_sw = reinterpret_cast<float *>(smem + kOffSw);  // [2][256]
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+  const int KB = args.K / kBK;
+  GemmArgs ga{};
+  ga.num_m = args.num_m;
+  ga.num_n = args.num_n;
+  ga.M = args.M;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_tfull + 8 * i, 1);
+      mbar_init(bar_tempty + 8 * i, 8);
+      mbar_init(bar_swfull + 8 * i, 32);
+      mbar_init(bar_swempty + 8 * i, 8);
+    }
+    mbar_init(bar_done, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total_tiles = args.num_m * args.num_n;
+
+  if (warp < 4) {
+    reg_dealloc<kProducerRegs>();
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_b);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+          const Tile tl = dense_tile(ga, t);
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            if (!wait_one(bar_empty + 8 * s, ph ^ 1u, s_abort)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar_full + 8 * s, kStageBytes);
+            tma_load_2d(sbase + kOffA + s * kTileABytes, &tm_a, kb * kBK, tl.m0, bar_full + 8 * s);
+            tma_load_2d(sbase + kOffB + s * kTileBBytes, &tm_b, kb * kBK, tl.b_row,
+                        bar_full + 8 * s);
+          }
+        }
+        for (uint32_t s = 0; s < kStages && s < it; ++s) {
+          const uint32_t last = s + ((it - 1 - s) / kStages) * kStages;  // last fill of stage s
+          wait_drain(bar_full + 8 * s, (last / kStages) & 1u);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 2) {
+      // ---------------------------------------------------------------- scale producer
+      uint32_t tile_it = 0;
+      for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tile_it) {
+        const Tile tl = dense_tile(ga, t);
+        const uint32_t tp = tile_it & 1u;
+        if (!wait_warp(bar_swempty + 8 * tp, ((tile_it >> 1) & 1u) ^ 1u, s_abort)) break;
+        for (int j = lane; j < kBN; j += 32) {
+          const int n = tl.n0 + j;
+          s_sw[tp * kBN + j] = n < args.N ? __ldg(args.sw + n) : 0.0f;
+        }
+        mbar_arrive(bar_swfull + 8 * tp);
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        uint32_t it = 0, tile_it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tile_it) {
+          const uint32_t b = tile_it & 1u, bph = (tile_it >> 1) & 1u;
+          if (!wait_one(bar_tempty + 8 * b, bph ^ 1u, s_abort)) { ok = false; break; }
+          const uint32_t d = tmem_base + b * kBN;
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            if (!wait_one(bar_full + 8 * s, ph, s_abort)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t ad = sdesc_k128(sbase + kOffA + s * kTileABytes);
+            const uint64_t bd = sdesc_k128(sbase + kOffB + s * kTileBBytes);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 32; ++kk)
+              mma_f8f6f4(d, ad + 2 * kk, bd + 2 * kk, kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar_empty + 8 * s);
+          }
+          if (!ok) break;
+          mma_commit(bar_tfull + 8 * b);
+        }
+        // Every MMA has completed before TMEM is released.
+        mma_commit(bar_done);
+        wait_drain(bar_done, 0);
+      }
+      __syncwarp();
+    }
+  } else {
+    reg_alloc<kEpilogueRegs>();
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;         // TMEM lane quarter = rows 32q .. 32q + 31 of the tile
+    const int h = (warp - 4) >> 2;  // column half of the 256-wide tile
+    const int NB = args.N / 128;
+    uint8_t *stage = smem + kOffStaging + (warp - 4) * kStagingBytesPerWarp;
+    const uint32_t stage_u32 = smem_u32(stage);
+    uint32_t tile_it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tile_it) {
+      const Tile tl = dense_tile(ga, t);
+      const int row = tl.m0 + 32 * q + lane;
+      const float sa_row = row < tl.row_end ? __ldg(args.sa + row) : 0.0f;
+      const bool col_ok = tl.n0 / 128 + h < NB;
+      const uint32_t tp = tile_it & 1u, b = tile_it & 1u, bph = (tile_it >> 1) & 1u;
+      if (!wait_warp(bar_swfull + 8 * tp, bph, s_abort)) { ok = false; break; }
+      if (!wait_warp(bar_tfull + 8 * b, bph, s_abort)) { ok = false; break; }
+      tc_fence_after();
+      const float *swh = s_sw + tp * kBN + 128 * h;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + b * kBN + h * 128;
+      uint16_t *out_base = args.out + static_cast<int64_t>(tl.n0 + 128 * h);
+#pragma unroll 1
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t r0[16], r1[16];
+        tmem_ld_32x32b_x16(taddr + 32 * c4, r0);
+        tmem_ld_32x32b_x16(taddr + 32 * c4 + 16, r1);
+        tmem_ld_wait(r0);
+        tmem_ld_wait(r1);
+        if (c4 == 3) {
+          // the whole buffer is in registers: hand it back to the MMA before the last stores
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_tempty + 8 * b);
+        }
+        float2 v[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = 32 * c4 + 2 * j;
+          v[j] = make_float2(__fmul_rn(__uint_as_float(r0[2 * j]), __fmul_rn(sa_row, swh[c])),
+                             __fmul_rn(__uint_as_float(r0[2 * j + 1]), __fmul_rn(sa_row, swh[c + 1])));
+          v[8 + j] = make_float2(
+              __fmul_rn(__uint_as_float(r1[2 * j]), __fmul_rn(sa_row, swh[c + 16])),
+              __fmul_rn(__uint_as_float(r1[2 * j + 1]), __fmul_rn(sa_row, swh[c + 17])));
+        }
+        store_chunk32(v, stage_u32, lane, out_base, tl, q, c4, col_ok, args.ldo);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_swempty + 8 * tp);  // done with this tile's weight scales
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// Split-K reduction: out[m, n] = bf16( sum over j = 0 .. S - 1, in that order, of partial_j )."""
+
 // Partials: [tile][split][half h][chunk c][row r] float4 = columns 128 h + 4 c .. + 3 of row r.
 // Grid: 8 CTAs of 256 threads per dense tile; thread (r, g) adds row r, columns 16 g .. 16 g + 15
 // (4 float4 per split, read coalesced across rows) and writes 32 contiguous output bytes.

@@ -423,4 +423,78 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Per-token (full-row) quantization, optionally after RMSNorm: one scale per row of K (the
+// "group size 0" per-token mode; applied to a weight it gives per-output-channel scales).  One
+// warp per row.  With RMSNorm, r is formed exactly as in k_rmsnorm_quant_token; then one pass
+// over the row finds its absolute maximum (of y with RMSNorm) and a second pass writes the codes.
+// Both passes read the row through L1 (the row was prefetched into L2 during the previous one).
+// ---------------------------------------------------------------------------------------------
+template <bool NORM>
+__global__ void __launch_bounds__(512) k_quant_rowwise(
+    const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
+    int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_out) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wpc = blockDim.x >> 5;
+  const int KB = K >> 7, KC = K >> 3;   // 128-blocks and 16-byte chunks per row
+  ScaleTab *tab = reinterpret_cast<ScaleTab *>(smem);
+  float4 *gA = reinterpret_cast<float4 *>(smem + sizeof(ScaleTab));
+  float4 *gB = gA + KC;
+  double *wsum = reinterpret_cast<double *>(smem + sizeof(ScaleTab) + K * 4) + warp * KB;  // NORM
+
+  build_scale_tab(tab, threadIdx.x, blockDim.x);
+  if (NORM) {
+    for (int j = threadIdx.x; j < KC; j += blockDim.x) {
+      const uint4 g = *reinterpret_cast<const uint4 *>(gamma + j * 8);
+      gA[j] = make_float4(bf16_lo(g.x), bf16_hi(g.x), bf16_lo(g.y), bf16_hi(g.y));
+      gB[j] = make_float4(bf16_lo(g.z), bf16_hi(g.z), bf16_lo(g.w), bf16_hi(g.w));
+    }
+  }
+  __syncthreads();
+
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
+  for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < M; m += stride) {
+    const uint16_t *xr = x + m * ldx;
+    const int64_t next = m + stride;
+    if (next < M) {
+      const char *nr = reinterpret_cast<const char *>(x + next * ldx);
+      for (int off = lane * 128; off < K * 2; off += 32 * 128) prefetch_l2(nr + off);
+    }
+    float r = 1.0f;
+    if (NORM) {
+      for (int b = lane; b < KB; b += 32) wsum[b] = block_sumsq(xr + b * 128);
+      __syncwarp();
+      if (lane == 0) {
+        double S = 0.0;
+        for (int b = 0; b < KB; ++b) S = __dadd_rn(S, wsum[b]);
+        const double var = __dadd_rn(__ddiv_rn(S, static_cast<double>(K)), static_cast<double>(eps));
+        r = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(var)));
+      }
+      r = __shfl_sync(0xffffffffu, r, 0);
+    }
+    // the row's absolute maximum
+    uint32_t m2 = 0u;
+#pragma unroll 4
+    for (int j = lane; j < KC; j += 32) {
+      uint4 v = *reinterpret_cast<const uint4 *>(xr + j * 8);
+      if (NORM) v = rms_apply8(v, r, gA[j], gB[j]);
+      m2 = absmax_uint4(m2, v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+    const QParams p = qparams_tab(absmax_finish(m2), tab);
+    // the codes
+    uint8_t *qr = q + m * ldq;
+#pragma unroll 4
+    for (int j = lane; j < KC; j += 32) {
+      uint4 v = *reinterpret_cast<const uint4 *>(xr + j * 8);
+      if (NORM) v = rms_apply8(v, r, gA[j], gB[j]);
+      *reinterpret_cast<uint2 *>(qr + j * 8) = quant8_f32(v, p);
+    }
+    if (lane == 0) s_out[m] = p.s;
+    __syncwarp();  // lane 0 has read every block sum before they are overwritten
+  }
+}
+
 }  // namespace fp8q

@@ -180,6 +180,35 @@ int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, i
                                  const int32_t *group_offsets, int64_t E, int64_t M, int64_t N,
                                  int64_t K, void *out_bf16, int64_t ldo, cudaStream_t stream);
 
+/* Per-token (full-row) quantization, optionally fused with RMSNorm: one fp32 scale per row of K
+ * (the "group size 0 = per token" mode).  Applied to a weight W [N, K] it gives the
+ * per-output-channel codes and scales the per-channel GEMM below takes.
+ *   x_bf16      [M][ldx] bf16, read
+ *   gamma_bf16  [K] bf16 RMSNorm weight, or NULL (no normalisation); eps as fp8q_rmsnorm_quant_token
+ *   q_e4m3      [M][ldq] uint8 codes, written
+ *   s           [M] fp32 scales, written (4-byte aligned)
+ * s = amax / 448 over the whole (normalised) row, IEEE division, 1 for an all-zero row; codes
+ * q = RNEsat(y / s).  RMSNorm arithmetic as fp8q_rmsnorm_quant_token.  K % 128 == 0, K <= 16384.
+ * Bit-exact against the CPU oracle.  Source: SGLang PR 21403 analysis, section 1 (RMSNorm with
+ * weight and epsilon fused with FP8 quant, group_size 0 = per token) and section 2 (CHANNEL
+ * weight strategy -> per-token path). */
+int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
+                       int64_t K, int64_t ldx, void *q_e4m3, int64_t ldq, float *s,
+                       cudaStream_t stream);
+
+/* Per-token x per-channel W8A8 GEMM:
+ *   out[m, n] = bf16( P[m, n] * fp32(sa[m] * sw[n]) ),  P = fp32 tensor-core dot product over K
+ * with no per-K-block promotion (the scales are constant along K).
+ *   aq [M][lda] uint8 codes, sa [M] fp32; wq [N][ldw] uint8 codes, sw [N] fp32
+ *   out [M][ldo] bf16, written (rows < M, columns < N)
+ * Shapes and alignment as fp8q_gemm_w8a8_block (sa and sw 4-byte aligned).  Error bound as the
+ * block-scaled GEMM: |out - ref| <= 8e-3 sum_k |dec(a) dec(w)| sa sw + 1 bf16 ulp.  Source: SGLang
+ * PR 21403 analysis, section 3 (the PTPC GEMM takes the (codes, x_scale) tuple and the per-channel
+ * weight scale, no bias, bf16 out). */
+int fp8q_gemm_w8a8_rowwise(const void *aq, int64_t lda, const float *sa, const void *wq,
+                           int64_t ldw, const float *sw, int64_t M, int64_t N, int64_t K,
+                           void *out_bf16, int64_t ldo, cudaStream_t stream);
+
 /* Synchronize `stream`, then read and clear the device error word of the current device.
  * Returns FP8Q_OK, FP8Q_ERR_TIMEOUT (a kernel gave up on a bounded wait since the last call;
  * its outputs are incomplete) or FP8Q_ERR_LAUNCH (the synchronize failed). */

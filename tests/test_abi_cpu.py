@@ -131,3 +131,27 @@ def test_splitk_noalloc_host_checks(L):
     assert g(*a, 64, 256, 512, FAKE, 256, 5, None) == _lib.FP8Q_ERR_ARG
     assert g(*a, 64, 200, 512, FAKE, 256, 2, None) == _lib.FP8Q_ERR_SHAPE
     assert g(*a, 0, 256, 512, None, 256, 2, None) == _lib.FP8Q_OK
+
+
+def test_rowwise_host_checks(L):
+    f = L.fp8q_quant_rowwise
+    assert f(FAKE, None, 1e-6, 4, 100, 100, FAKE, 112, FAKE, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, None, 1e-6, 4, 32768, 32768, FAKE, 32768, FAKE, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, None, 1e-6, 4, 128, 128, FAKE, 128, FAKE + 2, None) == _lib.FP8Q_ERR_ALIGN
+    assert f(FAKE, FAKE + 8, 1e-6, 4, 128, 128, FAKE, 128, FAKE, None) == _lib.FP8Q_ERR_ALIGN
+    assert f(None, None, 1e-6, 4, 128, 128, FAKE, 128, FAKE, None) == _lib.FP8Q_ERR_NULL
+    assert f(None, None, 1e-6, 0, 128, 128, None, 128, None, None) == _lib.FP8Q_OK
+    g = L.fp8q_gemm_w8a8_rowwise
+    a = dict(aq=FAKE, lda=256, sa=FAKE, wq=FAKE, ldw=256, sw=FAKE, M=64, N=128, K=256, out=FAKE,
+             ldo=128)
+
+    def call(**kw):
+        b = dict(a, **kw)
+        return g(b["aq"], b["lda"], b["sa"], b["wq"], b["ldw"], b["sw"], b["M"], b["N"], b["K"],
+                 b["out"], b["ldo"], None)
+    assert call(N=100) == _lib.FP8Q_ERR_SHAPE
+    assert call(K=200, lda=208, ldw=208) == _lib.FP8Q_ERR_SHAPE
+    assert call(sw=None) == _lib.FP8Q_ERR_NULL
+    assert call(sa=FAKE + 2) == _lib.FP8Q_ERR_ALIGN
+    assert call(lda=264) == _lib.FP8Q_ERR_ALIGN
+    assert call(M=0, aq=None, sa=None, out=None) == _lib.FP8Q_OK
