@@ -277,6 +277,41 @@ def measure_rows(fq, device, steps, warmup, pk):
                                      "frac": byts / ms / 1e6 / hbm, "workload": "A [128, 4096]"}
     del a, w, wq, sw, aq, sa, out
 
+    # per-token x per-channel variant of the prefill linear: per-channel requant of W, fused
+    # RMSNorm + per-token quant of X, and the per-channel GEMM (no per-K-block promotion)
+    d = inputs.prefill_linear()
+    x = dev_bf16(d["X"], device)
+    gam = dev_bf16(d["gamma"], device)
+    w = dev_bf16(d["W"], device)
+    wq, sw = fq.quant_rowwise(w)
+    aq, sa = fq.quant_rowwise(x, gam, d["eps"])
+    out = torch.empty((M_, N_), dtype=torch.bfloat16, device=device)
+    ms, _ = timed_loop(lambda: fq.quant_rowwise(w, out_q=wq, out_s=sw), steps, warmup)
+    byts = N_ * K_ * 3 + N_ * 4
+    rows["ptpc_weight_quant_prefill_W"] = {"ms": ms, "GB/s": byts / ms / 1e6,
+                                           "frac": byts / ms / 1e6 / hbm,
+                                           "workload": "W [24576, 4096], one scale per output channel"}
+    ms, _ = timed_loop(lambda: fq.quant_rowwise(x, gam, d["eps"], out_q=aq, out_s=sa), steps,
+                       warmup)
+    byts = M_ * K_ * 3 + M_ * 4 + K_ * 2
+    rows["ptpc_rmsnorm_quant_prefill_X"] = {"ms": ms, "GB/s": byts / ms / 1e6,
+                                            "frac": byts / ms / 1e6 / hbm,
+                                            "workload": "X [8192, 4096], RMSNorm + one scale per token"}
+    ms, _ = timed_loop(lambda: fq.gemm_w8a8_rowwise(aq, sa, wq, sw, out=out), steps, warmup)
+    rows["ptpc_gemm_prefill"] = {"ms": ms, "TFLOP/s": FLOPS / ms / 1e9,
+                                 "frac_fp8_sustained": FLOPS / ms / 1e9 / (2.0 * pk["bf16_sustained"]),
+                                 "workload": "M=8192 N=24576 K=4096, per-token x per-channel scales"}
+
+    def ptpc_step():
+        fq.quant_rowwise(w, out_q=wq, out_s=sw)
+        fq.quant_rowwise(x, gam, d["eps"], out_q=aq, out_s=sa)
+        fq.gemm_w8a8_rowwise(aq, sa, wq, sw, out=out)
+    ms, _ = timed_loop(ptpc_step, steps, warmup)
+    rows["ptpc_prefill_step"] = {"ms": ms, "TFLOP/s": FLOPS / ms / 1e9,
+                                 "workload": "the prefill step with per-channel W and per-token X scales"}
+    del x, gam, w, wq, sw, aq, sa, out
+    torch.cuda.empty_cache()
+
     # MoE: token quant of the routed rows and the two grouped GEMMs
     mo = inputs.moe()
     off = torch.from_numpy(mo["offsets"]).to(device)
