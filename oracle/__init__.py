@@ -53,6 +53,14 @@ def lib():
                                                           ctypes.c_int, P, I64, I64, I64, P,
                                                           I64, P, P]
         L.oracle_e4m3_encode_array.restype = None
+        L.oracle_exp_f32.argtypes = [ctypes.c_float]
+        L.oracle_exp_f32.restype = ctypes.c_float
+        L.oracle_silu_f32.argtypes = [ctypes.c_float]
+        L.oracle_silu_f32.restype = ctypes.c_float
+        L.oracle_silu_mul_quant.argtypes = [P, I64, I64, I64, P, I64, P, I64]
+        L.oracle_silu_mul_quant.restype = None
+        L.oracle_silu_mul_bf16.argtypes = [P, I64, I64, I64, P]
+        L.oracle_silu_mul_bf16.restype = None
         L.oracle_quant_rowwise.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64, P]
         L.oracle_quant_rowwise.restype = None
         L.oracle_gemm_w8a8_rowwise_rows.argtypes = [P, I64, P, P, I64, P, I64, I64, P, I64, P, P]
@@ -221,6 +229,36 @@ def grouped_gemm_w8a8_block(aq, sa, wq, sw, group_offsets, sw_fmt: int = SCALE_F
                                               _ptr(sw), int(sw_fmt), _ptr(off), E, N, K,
                                               _ptr(rows), rows.size, _ptr(ref), _ptr(absref))
     return ref, absref
+
+
+def exp_f32(x: float) -> float:
+    """e^x in fp32 by the method of reading R8 (Cody-Waite reduction, degree-7 Taylor)."""
+    return float(lib().oracle_exp_f32(float(x)))
+
+
+def silu_f32(g: float) -> float:
+    return float(lib().oracle_silu_f32(float(g)))
+
+
+def silu_mul_bf16(h_bf16: np.ndarray) -> np.ndarray:
+    """y = bf16(silu(gate) * up) of reading R8 for h = [gate | up] bf16 [R, 2I]."""
+    h = _c(h_bf16, np.uint16)
+    R, I2 = h.shape
+    y = np.empty((R, I2 // 2), np.uint16)
+    lib().oracle_silu_mul_bf16(_ptr(h), R, I2 // 2, I2, _ptr(y))
+    return y
+
+
+def silu_mul_quant(h_bf16: np.ndarray, lds: int = None):
+    """SiLU-and-mul then 1x128 token quant (reading R8): codes [R, I] and sa [I/128, lds]."""
+    h = _c(h_bf16, np.uint16)
+    R, I2 = h.shape
+    I = I2 // 2
+    lds = R if lds is None else lds
+    q = np.empty((R, I), np.uint8)
+    sa = np.zeros((I // 128, lds), np.float32)
+    lib().oracle_silu_mul_quant(_ptr(h), R, I, I2, _ptr(q), I, _ptr(sa), lds)
+    return q, sa
 
 
 def quant_rowwise(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6):

@@ -47,6 +47,11 @@
  *       same rule quantizes a weight per output channel (one row of W).  With gamma, the row
  *       is first normalised as in R4.  GEMM reference: out[m,n] = sa[m] * sw[n] * P[m,n], P the
  *       exact dot product of the decoded codes over all of K, in fp64.
+ *   R8  SiLU-and-mul front end of the MoE down projection [FP8-RL abstract (i): MoE models; the
+ *       gate/up GEMM output feeds the down GEMM]: h = [gate | up] (bf16 [R, 2I]), y_k =
+ *       bf16_RNE( fp32( silu(g_k) * u_k ) ) with silu(g) = g / (1 + e^-g) in fp32 (IEEE division)
+ *       and e^x in fp32 by Cody-Waite range reduction and a degree-7 Taylor polynomial (below);
+ *       then the 1x128 token quant of R1 on y.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math -fopenmp.
  * fp32 arithmetic below relies on FLT_EVAL_METHOD == 0 (SSE on x86-64), so every float
@@ -305,6 +310,69 @@ void oracle_rmsnorm_quant_token(const uint16_t *x, const uint16_t *gamma, float 
             sa[kb * lds + m] = quant_group_1x128(y, q + m * ldq + kb * 128);
         }
     }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* SiLU-and-mul + 1x128 quant, reading R8                                                      */
+/* ------------------------------------------------------------------------------------------ */
+
+/* e^x in fp32 by the method of Cody and Waite (1980): k = rint(x / ln 2); r = (x - k c1) - k c2
+ * with ln 2 = c1 + c2 split so that k c1 is exact for |k| <= 150; e^r from its Taylor series to
+ * degree 7 by Horner's rule (|r| <= ln2 / 2, truncation below 2^-27 relative); then the exact
+ * scaling by 2^k (in two steps where 2^k alone is not a normal fp32).  Each operation below is
+ * one IEEE fp32 rounding. */
+float oracle_exp_f32(float x) {
+    if (x > 0x1.62e430p+6f) return INFINITY;          /* above ln(FLT_MAX) */
+    if (x < -104.0f) return 0.0f;                      /* below half the smallest subnormal */
+    const float inv_ln2 = 0x1.715476p+0f, c1 = 0x1.62e400p-1f, c2 = 0x1.7f7d1cp-20f;
+    float kf = rintf(x * inv_ln2);
+    float r = (x - kf * c1) - kf * c2;
+    float p = 0x1.a01a02p-13f;                         /* 1/7! */
+    p = p * r + 0x1.6c16c2p-10f;                       /* 1/6! */
+    p = p * r + 0x1.111112p-7f;                        /* 1/5! */
+    p = p * r + 0x1.555556p-5f;                        /* 1/4! */
+    p = p * r + 0x1.555556p-3f;                        /* 1/3! */
+    p = p * r + 0x1.000000p-1f;                        /* 1/2! */
+    p = p * r + 1.0f;
+    p = p * r + 1.0f;
+    int k = (int)kf;
+    if (k > 127) { p = p * 0x1p127f; k -= 127; }
+    if (k < -126) { p = p * 0x1p-126f; k += 126; }
+    union { uint32_t u; float f; } two_k = { (uint32_t)(k + 127) << 23 };
+    return p * two_k.f;
+}
+
+/* silu(g) = g / (1 + e^-g), fp32 (IEEE division). */
+float oracle_silu_f32(float g) {
+    return g / (1.0f + oracle_exp_f32(-g));
+}
+
+/* h bf16 [R, 2I] (leading dimension ldh): gate = h[:, 0:I], up = h[:, I:2I].  Writes the codes
+ * of y = bf16(silu(gate) * up) [R, I] (ldq) and fp32 scales sa[kb * lds + m] (1x128 groups). */
+void oracle_silu_mul_quant(const uint16_t *h, int64_t R, int64_t I, int64_t ldh, uint8_t *q,
+                           int64_t ldq, float *sa, int64_t lds) {
+    int64_t IB = I / 128;
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t m = 0; m < R; ++m) {
+        float y[128];
+        for (int64_t kb = 0; kb < IB; ++kb) {
+            for (int j = 0; j < 128; ++j) {
+                int64_t k = kb * 128 + j;
+                float g = bf16_to_f32(h[m * ldh + k]), u = bf16_to_f32(h[m * ldh + I + k]);
+                y[j] = bf16_to_f32(f32_to_bf16_rne(oracle_silu_f32(g) * u));
+            }
+            sa[kb * lds + m] = quant_group_1x128(y, q + m * ldq + kb * 128);
+        }
+    }
+}
+
+/* The bf16 y of reading R8 alone (for the oracle's own pins). */
+void oracle_silu_mul_bf16(const uint16_t *h, int64_t R, int64_t I, int64_t ldh, uint16_t *y) {
+    for (int64_t m = 0; m < R; ++m)
+        for (int64_t k = 0; k < I; ++k) {
+            float g = bf16_to_f32(h[m * ldh + k]), u = bf16_to_f32(h[m * ldh + I + k]);
+            y[m * I + k] = f32_to_bf16_rne(oracle_silu_f32(g) * u);
+        }
 }
 
 /* ------------------------------------------------------------------------------------------ */
