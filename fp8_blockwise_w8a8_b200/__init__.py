@@ -23,7 +23,7 @@ import ctypes
 
 __all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
-           "quant_rowwise", "gemm_w8a8_rowwise",
+           "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -154,6 +154,22 @@ def grouped_gemm_w8a8_block(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor
                                                  _ld(o), _stream(stream))
     _lib.check(st, "fp8q_grouped_gemm_w8a8_block")
     return o
+
+
+def silu_mul_quant(h: torch.Tensor, lds=None, out_q=None, out_sa=None, stream=None):
+    """h = [gate | up] bf16 [R, 2I] -> (codes uint8 [R, I] of bf16(silu(gate) * up),
+    sa fp32 [I/128, lds]): the front end of an MoE down projection."""
+    R, I2 = h.shape
+    I = I2 // 2
+    if lds is None:
+        lds = max(4, (R + 3) // 4 * 4)
+    q = torch.empty((R, I), dtype=torch.uint8, device=h.device) if out_q is None else out_q
+    sa = (torch.empty((I // 128, lds), dtype=torch.float32, device=h.device)
+          if out_sa is None else out_sa)
+    st = _lib.lib().fp8q_silu_mul_quant(_ptr(h), R, I, _ld(h), _ptr(q), _ld(q), _ptr(sa),
+                                        sa.stride(0), _stream(stream))
+    _lib.check(st, "fp8q_silu_mul_quant")
+    return q, sa
 
 
 def quant_rowwise(x: torch.Tensor, gamma=None, eps: float = 1e-6, out_q=None, out_s=None,

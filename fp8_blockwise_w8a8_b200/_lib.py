@@ -38,6 +38,7 @@ SIGNATURES = {
     "fp8q_gemm_splitk_workspace_bytes": (_I, [_I64, _I64, _I64, _I, ctypes.POINTER(_I64)]),
     "fp8q_grouped_gemm_w8a8_block": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _P, _I64, _I64,
                                           _I64, _I64, _P, _I64, _P]),
+    "fp8q_silu_mul_quant": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _P]),
     "fp8q_quant_rowwise": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "fp8q_gemm_w8a8_rowwise": (_I, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I64, _P]),
     "fp8q_check_device_error": (_I, [_P]),

@@ -465,6 +465,39 @@ int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, in
   return launch_status();
 }
 
+int fp8q_silu_mul_quant(const void *h_bf16, int64_t R, int64_t I, int64_t ldh, void *q_e4m3,
+                        int64_t ldq, float *sa, int64_t lds, cudaStream_t stream) {
+  if (R < 0 || I <= 0 || I % 128 || I > kMaxTokenK) return FP8Q_ERR_SHAPE;
+  if (ldh < 2 * I || ldq < I || lds < R) return FP8Q_ERR_SHAPE;
+  if (R == 0) return FP8Q_OK;
+  if (!h_bf16 || !q_e4m3 || !sa) return FP8Q_ERR_NULL;
+  if (!aligned16(h_bf16) || !aligned16(q_e4m3) || !aligned16(sa) || ldh % 8 || ldq % 16 ||
+      lds % 4)
+    return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  const int smem = static_cast<int>(sizeof(fp8q::ScaleTab));
+  int best_wpc = 0, best_ctas = 0;
+  for (int wpc : {16, 8, 4}) {
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_silu_mul_quant, 32 * wpc,
+                                                  smem);
+    if (per_sm * wpc > best_ctas * best_wpc) {
+      best_wpc = wpc;
+      best_ctas = per_sm;
+    }
+  }
+  if (best_wpc == 0) return FP8Q_ERR_LAUNCH;
+  const int64_t need = (R + best_wpc - 1) / best_wpc;
+  const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  fp8q::k_silu_mul_quant<<<grid, 32 * best_wpc, smem, stream>>>(
+      static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
+      static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
+  return launch_status();
+}
+
 int fp8q_gemm_w8a8_rowwise(const void *aq, int64_t lda, const float *sa, const void *wq,
                            int64_t ldw, const float *sw, int64_t M, int64_t N, int64_t K,
                            void *out_bf16, int64_t ldo, cudaStream_t stream) {

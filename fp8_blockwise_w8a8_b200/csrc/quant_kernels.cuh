@@ -497,4 +497,108 @@ __global__ void __launch_bounds__(512) k_quant_rowwise(
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// SiLU-and-mul + 1x128 quant, the front end of an MoE down projection: h = [gate | up] bf16
+// [R, 2I] -> codes of y = bf16(silu(gate) * up) [R, I] and fp32 scales sa[kb * lds + m].
+//
+// e^x is computed by the method of Cody and Waite (1980): k = rint(x / ln 2), r = (x - k c1) -
+// k c2 with ln 2 = c1 + c2 split so that k c1 is exact, e^r from its degree-7 Taylor polynomial
+// by Horner's rule (|r| <= ln2 / 2: truncation below 2^-27 relative), scaled by 2^k exactly.
+// Every step is an explicit IEEE round-to-nearest fp32 operation (no contraction), so y is
+// reproducible bit for bit; silu(g) = g / (1 + e^-g) with an IEEE division.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ float exp_cw(float x) {
+  if (x > 0x1.62e430p+6f) return __int_as_float(0x7f800000);  // above ln(FLT_MAX)
+  if (x < -104.0f) return 0.0f;                               // below half the least subnormal
+  const float kf = rintf(__fmul_rn(x, 0x1.715476p+0f));
+  const float r = __fsub_rn(__fsub_rn(x, __fmul_rn(kf, 0x1.62e400p-1f)),
+                            __fmul_rn(kf, 0x1.7f7d1cp-20f));
+  float p = 0x1.a01a02p-13f;                                   // 1/7!
+  p = __fadd_rn(__fmul_rn(p, r), 0x1.6c16c2p-10f);             // 1/6!
+  p = __fadd_rn(__fmul_rn(p, r), 0x1.111112p-7f);              // 1/5!
+  p = __fadd_rn(__fmul_rn(p, r), 0x1.555556p-5f);              // 1/4!
+  p = __fadd_rn(__fmul_rn(p, r), 0x1.555556p-3f);              // 1/3!
+  p = __fadd_rn(__fmul_rn(p, r), 0.5f);                        // 1/2!
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  int k = static_cast<int>(kf);
+  if (k > 127) { p = __fmul_rn(p, 0x1p127f); k -= 127; }
+  if (k < -126) { p = __fmul_rn(p, 0x1p-126f); k += 126; }
+  return __fmul_rn(p, __int_as_float((k + 127) << 23));
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, exp_cw(-g))), u);
+}
+
+// y = bf16(silu(g) * u) for the 8 elements of one uint4 of gate and the matching uint4 of up.
+__device__ __forceinline__ uint4 silu_mul8(const uint4 g, const uint4 u) {
+  const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, uw[4] = {u.x, u.y, u.z, u.w};
+  uint32_t y[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    y[j] = pack_bf16x2(silu_mul(bf16_lo(gw[j]), bf16_lo(uw[j])),
+                       silu_mul(bf16_hi(gw[j]), bf16_hi(uw[j])));
+  return make_uint4(y[0], y[1], y[2], y[3]);
+}
+
+// One warp per row at a time; 4 lanes per 128-block (8 blocks per warp step), lane `sub` of a
+// block owns the 16-byte chunks sub + 4 c, c = 0 .. 3.  The gate and up loads of the next step
+// are issued before the current step is processed.
+__global__ void __launch_bounds__(512) k_silu_mul_quant(
+    const uint16_t *__restrict__ h, int64_t ldh, int64_t R, int I, uint8_t *__restrict__ q,
+    int64_t ldq, float *__restrict__ sa, int64_t lds) {
+  constexpr int LPB = 4, CPL = 4, BPS = 8;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wpc = blockDim.x >> 5;
+  const int IB = I >> 7;
+  ScaleTab *tab = reinterpret_cast<ScaleTab *>(smem);
+  const int grp = lane / LPB, sub = lane % LPB;
+  build_scale_tab(tab, threadIdx.x, blockDim.x);
+  __syncthreads();
+
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
+  for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < R; m += stride) {
+    const uint16_t *gr = h + m * ldh, *ur = gr + I;
+    uint4 gn[CPL], un[CPL];
+    {
+      const int bb = grp < IB ? grp : 0;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        gn[c] = ld_stream_v4(gr + bb * 128 + (sub + LPB * c) * 8);
+        un[c] = ld_stream_v4(ur + bb * 128 + (sub + LPB * c) * 8);
+      }
+    }
+    for (int b0 = 0; b0 < IB; b0 += BPS) {
+      const int b = b0 + grp;
+      const bool active = b < IB;
+      uint4 v[CPL];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) v[c] = silu_mul8(gn[c], un[c]);
+      if (b0 + BPS < IB) {
+        const int bn = b0 + BPS + grp < IB ? b0 + BPS + grp : b0 + BPS;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          gn[c] = ld_stream_v4(gr + bn * 128 + (sub + LPB * c) * 8);
+          un[c] = ld_stream_v4(ur + bn * 128 + (sub + LPB * c) * 8);
+        }
+      }
+      uint32_t m2 = 0u;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) m2 = absmax_uint4(m2, v[c]);
+#pragma unroll
+      for (int o = LPB / 2; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+      const QParams p = qparams_tab(absmax_finish(m2), tab);
+      uint8_t *qb = q + m * ldq + b * 128;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        const uint2 codes = quant8_f32(v[c], p);
+        if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
+      }
+      if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
+    }
+  }
+}
+
 }  // namespace fp8q

@@ -180,6 +180,19 @@ int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, i
                                  const int32_t *group_offsets, int64_t E, int64_t M, int64_t N,
                                  int64_t K, void *out_bf16, int64_t ldo, cudaStream_t stream);
 
+/* SiLU-and-mul + 1x128 quant: the front end of an MoE down projection, fed by the gate/up GEMM.
+ *   h_bf16   [R][ldh] bf16 = [gate | up]: gate in columns [0, I), up in [I, 2I), read
+ *   q_e4m3   [R][ldq] uint8 codes of y = bf16_RNE( fp32(silu(gate) * up) ), written
+ *   sa       fp32 scales, sa[kb * lds + r] (1x128 groups of y), written for r < R only
+ * silu(g) = g / (1 + e^-g) in fp32 with an IEEE division; e^x in fp32 by Cody-Waite range
+ * reduction and a degree-7 Taylor polynomial with every step an IEEE fp32 rounding (reproducible
+ * bit for bit; within 2 ulp of the true e^x).  Scales and codes as fp8q_rmsnorm_quant_token.
+ * I % 128 == 0, I <= 16384, ldh >= 2 I.  Bit-exact against the CPU oracle.  Source: FP8-RL
+ * abstract, item (i) (W8A8 linear layers of MoE models: the down projection's input is the
+ * activated gate/up output, quantized 1x128 like every activation here). */
+int fp8q_silu_mul_quant(const void *h_bf16, int64_t R, int64_t I, int64_t ldh, void *q_e4m3,
+                        int64_t ldq, float *sa, int64_t lds, cudaStream_t stream);
+
 /* Per-token (full-row) quantization, optionally fused with RMSNorm: one fp32 scale per row of K
  * (the "group size 0 = per token" mode).  Applied to a weight W [N, K] it gives the
  * per-output-channel codes and scales the per-channel GEMM below takes.

@@ -155,3 +155,13 @@ def test_rowwise_host_checks(L):
     assert call(sa=FAKE + 2) == _lib.FP8Q_ERR_ALIGN
     assert call(lda=264) == _lib.FP8Q_ERR_ALIGN
     assert call(M=0, aq=None, sa=None, out=None) == _lib.FP8Q_OK
+
+
+def test_silu_mul_quant_host_checks(L):
+    f = L.fp8q_silu_mul_quant
+    assert f(FAKE, 4, 100, 200, FAKE, 112, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE   # I % 128
+    assert f(FAKE, 4, 128, 200, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE   # ldh < 2I
+    assert f(FAKE, 8, 128, 256, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE   # lds < R
+    assert f(FAKE, 4, 128, 260, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_ALIGN   # ldh % 8
+    assert f(None, 4, 128, 256, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_NULL
+    assert f(None, 0, 128, 256, None, 128, None, 4, None) == _lib.FP8Q_OK
