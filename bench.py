@@ -341,6 +341,43 @@ def measure_rows(fq, device, steps, warmup, pk):
             "workload": f"128 experts, {R} routed rows, N={N} K={K}"}
         del a, W, wq, sw, aq, sa, out
     torch.cuda.empty_cache()
+
+    # the MoE FFN chain: quant of the routed rows -> grouped gate/up GEMM -> SiLU-and-mul + 1x128
+    # quant -> grouped down GEMM (all on the device, in this library's kernels)
+    a = dev_bf16(mo["A_gateup"], device)
+    Wgu = dev_bf16(mo["W_gateup"], device)
+    Wd = dev_bf16(mo["W_down"], device)
+    E, Ngu, Kgu = Wgu.shape
+    _, Nd, Kd = Wd.shape
+    wq_gu, sw_gu = fq.quant_weight_block(Wgu.view(E * Ngu, Kgu), "f32")
+    wq_gu, sw_gu = wq_gu.view(E, Ngu, Kgu), sw_gu.view(E, Ngu // 128, Kgu // 128)
+    wq_d, sw_d = fq.quant_weight_block(Wd.view(E * Nd, Kd), "f32")
+    wq_d, sw_d = wq_d.view(E, Nd, Kd), sw_d.view(E, Nd // 128, Kd // 128)
+    aq, sa = fq.rmsnorm_quant_token(a)
+    hgu = torch.empty((R, Ngu), dtype=torch.bfloat16, device=device)
+    aq_d = torch.empty((R, Kd), dtype=torch.uint8, device=device)
+    sa_d = torch.empty((Kd // 128, R), dtype=torch.float32, device=device)
+    out_d = torch.empty((R, Nd), dtype=torch.bfloat16, device=device)
+    fq.grouped_gemm_w8a8_block(aq, sa, wq_gu, sw_gu, off, out=hgu)
+    ms, _ = timed_loop(lambda: fq.silu_mul_quant(hgu, out_q=aq_d, out_sa=sa_d), steps, warmup,
+                       flush)
+    byts = R * Ngu * 2 + R * Kd + R * (Kd // 128) * 4
+    rows["silu_mul_quant_moe"] = {"ms": ms, "GB/s": byts / ms / 1e6, "frac": byts / ms / 1e6 / hbm,
+                                  "workload": f"[gate | up] [{R}, {Ngu}] -> codes [{R}, {Kd}]"}
+
+    def moe_chain():
+        fq.rmsnorm_quant_token(a, out_q=aq, out_sa=sa)
+        fq.grouped_gemm_w8a8_block(aq, sa, wq_gu, sw_gu, off, out=hgu)
+        fq.silu_mul_quant(hgu, out_q=aq_d, out_sa=sa_d)
+        fq.grouped_gemm_w8a8_block(aq_d, sa_d, wq_d, sw_d, off, out=out_d)
+    ms, _ = timed_loop(moe_chain, steps, warmup, flush)
+    fl = 2.0 * R * Ngu * Kgu + 2.0 * R * Nd * Kd
+    rows["moe_ffn_chain"] = {"ms": ms, "TFLOP/s": fl / ms / 1e9,
+                             "workload": f"128 experts, {R} routed rows: quant -> gate/up {Ngu}x{Kgu} "
+                                         f"-> SiLU-and-mul quant -> down {Nd}x{Kd}",
+                             "launches": 4}
+    del a, Wgu, Wd, wq_gu, sw_gu, wq_d, sw_d, aq, sa, hgu, aq_d, sa_d, out_d
+    torch.cuda.empty_cache()
     return rows
 
 

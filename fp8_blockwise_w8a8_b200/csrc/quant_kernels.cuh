@@ -505,30 +505,47 @@ __global__ void __launch_bounds__(512) k_quant_rowwise(
 // k c2 with ln 2 = c1 + c2 split so that k c1 is exact, e^r from its degree-7 Taylor polynomial
 // by Horner's rule (|r| <= ln2 / 2: truncation below 2^-27 relative), scaled by 2^k exactly.
 // Every step is an explicit IEEE round-to-nearest fp32 operation (no contraction), so y is
-// reproducible bit for bit; silu(g) = g / (1 + e^-g) with an IEEE division.
+// reproducible bit for bit; silu(g) = g / (1 + e^-g) with an IEEE division.  The kernel uses the
+// two-element form exp_cw2 (packed fp32x2 operations round each lane as the scalar ones do).
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ float exp_cw(float x) {
-  if (x > 0x1.62e430p+6f) return __int_as_float(0x7f800000);  // above ln(FLT_MAX)
-  if (x < -104.0f) return 0.0f;                               // below half the least subnormal
-  const float kf = rintf(__fmul_rn(x, 0x1.715476p+0f));
-  const float r = __fsub_rn(__fsub_rn(x, __fmul_rn(kf, 0x1.62e400p-1f)),
-                            __fmul_rn(kf, 0x1.7f7d1cp-20f));
-  float p = 0x1.a01a02p-13f;                                   // 1/7!
-  p = __fadd_rn(__fmul_rn(p, r), 0x1.6c16c2p-10f);             // 1/6!
-  p = __fadd_rn(__fmul_rn(p, r), 0x1.111112p-7f);              // 1/5!
-  p = __fadd_rn(__fmul_rn(p, r), 0x1.555556p-5f);              // 1/4!
-  p = __fadd_rn(__fmul_rn(p, r), 0x1.555556p-3f);              // 1/3!
-  p = __fadd_rn(__fmul_rn(p, r), 0.5f);                        // 1/2!
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
-  int k = static_cast<int>(kf);
-  if (k > 127) { p = __fmul_rn(p, 0x1p127f); k -= 127; }
-  if (k < -126) { p = __fmul_rn(p, 0x1p-126f); k += 126; }
-  return __fmul_rn(p, __int_as_float((k + 127) << 23));
+// e^x for two elements at once (packed fp32x2 operations round each lane as a scalar IEEE
+// operation would).  Branch-free: the polynomial runs on x clamped into range, then the results
+// out of range (inf above ln(FLT_MAX), 0 below half the least subnormal) are selected; the
+// scaling by 2^k always takes two exact steps 2^k1 * 2^(k - k1) with k1 = clamp(k, -126, 127).
+__device__ __forceinline__ float2 exp_cw2(float2 x) {
+  const float2 xc = make_float2(fminf(fmaxf(x.x, -104.0f), 0x1.62e430p+6f),
+                                fminf(fmaxf(x.y, -104.0f), 0x1.62e430p+6f));
+  const float2 t = __fmul2_rn(xc, make_float2(0x1.715476p+0f, 0x1.715476p+0f));
+  const float2 kf = make_float2(rintf(t.x), rintf(t.y));
+  const float2 nk = make_float2(-kf.x, -kf.y);
+  float2 r = __fadd2_rn(xc, __fmul2_rn(nk, make_float2(0x1.62e400p-1f, 0x1.62e400p-1f)));
+  r = __fadd2_rn(r, __fmul2_rn(nk, make_float2(0x1.7f7d1cp-20f, 0x1.7f7d1cp-20f)));
+  float2 p = make_float2(0x1.a01a02p-13f, 0x1.a01a02p-13f);
+  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0x1.6c16c2p-10f, 0x1.6c16c2p-10f));
+  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0x1.111112p-7f, 0x1.111112p-7f));
+  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0x1.555556p-5f, 0x1.555556p-5f));
+  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0x1.555556p-3f, 0x1.555556p-3f));
+  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0.5f, 0.5f));
+  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(1.0f, 1.0f));
+  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(1.0f, 1.0f));
+  const int ka = static_cast<int>(kf.x), kb = static_cast<int>(kf.y);
+  const int ka1 = min(max(ka, -126), 127), kb1 = min(max(kb, -126), 127);
+  p = __fmul2_rn(p, make_float2(__int_as_float((ka1 + 127) << 23), __int_as_float((kb1 + 127) << 23)));
+  p = __fmul2_rn(p, make_float2(__int_as_float((ka - ka1 + 127) << 23),
+                                __int_as_float((kb - kb1 + 127) << 23)));
+  const float inf = __int_as_float(0x7f800000);
+  p.x = x.x > 0x1.62e430p+6f ? inf : (x.x < -104.0f ? 0.0f : p.x);
+  p.y = x.y > 0x1.62e430p+6f ? inf : (x.y < -104.0f ? 0.0f : p.y);
+  return p;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) {
-  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, exp_cw(-g))), u);
+// silu(g) = g / (1 + e^-g) given e = e^-g.  Where 1 + e^-g is infinite the quotient is a zero
+// with g's sign, selected after dividing by 1 instead (an infinite divisor would take the
+// division's slow path).
+__device__ __forceinline__ float silu_from_exp(float g, float e) {
+  const float d = __fadd_rn(1.0f, e);
+  const bool big = d == __int_as_float(0x7f800000);
+  return big ? __int_as_float(__float_as_int(g) & 0x80000000) : __fdiv_rn(g, big ? 1.0f : d);
 }
 
 // y = bf16(silu(g) * u) for the 8 elements of one uint4 of gate and the matching uint4 of up.
@@ -536,19 +553,23 @@ __device__ __forceinline__ uint4 silu_mul8(const uint4 g, const uint4 u) {
   const uint32_t gw[4] = {g.x, g.y, g.z, g.w}, uw[4] = {u.x, u.y, u.z, u.w};
   uint32_t y[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    y[j] = pack_bf16x2(silu_mul(bf16_lo(gw[j]), bf16_lo(uw[j])),
-                       silu_mul(bf16_hi(gw[j]), bf16_hi(uw[j])));
+  for (int j = 0; j < 4; ++j) {
+    const float2 gg = make_float2(bf16_lo(gw[j]), bf16_hi(gw[j]));
+    const float2 e = exp_cw2(make_float2(-gg.x, -gg.y));
+    const float2 sl = make_float2(silu_from_exp(gg.x, e.x), silu_from_exp(gg.y, e.y));
+    const float2 v = __fmul2_rn(sl, make_float2(bf16_lo(uw[j]), bf16_hi(uw[j])));
+    y[j] = pack_bf16x2(v.x, v.y);
+  }
   return make_uint4(y[0], y[1], y[2], y[3]);
 }
 
-// One warp per row at a time; 4 lanes per 128-block (8 blocks per warp step), lane `sub` of a
-// block owns the 16-byte chunks sub + 4 c, c = 0 .. 3.  The gate and up loads of the next step
+// One warp per row at a time; 8 lanes per 128-block (4 blocks per warp step), lane `sub` of a
+// block owns the 16-byte chunks sub + 8 c, c = 0, 1.  The gate and up loads of the next step
 // are issued before the current step is processed.
 __global__ void __launch_bounds__(512) k_silu_mul_quant(
     const uint16_t *__restrict__ h, int64_t ldh, int64_t R, int I, uint8_t *__restrict__ q,
     int64_t ldq, float *__restrict__ sa, int64_t lds) {
-  constexpr int LPB = 4, CPL = 4, BPS = 8;
+  constexpr int LPB = 8, CPL = 2, BPS = 4;
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int wpc = blockDim.x >> 5;
