@@ -20,6 +20,10 @@ bf16 tensors are returned as numpy ``uint16`` bit patterns (host) or torch ``bfl
                    (Gumbel-top-k); rows sorted by expert; gate/up input = the token rows
                    gathered in routed order; down input ~ N(0,1) [routed, 768];
                    W_gateup [128, 1536, 2048], W_down [128, 2048, 768] ~ N(0, 0.02); seed 4
+* attention output projection (wo_a): o [8192, 32 heads, 512] ~ N(0,1) with the last 64 dims
+                   of each head the rotary part; positions ~ U[0, 16384); cos/sin caches
+                   [16384, 32] of the angle p * 10000^(-2i/64), computed in float64 and rounded
+                   to fp32; 4 head groups, W_wo_a [4, 1024, 8 * 512] ~ N(0, 0.02); seed 5
 """
 import numpy as np
 import torch
@@ -125,4 +129,25 @@ def moe(tokens: int = 4096, hidden: int = 2048, experts: int = 128, topk: int = 
     if with_weights:
         out["W_gateup"] = randn_bf16((experts, 2 * ffn, hidden), 0.02, seed, 3)
         out["W_down"] = randn_bf16((experts, hidden, ffn), 0.02, seed, 4)
+    return out
+
+
+def rope_caches(max_pos: int, rope_dim: int, base: float = 10000.0):
+    """fp32 cos/sin tables [max_pos, rope_dim / 2] of the angles p * base^(-2i / rope_dim)."""
+    inv_freq = base ** (-np.arange(0, rope_dim, 2, dtype=np.float64) / rope_dim)
+    ang = np.arange(max_pos, dtype=np.float64)[:, None] * inv_freq[None, :]
+    return np.cos(ang).astype(np.float32), np.sin(ang).astype(np.float32)
+
+
+def wo_a(tokens: int = 8192, heads: int = 32, head_dim: int = 512, rope_dim: int = 64,
+         groups: int = 4, out_per_group: int = 1024, max_pos: int = 16384,
+         with_weight: bool = True):
+    seed = 5
+    r = rng_for(seed, 1)
+    cos, sin = rope_caches(max_pos, rope_dim)
+    out = {"o": randn_bf16((tokens, heads, head_dim), 1.0, seed, 0),
+           "positions": r.integers(0, max_pos, tokens).astype(np.int64),
+           "cos": cos, "sin": sin}
+    if with_weight:
+        out["W"] = randn_bf16((groups, out_per_group, heads // groups * head_dim), 0.02, seed, 2)
     return out

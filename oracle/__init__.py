@@ -61,6 +61,11 @@ def lib():
         L.oracle_silu_mul_quant.restype = None
         L.oracle_silu_mul_bf16.argtypes = [P, I64, I64, I64, P]
         L.oracle_silu_mul_bf16.restype = None
+        L.oracle_inverse_rope_bf16.argtypes = [P, P, P, P, I64, I64, I64, I64, ctypes.c_int, P]
+        L.oracle_inverse_rope_bf16.restype = None
+        L.oracle_inverse_rope_quant.argtypes = [P, P, P, P, I64, I64, I64, I64, ctypes.c_int,
+                                                ctypes.c_int, P, P, I64]
+        L.oracle_inverse_rope_quant.restype = None
         L.oracle_quant_rowwise.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64, P]
         L.oracle_quant_rowwise.restype = None
         L.oracle_gemm_w8a8_rowwise_rows.argtypes = [P, I64, P, P, I64, P, I64, I64, P, I64, P, P]
@@ -258,6 +263,37 @@ def silu_mul_quant(h_bf16: np.ndarray, lds: int = None):
     q = np.empty((R, I), np.uint8)
     sa = np.zeros((I // 128, lds), np.float32)
     lib().oracle_silu_mul_quant(_ptr(h), R, I, I2, _ptr(q), I, _ptr(sa), lds)
+    return q, sa
+
+
+def inverse_rope_bf16(o_bf16: np.ndarray, positions, cos_cache, sin_cache, rope_dim: int,
+                      interleaved: bool = True):
+    """The bf16 inverse RoPE of reading R9: o [T, H, D] -> y [T, H*D]."""
+    o = _c(o_bf16, np.uint16)
+    T, H, D = o.shape
+    pos = _c(np.asarray(positions), np.int64)
+    c = _c(cos_cache, np.float32)
+    sn = _c(sin_cache, np.float32)
+    y = np.empty((T, H * D), np.uint16)
+    lib().oracle_inverse_rope_bf16(_ptr(o), _ptr(pos), _ptr(c), _ptr(sn), T, H, D, rope_dim,
+                                   int(interleaved), _ptr(y))
+    return y
+
+
+def inverse_rope_quant(o_bf16: np.ndarray, positions, cos_cache, sin_cache, rope_dim: int,
+                       interleaved: bool = True, fmt: int = 0, lds: int = None):
+    """Inverse RoPE + 1x128 quant (reading R9): codes [T, H*D] and sa [H*D/128, lds]
+    (fmt 0: fp32 amax/448 scales; fmt 1: E8M0 powers of two stored as fp32)."""
+    o = _c(o_bf16, np.uint16)
+    T, H, D = o.shape
+    lds = T if lds is None else lds
+    pos = _c(np.asarray(positions), np.int64)
+    c = _c(cos_cache, np.float32)
+    sn = _c(sin_cache, np.float32)
+    q = np.empty((T, H * D), np.uint8)
+    sa = np.zeros((H * D // 128, lds), np.float32)
+    lib().oracle_inverse_rope_quant(_ptr(o), _ptr(pos), _ptr(c), _ptr(sn), T, H, D, rope_dim,
+                                    int(interleaved), int(fmt), _ptr(q), _ptr(sa), lds)
     return q, sa
 
 

@@ -52,6 +52,16 @@
  *       bf16_RNE( fp32( silu(g_k) * u_k ) ) with silu(g) = g / (1 + e^-g) in fp32 (IEEE division)
  *       and e^x in fp32 by Cody-Waite range reduction and a degree-7 Taylor polynomial (below);
  *       then the 1x128 token quant of R1 on y.
+ *   R9  inverse RoPE + group-128 quant [DSv4-WOA section 3: inverse_rope_group_quant(o [T,
+ *       heads, head_dim], positions, cos cache, sin cache, num_groups, quant_group_size=128)
+ *       feeding a batched per-group GEMM]: the rotary part is the last R dims of each head,
+ *       rotated by -theta_i in pairs (a, b) = (2i, 2i+1) (interleaved) or (i, i+R/2) (halves):
+ *       with c = cos[p][i], s = sin[p][i] (fp32 caches [max_pos][R/2]), y_a = bf16(fp32(x_a c)
+ *       + fp32(x_b s)) and y_b = bf16(fp32(x_b c) - fp32(x_a s)), each product and sum one fp32
+ *       rounding; the other dims pass through.  Then 1x128 groups along the flattened
+ *       heads x head_dim row of each token, scales K-block-major as R5 (each head group's
+ *       K-blocks are then contiguous).  The scale is R1's fp32 amax/448, or, since the GEMM that
+ *       follows on the page takes MX (E8M0) scales, R2's power of two, stored as its fp32 value.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math -fopenmp.
  * fp32 arithmetic below relies on FLT_EVAL_METHOD == 0 (SSE on x86-64), so every float
@@ -373,6 +383,95 @@ void oracle_silu_mul_bf16(const uint16_t *h, int64_t R, int64_t I, int64_t ldh, 
             float g = bf16_to_f32(h[m * ldh + k]), u = bf16_to_f32(h[m * ldh + I + k]);
             y[m * I + k] = f32_to_bf16_rne(oracle_silu_f32(g) * u);
         }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Inverse RoPE + group-128 quant [DSv4-WOA section 3], reading R9                              */
+/* ------------------------------------------------------------------------------------------ */
+
+/* The inverse rotation of one rotary element of a head.  x is the head (D bf16 values), j the
+ * index inside the rotary part (0 <= j < R), cs/sn the cache rows of the token's position.
+ * Pairs are (2i, 2i+1) when interleaved, else (i, i + R/2); both rotate by -theta_i:
+ * first = x_a cos + x_b sin, second = x_b cos - x_a sin, every product and sum rounded once
+ * in fp32, the result rounded to bf16. */
+static float inverse_rope_element(const uint16_t *x, int64_t D, int64_t R, int64_t j,
+                                  const float *cs, const float *sn, int interleaved) {
+    int64_t half = R / 2, i, ia, ib;
+    int second;
+    if (interleaved) {
+        i = j / 2;
+        second = (int)(j % 2);
+        ia = 2 * i;
+        ib = 2 * i + 1;
+    } else {
+        i = j % half;
+        second = j >= half;
+        ia = i;
+        ib = i + half;
+    }
+    float xa = bf16_to_f32(x[D - R + ia]), xb = bf16_to_f32(x[D - R + ib]);
+    float c = cs[i], s = sn[i];
+    float v;
+    if (!second) {
+        float p = xa * c, r = xb * s;
+        v = p + r;
+    } else {
+        float p = xb * c, r = xa * s;
+        v = p - r;
+    }
+    return bf16_to_f32(f32_to_bf16_rne(v));
+}
+
+/* o bf16 [T][H][D] (contiguous), positions [T], cos/sin fp32 [max_pos][R/2].  Writes the
+ * rotated bf16 values y [T][H*D] (what an unfused inverse RoPE would write to memory). */
+void oracle_inverse_rope_bf16(const uint16_t *o, const int64_t *pos, const float *cosc,
+                              const float *sinc, int64_t T, int64_t H, int64_t D, int64_t R,
+                              int interleaved, uint16_t *y) {
+    int64_t half = R / 2;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t h = 0; h < H; ++h) {
+            const uint16_t *x = o + (t * H + h) * D;
+            const float *cs = cosc + pos[t] * half, *sn = sinc + pos[t] * half;
+            for (int64_t d = 0; d < D; ++d)
+                y[(t * H + h) * D + d] =
+                    d < D - R ? x[d]
+                              : f32_to_bf16_rne(inverse_rope_element(x, D, R, d - (D - R), cs,
+                                                                     sn, interleaved));
+        }
+}
+
+/* The fused front end: inverse RoPE, then 1x128 quant along each token's flattened H*D row.
+ * Codes q [T][H*D]; scales sa[kb * lds + t], fp32 amax/448 when fmt == 0 (reading R1), the
+ * E8M0 power of two of reading R2 stored as its fp32 value when fmt == 1. */
+void oracle_inverse_rope_quant(const uint16_t *o, const int64_t *pos, const float *cosc,
+                               const float *sinc, int64_t T, int64_t H, int64_t D, int64_t R,
+                               int interleaved, int fmt, uint8_t *q, float *sa, int64_t lds) {
+    int64_t K = H * D, KB = K / 128, half = R / 2;
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t t = 0; t < T; ++t) {
+        const float *cs = cosc + pos[t] * half, *sn = sinc + pos[t] * half;
+        for (int64_t kb = 0; kb < KB; ++kb) {
+            float y[128];
+            for (int j = 0; j < 128; ++j) {
+                int64_t k = kb * 128 + j, h = k / D, d = k % D;
+                const uint16_t *x = o + (t * H + h) * D;
+                y[j] = d < D - R ? bf16_to_f32(x[d])
+                                 : inverse_rope_element(x, D, R, d - (D - R), cs, sn,
+                                                        interleaved);
+            }
+            uint8_t *qg = q + t * K + kb * 128;
+            if (fmt == 0) {
+                sa[kb * lds + t] = quant_group_1x128(y, qg);
+            } else {
+                float amax = 0.0f;
+                for (int j = 0; j < 128; ++j)
+                    if (fabsf(y[j]) > amax) amax = fabsf(y[j]);
+                float s = e8m0_value(e8m0_from_amax(amax));
+                for (int j = 0; j < 128; ++j) qg[j] = oracle_e4m3_encode(y[j] / s);
+                sa[kb * lds + t] = s;
+            }
+        }
+    }
 }
 
 /* ------------------------------------------------------------------------------------------ */
