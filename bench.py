@@ -378,6 +378,50 @@ def measure_rows(fq, device, steps, warmup, pk):
                              "launches": 4}
     del a, Wgu, Wd, wq_gu, sw_gu, wq_d, sw_d, aq, sa, hgu, aq_d, sa_d, out_d
     torch.cuda.empty_cache()
+
+    # attention output projection (wo_a): inverse RoPE + 1x128 quant, then the block-diagonal
+    # GEMM over the head groups (E8M0 scales on both sides, as the page's MX-scaled GEMM)
+    wa = inputs.wo_a()
+    T, H, D = wa["o"].shape
+    G, N_g, K_g = wa["W"].shape
+    Kt = H * D
+    o_d = dev_bf16(wa["o"], device)
+    pos_d = torch.from_numpy(wa["positions"]).to(device)
+    cos_d = torch.from_numpy(wa["cos"]).to(device)
+    sin_d = torch.from_numpy(wa["sin"]).to(device)
+    W = dev_bf16(wa["W"], device)
+    wq, sw = fq.quant_weight_block(W.view(G * N_g, K_g), "e8m0")
+    wq, sw = wq.view(G, N_g, K_g), sw.view(G, N_g // 128, K_g // 128)
+    q_d = torch.empty((T, Kt), dtype=torch.uint8, device=device)
+    sa_d = torch.empty((Kt // 128, T), dtype=torch.float32, device=device)
+    out_d = torch.empty((T, G * N_g), dtype=torch.bfloat16, device=device)
+    byts = T * Kt * 2 + T * Kt + T * (Kt // 128) * 4 + T * 8 + T * 64 * 4
+    for fmt, tag in ((fq.FP8Q_SCALE_E8M0, "e8m0"), (fq.FP8Q_SCALE_F32, "f32")):
+        ms, _ = timed_loop(lambda: fq.inverse_rope_quant(o_d, pos_d, cos_d, sin_d, 64, True, fmt,
+                                                         out_q=q_d, out_sa=sa_d),
+                           steps, warmup, flush)
+        rows[f"inverse_rope_quant_wo_a_{tag}"] = {
+            "ms": ms, "GB/s": byts / ms / 1e6, "frac": byts / ms / 1e6 / hbm,
+            "workload": f"o [{T}, {H}, {D}] (64 rotary dims, interleaved) -> codes [{T}, {Kt}]"}
+    fq.inverse_rope_quant(o_d, pos_d, cos_d, sin_d, 64, True, fq.FP8Q_SCALE_E8M0, out_q=q_d,
+                          out_sa=sa_d)
+    fl = 2.0 * T * G * N_g * K_g
+    ms, _ = timed_loop(lambda: fq.gemm_w8a8_block_diag(q_d, sa_d, wq, sw, out=out_d), steps,
+                       warmup, flush)
+    rows["gemm_diag_wo_a"] = {"ms": ms, "TFLOP/s": fl / ms / 1e9,
+                              "frac_fp8_sustained": fl / ms / 1e9 / (2.0 * pk["bf16_sustained"]),
+                              "workload": f"{G} head groups: [{T}, {K_g}] x [{N_g}, {K_g}] each"}
+
+    def wo_a_chain():
+        fq.inverse_rope_quant(o_d, pos_d, cos_d, sin_d, 64, True, fq.FP8Q_SCALE_E8M0,
+                              out_q=q_d, out_sa=sa_d)
+        fq.gemm_w8a8_block_diag(q_d, sa_d, wq, sw, out=out_d)
+    ms, _ = timed_loop(wo_a_chain, steps, warmup, flush)
+    rows["wo_a_chain"] = {"ms": ms, "TFLOP/s": fl / ms / 1e9,
+                          "workload": f"inverse RoPE quant -> {G}-group GEMM, {T} tokens",
+                          "launches": 2}
+    del o_d, pos_d, cos_d, sin_d, W, wq, sw, q_d, sa_d, out_d
+    torch.cuda.empty_cache()
     return rows
 
 

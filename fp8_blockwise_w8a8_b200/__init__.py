@@ -16,14 +16,15 @@ import torch
 
 from . import _lib
 from ._lib import (FP8Q_ERR_ALIGN, FP8Q_ERR_ARCH, FP8Q_ERR_ARG, FP8Q_ERR_LAUNCH, FP8Q_ERR_NULL,
-                   FP8Q_ERR_SHAPE, FP8Q_ERR_TIMEOUT, FP8Q_OK, FP8Q_SCALE_E8M0, FP8Q_SCALE_F32,
+                   FP8Q_ERR_RANGE, FP8Q_ERR_SHAPE, FP8Q_ERR_TIMEOUT, FP8Q_OK, FP8Q_SCALE_E8M0, FP8Q_SCALE_F32,
                    Fp8qError)
 
 import ctypes
 
 __all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
-           "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant",
+           "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant", "inverse_rope_quant",
+           "gemm_w8a8_block_diag",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -170,6 +171,57 @@ def silu_mul_quant(h: torch.Tensor, lds=None, out_q=None, out_sa=None, stream=No
                                         sa.stride(0), _stream(stream))
     _lib.check(st, "fp8q_silu_mul_quant")
     return q, sa
+
+
+def inverse_rope_quant(o: torch.Tensor, positions: torch.Tensor, cos_cache: torch.Tensor,
+                       sin_cache: torch.Tensor, rope_dim: int, interleaved: bool = True,
+                       fmt=FP8Q_SCALE_F32, lds=None, out_q=None, out_sa=None, stream=None):
+    """Attention output o bf16 [T, H, D] (token stride o.stride(0); heads contiguous) ->
+    (codes uint8 [T, H*D], sa fp32 [H*D/128, lds]): inverse RoPE of the last rope_dim dims of
+    each head at the tokens' positions (int64 [T]; fp32 cos/sin caches [max_pos, rope_dim/2]),
+    then 1x128 quant; fmt SCALE_E8M0 gives power-of-two scales (stored as fp32)."""
+    T, H, D = o.shape
+    if o.stride(2) != 1 or o.stride(1) != D:
+        raise ValueError("o must have contiguous heads: strides (ldo, D, 1)")
+    K = H * D
+    if lds is None:
+        lds = max(4, (T + 3) // 4 * 4)
+    q = torch.empty((T, K), dtype=torch.uint8, device=o.device) if out_q is None else out_q
+    sa = (torch.empty((K // 128, lds), dtype=torch.float32, device=o.device)
+          if out_sa is None else out_sa)
+    max_pos = cos_cache.shape[0] if cos_cache is not None else 0
+    if rope_dim > 0:
+        for t, name in ((cos_cache, "cos_cache"), (sin_cache, "sin_cache")):
+            if (t.dtype != torch.float32 or not t.is_contiguous()
+                    or tuple(t.shape) != (max_pos, rope_dim // 2)):
+                raise ValueError(f"{name} must be contiguous fp32 [max_pos, rope_dim/2]")
+        if positions.dtype != torch.int64 or positions.numel() != T or not positions.is_contiguous():
+            raise ValueError("positions must be a contiguous int64 tensor of T entries")
+    f = scale_format(fmt)
+    st = _lib.lib().fp8q_inverse_rope_quant(
+        _ptr(o), o.stride(0), _ptr(positions), _ptr(cos_cache), _ptr(sin_cache), max_pos, T, H,
+        D, int(rope_dim), int(bool(interleaved)), f, _ptr(q), _ld(q), _ptr(sa), sa.stride(0),
+        _stream(stream))
+    _lib.check(st, "fp8q_inverse_rope_quant")
+    return q, sa
+
+
+def gemm_w8a8_block_diag(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                         fmt=None, out=None, stream=None):
+    """Per-group (block-diagonal) GEMM: codes aq [M, G*K_g] (scales sa [G*K_g/128, lds]) with
+    weights wq [G, N_g, K_g] (scales sw [G, N_g/128, K_g/128]) -> bf16 [M, G*N_g], group g's
+    columns from A's g-th K-slice and W[g]."""
+    f = scale_format(sw.dtype if fmt is None else fmt)
+    G, N_g, K_g = wq.shape
+    M = aq.shape[0]
+    if wq.stride(0) != N_g * wq.stride(1) or wq.stride(2) != 1:
+        raise ValueError("wq must be [G, N_g, ldw] with group stride N_g * ldw")
+    o = torch.empty((M, G * N_g), dtype=torch.bfloat16, device=aq.device) if out is None else out
+    st = _lib.lib().fp8q_gemm_w8a8_block_diag(_ptr(aq), _ld(aq), _ptr(sa), sa.stride(0),
+                                              _ptr(wq), wq.stride(1), _ptr(sw), f, G, M, N_g,
+                                              K_g, _ptr(o), _ld(o), _stream(stream))
+    _lib.check(st, "fp8q_gemm_w8a8_block_diag")
+    return o
 
 
 def quant_rowwise(x: torch.Tensor, gamma=None, eps: float = 1e-6, out_q=None, out_s=None,

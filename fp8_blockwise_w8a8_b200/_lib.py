@@ -17,6 +17,7 @@ FP8Q_ERR_LAUNCH = 5
 FP8Q_ERR_TIMEOUT = 6
 FP8Q_ERR_ARG = 7
 FP8Q_ERR_TOO_LARGE = 8
+FP8Q_ERR_RANGE = 9
 
 FP8Q_SCALE_F32 = 0
 FP8Q_SCALE_E8M0 = 1
@@ -39,6 +40,10 @@ SIGNATURES = {
     "fp8q_grouped_gemm_w8a8_block": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _P, _I64, _I64,
                                           _I64, _I64, _P, _I64, _P]),
     "fp8q_silu_mul_quant": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _P]),
+    "fp8q_inverse_rope_quant": (_I, [_P, _I64, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I,
+                                     _P, _I64, _P, _I64, _P]),
+    "fp8q_gemm_w8a8_block_diag": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64, _I64,
+                                       _I64, _P, _I64, _P]),
     "fp8q_quant_rowwise": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "fp8q_gemm_w8a8_rowwise": (_I, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I64, _P]),
     "fp8q_check_device_error": (_I, [_P]),

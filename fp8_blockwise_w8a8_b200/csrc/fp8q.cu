@@ -170,13 +170,15 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
                 const void *wq, int64_t ldw, const void *sw, int sw_fmt,
                 const int32_t *group_offsets, int64_t E, int64_t M, int64_t N, int64_t K,
                 void *out, int64_t ldo, cudaStream_t stream, int splits = 1,
-                void *workspace = nullptr) {
+                void *workspace = nullptr, int64_t groups = 0) {
   DeviceState *st = nullptr;
   int rc = device_state(&st);
   if (rc != FP8Q_OK) return rc;
   if ((rc = get_encoder()) != FP8Q_OK) return rc;
   CUtensorMap tm_a, tm_b;
-  if ((rc = make_u8_map(&tm_a, aq, M, K, lda, fp8q::kBM)) != FP8Q_OK) return rc;
+  // block-diagonal (groups > 0): A holds the groups' K-slices side by side, [M][groups * K]
+  const int64_t a_cols = groups > 0 ? groups * K : K;
+  if ((rc = make_u8_map(&tm_a, aq, M, a_cols, lda, fp8q::kBM)) != FP8Q_OK) return rc;
   const int64_t b_rows = grouped ? E * N : N;
   if ((rc = make_u8_map(&tm_b, wq, b_rows, K, ldw, fp8q::kBN)) != FP8Q_OK) return rc;
   fp8q::GemmArgs a;
@@ -195,6 +197,7 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
   a.num_m = static_cast<int>((M + fp8q::kBM - 1) / fp8q::kBM);
   a.splits = splits;
   a.ws = static_cast<float *>(workspace);
+  a.n_tiles_per_group = groups > 0 ? static_cast<int>(N / groups / fp8q::kBN) : 0;
   // Upper bound of the tile count (grouped: every expert may add one partial m-tile).
   const int64_t tiles = (static_cast<int64_t>(a.num_m) + (grouped ? E : 0)) * a.num_n;
   const int64_t units = tiles * splits;
@@ -217,7 +220,7 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
 
 extern "C" {
 
-int fp8q_abi_version(void) { return (1 << 16) | 2; }
+int fp8q_abi_version(void) { return (1 << 16) | 3; }
 
 const char *fp8q_status_string(int status) {
   switch (status) {
@@ -229,6 +232,7 @@ const char *fp8q_status_string(int status) {
     case FP8Q_ERR_LAUNCH: return "CUDA runtime or launch failure";
     case FP8Q_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (outputs incomplete)";
     case FP8Q_ERR_ARG: return "enum argument out of range";
+    case FP8Q_ERR_RANGE: return "an index input (a RoPE position) was outside its table; that row was not written";
     case FP8Q_ERR_TOO_LARGE: return "problem needs more split-K scratch than the library's static 24 MiB buffer (use fp8q_gemm_w8a8_block_splitk with a workspace, or fewer splits)";
     default: return "unknown status";
   }
@@ -320,6 +324,21 @@ int fp8q_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t l
   if (sw_fmt == FP8Q_SCALE_F32 && (reinterpret_cast<uintptr_t>(sw) & 3u)) return FP8Q_ERR_ALIGN;
   return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, N, K, out_bf16,
                      ldo, stream);
+}
+
+int fp8q_gemm_w8a8_block_diag(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                              const void *wq, int64_t ldw, const void *sw, int sw_fmt,
+                              int64_t G, int64_t M, int64_t N_g, int64_t K_g, void *out_bf16,
+                              int64_t ldo, cudaStream_t stream) {
+  if (G <= 0 || G > (1 << 16) || N_g <= 0 || N_g % fp8q::kBN) return FP8Q_ERR_SHAPE;
+  if (N_g > (1 << 30) / G || K_g > (1 << 30) / G) return FP8Q_ERR_SHAPE;
+  int rc = check_gemm_common(aq, lda, sa, lds, wq, ldw, sw, sw_fmt, M, G * N_g, K_g, out_bf16,
+                             ldo);
+  if (rc != FP8Q_OK || M == 0) return rc;
+  if (lda < G * K_g) return FP8Q_ERR_SHAPE;
+  if (sw_fmt == FP8Q_SCALE_F32 && (reinterpret_cast<uintptr_t>(sw) & 3u)) return FP8Q_ERR_ALIGN;
+  return launch_gemm(false, aq, lda, sa, lds, wq, ldw, sw, sw_fmt, nullptr, 1, M, G * N_g, K_g,
+                     out_bf16, ldo, stream, 1, nullptr, G);
 }
 
 int fp8q_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int splits,
@@ -495,6 +514,56 @@ int fp8q_silu_mul_quant(const void *h_bf16, int64_t R, int64_t I, int64_t ldh, v
   fp8q::k_silu_mul_quant<<<grid, 32 * best_wpc, smem, stream>>>(
       static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
       static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
+  return launch_status();
+}
+
+int fp8q_inverse_rope_quant(const void *o_bf16, int64_t ldo, const int64_t *positions,
+                            const float *cos_cache, const float *sin_cache, int64_t max_pos,
+                            int64_t T, int64_t H, int64_t D, int64_t rope_dim, int interleaved,
+                            int scale_fmt, void *q_e4m3, int64_t ldq, float *sa, int64_t lds,
+                            cudaStream_t stream) {
+  if (scale_fmt != FP8Q_SCALE_F32 && scale_fmt != FP8Q_SCALE_E8M0) return FP8Q_ERR_ARG;
+  if (interleaved != 0 && interleaved != 1) return FP8Q_ERR_ARG;
+  if (T < 0 || H <= 0 || D <= 0 || D % 8 || rope_dim < 0 || rope_dim > D || rope_dim % 8)
+    return FP8Q_ERR_SHAPE;
+  if (!interleaved && rope_dim % 16) return FP8Q_ERR_SHAPE;
+  if (H > (1 << 24) / D) return FP8Q_ERR_SHAPE;
+  const int64_t K = H * D;
+  if (K % 128 || ldo < K || ldq < K || lds < T) return FP8Q_ERR_SHAPE;
+  if (rope_dim > 0 && max_pos <= 0) return FP8Q_ERR_SHAPE;
+  if (T == 0) return FP8Q_OK;
+  if (!o_bf16 || !q_e4m3 || !sa) return FP8Q_ERR_NULL;
+  if (rope_dim > 0 && (!positions || !cos_cache || !sin_cache)) return FP8Q_ERR_NULL;
+  if (!aligned16(o_bf16) || !aligned16(q_e4m3) || !aligned16(sa) || ldo % 8 || ldq % 16 ||
+      lds % 4)
+    return FP8Q_ERR_ALIGN;
+  if (rope_dim > 0 && (!aligned16(cos_cache) || !aligned16(sin_cache) ||
+                       reinterpret_cast<uintptr_t>(positions) % 8))
+    return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  using Kernel = void (*)(const uint16_t *, int64_t, const int64_t *, const float *,
+                          const float *, int64_t, int64_t, int, int, int, uint8_t *, int64_t,
+                          float *, int64_t);
+  const Kernel k = scale_fmt == FP8Q_SCALE_F32
+                       ? (interleaved ? fp8q::k_inverse_rope_quant<fp8q::kScaleF32, true>
+                                      : fp8q::k_inverse_rope_quant<fp8q::kScaleF32, false>)
+                       : (interleaved ? fp8q::k_inverse_rope_quant<fp8q::kScaleE8M0, true>
+                                      : fp8q::k_inverse_rope_quant<fp8q::kScaleE8M0, false>);
+  const int smem = static_cast<int>(sizeof(fp8q::ScaleTab));
+  const int wpc = 16;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 32 * wpc, smem) != cudaSuccess ||
+      per_sm == 0)
+    return FP8Q_ERR_LAUNCH;
+  const int64_t need = (T + wpc - 1) / wpc;
+  const int64_t cap = static_cast<int64_t>(st->sms) * per_sm;
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  k<<<grid, 32 * wpc, smem, stream>>>(static_cast<const uint16_t *>(o_bf16), ldo, positions,
+                                     cos_cache, sin_cache, max_pos, T, static_cast<int>(D),
+                                     static_cast<int>(rope_dim), static_cast<int>(K),
+                                     static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
   return launch_status();
 }
 

@@ -91,6 +91,8 @@ struct GemmArgs {
   int num_m;            // dense: ceil(M / 128)
   int splits;           // K-splits per tile (1: no split)
   float *ws;            // splits > 1: fp32 partials, [tile][split][2][32][128] float4
+  int n_tiles_per_group;  // block-diagonal: 256-column tiles per group (0: plain dense); group
+                          // g of the output reads A's K-blocks [g K/128, (g + 1) K/128)
 };
 
 // Work unit u covers tile u / splits and the K-blocks [kb0, kb1) of split u % splits.
@@ -113,6 +115,7 @@ struct Tile {
   int n0;        // first column
   int b_row;     // first row of the tile in the B tensor map (expert * N + n0)
   int e;         // expert (0 when dense)
+  int a_kb;      // first K-block of the tile's slice of A (block-diagonal groups; else 0)
 };
 
 // Dense rasterization: groups of kGroupM m-blocks, m fastest inside a group, so that the CTAs
@@ -129,6 +132,7 @@ __device__ __forceinline__ Tile dense_tile(const GemmArgs &a, int t) {
   tl.row_end = a.M;
   tl.b_row = tl.n0;
   tl.e = 0;
+  tl.a_kb = a.n_tiles_per_group ? (tl.n0 / kBN) / a.n_tiles_per_group * (a.K / kBK) : 0;
   return tl;
 }
 
@@ -149,6 +153,7 @@ __device__ __forceinline__ Tile grouped_tile(const GemmArgs &a, const int *s_off
   tl.row_end = s_off[lo + 1];
   tl.n0 = nb * kBN;
   tl.b_row = lo * a.N + tl.n0;
+  tl.a_kb = 0;
   return tl;
 }
 
@@ -317,7 +322,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
             if (!wait_one(bar_empty + 8 * s, ph ^ 1u, s_abort)) { ok = false; break; }
             mbar_arrive_expect_tx(bar_full + 8 * s, kStageBytes);
-            tma_load_2d(sbase + kOffA + s * kTileABytes, &tm_a, kb * kBK, tl.m0, bar_full + 8 * s);
+            tma_load_2d(sbase + kOffA + s * kTileABytes, &tm_a, (tl.a_kb + kb) * kBK, tl.m0,
+                        bar_full + 8 * s);
             tma_load_2d(sbase + kOffB + s * kTileBBytes, &tm_b, kb * kBK, tl.b_row,
                         bar_full + 8 * s);
           }
@@ -436,7 +442,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // (measured faster for the short, many-tile grouped problems).
       const int row = tl.m0 + 32 * q + lane;
       const bool row_ok = row < tl.row_end;
-      const float *sa_row = args.sa + row;
+      const float *sa_row = args.sa + row + static_cast<int64_t>(tl.a_kb) * args.lds;
       float sa0 = 0.0f, sa1 = 0.0f;
       if constexpr (!GROUPED) {
         sa0 = (row_ok && un.kb0 < un.kb1)

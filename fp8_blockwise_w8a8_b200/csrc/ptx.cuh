@@ -26,6 +26,35 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Packed fp32x2 multiply and add with an explicit round-to-nearest-even modifier.  PTX never
+// contracts an add or multiply that names its rounding mode into a fused multiply-add, so each
+// lane rounds exactly as the scalar IEEE operation does, wherever the result goes next.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float2 a) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(a.x), "f"(a.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 f2_unpack(uint64_t d) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+  return r;
+}
+
+__device__ __forceinline__ float2 f2_mul_rn(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a)), "l"(f2_pack(b)));
+  return f2_unpack(d);
+}
+
+__device__ __forceinline__ float2 f2_add_rn(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a)), "l"(f2_pack(b)));
+  return f2_unpack(d);
+}
+
+// ---------------------------------------------------------------------------------------------
 // E4M3 conversion: round-to-nearest-even with saturation to the largest finite value (+-448).
 // `hi` lands in bits [15:8], `lo` in bits [7:0].
 // ---------------------------------------------------------------------------------------------

@@ -508,30 +508,30 @@ __global__ void __launch_bounds__(512) k_quant_rowwise(
 // reproducible bit for bit; silu(g) = g / (1 + e^-g) with an IEEE division.  The kernel uses the
 // two-element form exp_cw2 (packed fp32x2 operations round each lane as the scalar ones do).
 // ---------------------------------------------------------------------------------------------
-// e^x for two elements at once (packed fp32x2 operations round each lane as a scalar IEEE
-// operation would).  Branch-free: the polynomial runs on x clamped into range, then the results
+// e^x for two elements at once (packed fp32x2 operations with explicit rounding: each lane
+// rounds as a scalar IEEE operation would, and no multiply and add are fused).  Branch-free: the polynomial runs on x clamped into range, then the results
 // out of range (inf above ln(FLT_MAX), 0 below half the least subnormal) are selected; the
 // scaling by 2^k always takes two exact steps 2^k1 * 2^(k - k1) with k1 = clamp(k, -126, 127).
 __device__ __forceinline__ float2 exp_cw2(float2 x) {
   const float2 xc = make_float2(fminf(fmaxf(x.x, -104.0f), 0x1.62e430p+6f),
                                 fminf(fmaxf(x.y, -104.0f), 0x1.62e430p+6f));
-  const float2 t = __fmul2_rn(xc, make_float2(0x1.715476p+0f, 0x1.715476p+0f));
+  const float2 t = f2_mul_rn(xc, make_float2(0x1.715476p+0f, 0x1.715476p+0f));
   const float2 kf = make_float2(rintf(t.x), rintf(t.y));
   const float2 nk = make_float2(-kf.x, -kf.y);
-  float2 r = __fadd2_rn(xc, __fmul2_rn(nk, make_float2(0x1.62e400p-1f, 0x1.62e400p-1f)));
-  r = __fadd2_rn(r, __fmul2_rn(nk, make_float2(0x1.7f7d1cp-20f, 0x1.7f7d1cp-20f)));
+  float2 r = f2_add_rn(xc, f2_mul_rn(nk, make_float2(0x1.62e400p-1f, 0x1.62e400p-1f)));
+  r = f2_add_rn(r, f2_mul_rn(nk, make_float2(0x1.7f7d1cp-20f, 0x1.7f7d1cp-20f)));
   float2 p = make_float2(0x1.a01a02p-13f, 0x1.a01a02p-13f);
-  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0x1.6c16c2p-10f, 0x1.6c16c2p-10f));
-  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0x1.111112p-7f, 0x1.111112p-7f));
-  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0x1.555556p-5f, 0x1.555556p-5f));
-  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0x1.555556p-3f, 0x1.555556p-3f));
-  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0.5f, 0.5f));
-  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(1.0f, 1.0f));
-  p = __fadd2_rn(__fmul2_rn(p, r), make_float2(1.0f, 1.0f));
+  p = f2_add_rn(f2_mul_rn(p, r), make_float2(0x1.6c16c2p-10f, 0x1.6c16c2p-10f));
+  p = f2_add_rn(f2_mul_rn(p, r), make_float2(0x1.111112p-7f, 0x1.111112p-7f));
+  p = f2_add_rn(f2_mul_rn(p, r), make_float2(0x1.555556p-5f, 0x1.555556p-5f));
+  p = f2_add_rn(f2_mul_rn(p, r), make_float2(0x1.555556p-3f, 0x1.555556p-3f));
+  p = f2_add_rn(f2_mul_rn(p, r), make_float2(0.5f, 0.5f));
+  p = f2_add_rn(f2_mul_rn(p, r), make_float2(1.0f, 1.0f));
+  p = f2_add_rn(f2_mul_rn(p, r), make_float2(1.0f, 1.0f));
   const int ka = static_cast<int>(kf.x), kb = static_cast<int>(kf.y);
   const int ka1 = min(max(ka, -126), 127), kb1 = min(max(kb, -126), 127);
-  p = __fmul2_rn(p, make_float2(__int_as_float((ka1 + 127) << 23), __int_as_float((kb1 + 127) << 23)));
-  p = __fmul2_rn(p, make_float2(__int_as_float((ka - ka1 + 127) << 23),
+  p = f2_mul_rn(p, make_float2(__int_as_float((ka1 + 127) << 23), __int_as_float((kb1 + 127) << 23)));
+  p = f2_mul_rn(p, make_float2(__int_as_float((ka - ka1 + 127) << 23),
                                 __int_as_float((kb - kb1 + 127) << 23)));
   const float inf = __int_as_float(0x7f800000);
   p.x = x.x > 0x1.62e430p+6f ? inf : (x.x < -104.0f ? 0.0f : p.x);
@@ -618,6 +618,159 @@ __global__ void __launch_bounds__(512) k_silu_mul_quant(
         if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
       }
       if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Inverse RoPE + 1x128 quant: the front end of the attention output projection (wo_a).  o is
+// [T][H][D] bf16 with token stride ldo; the last R dims of each head are rotated by -theta_i in
+// pairs (a, b) = (2i, 2i + 1) (INTERLEAVED) or (i, i + R/2), with c = cos[p][i], s = sin[p][i]:
+//   y_a = bf16( fp32(x_a c) + fp32(x_b s) ),   y_b = bf16( fp32(x_b c) - fp32(x_a s) ),
+// every product and sum one IEEE fp32 rounding; the first D - R dims pass through.  The result is
+// quantized in 1x128 groups along the token's H*D row.  The host guarantees D % 8 == 0 and
+// R % 8 == 0 (R % 16 == 0 for half-split pairs), so every 16-byte chunk lies inside one head and
+// is all rotary or all pass-through, and the cache entries a chunk needs are 16-byte aligned.
+// ---------------------------------------------------------------------------------------------
+constexpr int kErrRange = 9;  // FP8Q_ERR_RANGE: a position outside [0, max_pos)
+
+__device__ __forceinline__ float4 ldg_f4(const float *p) {
+  return __ldg(reinterpret_cast<const float4 *>(p));
+}
+
+// Products and sums here use the scalar IEEE intrinsics, which are never merged into a fused
+// multiply-add: the rotation must round x_a c and x_b s separately, and a pair of packed
+// multiply and add intrinsics was measured to be contracted (a tie rounded the other way).
+
+// Four interleaved pairs (x_2i, x_2i+1), i = i0 .. i0 + 3, with their cos / sin entries.
+__device__ __forceinline__ uint4 inv_rope8_pairs(const uint4 x, const float4 c, const float4 s) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  const float cc[4] = {c.x, c.y, c.z, c.w}, ss[4] = {s.x, s.y, s.z, s.w};
+  uint32_t y[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float xa = bf16_lo(w[j]), xb = bf16_hi(w[j]);
+    const float ya = __fadd_rn(__fmul_rn(xa, cc[j]), __fmul_rn(xb, ss[j]));
+    const float yb = __fsub_rn(__fmul_rn(xb, cc[j]), __fmul_rn(xa, ss[j]));
+    y[j] = pack_bf16x2(ya, yb);
+  }
+  return make_uint4(y[0], y[1], y[2], y[3]);
+}
+
+// Eight elements of one half of the rotary part (x) with their partners in the other half (z):
+// y = fp32(x c) + fp32(z s) for the first half, fp32(x c) - fp32(z s) for the second.
+__device__ __forceinline__ uint4 inv_rope8_halves(const uint4 x, const uint4 z, bool second,
+                                                  const float *cs, const float *sn) {
+  const float4 c0 = ldg_f4(cs), c1 = ldg_f4(cs + 4), s0 = ldg_f4(sn), s1 = ldg_f4(sn + 4);
+  const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  const uint32_t wx[4] = {x.x, x.y, x.z, x.w}, wz[4] = {z.x, z.y, z.z, z.w};
+  uint32_t y[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float v[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float xv = h ? bf16_hi(wx[j]) : bf16_lo(wx[j]);
+      const float zv = h ? bf16_hi(wz[j]) : bf16_lo(wz[j]);
+      const float pc = __fmul_rn(xv, cc[2 * j + h]), ps = __fmul_rn(zv, ss[2 * j + h]);
+      v[h] = second ? __fsub_rn(pc, ps) : __fadd_rn(pc, ps);
+    }
+    y[j] = pack_bf16x2(v[0], v[1]);
+  }
+  return make_uint4(y[0], y[1], y[2], y[3]);
+}
+
+// One warp per token at a time; 8 lanes per 128-block (4 blocks per warp step), lane `sub` of a
+// block owns the 16-byte chunks sub + 8 c, c = 0, 1; the next step's chunks are loaded before
+// the current step is processed.  A token whose position is outside [0, max_pos) is not written
+// and records kErrRange in the device error word.
+template <int FMT, bool INTERLEAVED>
+__global__ void __launch_bounds__(512) k_inverse_rope_quant(
+    const uint16_t *__restrict__ o, int64_t ldo, const int64_t *__restrict__ pos,
+    const float *__restrict__ cosc, const float *__restrict__ sinc, int64_t max_pos, int64_t T,
+    int D, int R, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ sa,
+    int64_t lds) {
+  constexpr int LPB = 8, CPL = 2, BPS = 4;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wpc = blockDim.x >> 5;
+  const int KB = K >> 7, half = R >> 1, pass = D - R;
+  ScaleTab *tab = reinterpret_cast<ScaleTab *>(smem);
+  const int grp = lane / LPB, sub = lane % LPB;
+  if (FMT == kScaleF32) build_scale_tab(tab, threadIdx.x, blockDim.x);
+  __syncthreads();
+
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
+  for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < T; m += stride) {
+    int64_t p = 0;
+    if (R > 0) {
+      p = __ldg(pos + m);
+      if (p < 0 || p >= max_pos) {
+        if (lane == 0) record_error(kErrRange);
+        continue;
+      }
+    }
+    const float *cs = cosc + p * half, *sn = sinc + p * half;
+    const uint16_t *xr = o + m * ldo;
+    int bl = grp < KB ? grp : 0;  // the block whose chunks xn holds
+    uint4 xn[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) xn[c] = ld_stream_v4(xr + bl * 128 + (sub + LPB * c) * 8);
+    for (int b0 = 0; b0 < KB; b0 += BPS) {
+      const int b = b0 + grp;
+      const bool active = b < KB;
+      uint4 v[CPL];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        const int k0 = bl * 128 + (sub + LPB * c) * 8;
+        const int d0 = k0 % D;
+        v[c] = xn[c];
+        if (d0 >= pass) {
+          const int j0 = d0 - pass;
+          if (INTERLEAVED) {
+            v[c] = inv_rope8_pairs(xn[c], ldg_f4(cs + j0 / 2), ldg_f4(sn + j0 / 2));
+          } else {
+            const bool second = j0 >= half;
+            const int i0 = second ? j0 - half : j0;
+            const uint4 z = ld_stream_v4(xr + (second ? k0 - half : k0 + half));
+            v[c] = inv_rope8_halves(xn[c], z, second, cs + i0, sn + i0);
+          }
+        }
+      }
+      if (b0 + BPS < KB) {
+        bl = b0 + BPS + grp < KB ? b0 + BPS + grp : b0 + BPS;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) xn[c] = ld_stream_v4(xr + bl * 128 + (sub + LPB * c) * 8);
+      }
+      uint32_t m2 = 0u;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) m2 = absmax_uint4(m2, v[c]);
+#pragma unroll
+      for (int s = LPB / 2; s > 0; s >>= 1)
+        m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, s));
+      const float amax = absmax_finish(m2);
+      uint8_t *qb = q + m * ldq + b * 128;
+      float scale;
+      if (FMT == kScaleF32) {
+        const QParams qp = qparams_tab(amax, tab);
+        scale = qp.s;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          const uint2 codes = quant8_f32(v[c], qp);
+          if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
+        }
+      } else {
+        const int e = e8m0_exponent(amax);
+        scale = pow2_f32(e);
+        const float inv = pow2_f32(-e);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          const uint2 codes = quant8_pow2(v[c], make_float2(inv, inv));
+          if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
+        }
+      }
+      if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = scale;
     }
   }
 }

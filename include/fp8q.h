@@ -67,7 +67,8 @@ typedef enum {
   FP8Q_ERR_LAUNCH = 5,  /* a CUDA runtime call or kernel launch failed */
   FP8Q_ERR_TIMEOUT = 6, /* (device error word) a kernel gave up on a bounded wait */
   FP8Q_ERR_ARG = 7,     /* an enum argument is out of range */
-  FP8Q_ERR_TOO_LARGE = 8 /* the problem does not fit the library's static split-K scratch */
+  FP8Q_ERR_TOO_LARGE = 8, /* the problem does not fit the library's static split-K scratch */
+  FP8Q_ERR_RANGE = 9      /* (device error word) a RoPE position was outside [0, max_pos) */
 } fp8q_status;
 
 typedef enum {
@@ -166,6 +167,27 @@ int fp8q_gemm_w8a8_block_splitk_noalloc(const void *aq, int64_t lda, const float
                                         void *out_bf16, int64_t ldo, int splits,
                                         cudaStream_t stream);
 
+/* Block-diagonal W8A8 GEMM over G head groups: the batched projection that follows
+ * fp8q_inverse_rope_quant.  Group g multiplies its own K-slice of each token's row by its own
+ * weight and writes its own column range:
+ *   out[m][g N_g + n] = sum over kb of fp32(sa[(g KB_g + kb) lds + m] * sw[g][n/128][kb])
+ *                       * (fp32 dot product of the 128 codes of A[m][g K_g + 128 kb ...] and
+ *                          W[g][n][128 kb ...]),  KB_g = K_g / 128
+ *   aq      [M][lda] uint8 codes, lda >= G K_g (the groups' K-slices side by side)
+ *   sa      fp32 activation scales, K-block-major over all G K_g columns
+ *   wq      [G][N_g][ldw] uint8 codes (group stride N_g ldw), i.e. G N_g rows of K_g codes
+ *   sw      [G][N_g/128][K_g/128] fp32 or E8M0
+ *   out     [M][ldo] bf16, ldo >= G N_g: the [M, G, N_g] result flattened over (G, N_g)
+ * N_g % 256 == 0 (a 128 x 256 output tile never straddles two groups), K_g % 128 == 0; the other
+ * rules, the arithmetic and the tolerance are those of fp8q_gemm_w8a8_block.  Source: vLLM PR
+ * 54894 analysis, sections 2-3 (weights viewed as [groups, out_per_group, in_features] with
+ * scales [groups, out/128, in/128]; a batched FP8 GEMM over the groups, flattened over
+ * (groups, out) afterwards). */
+int fp8q_gemm_w8a8_block_diag(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                              const void *wq, int64_t ldw, const void *sw, int sw_fmt,
+                              int64_t G, int64_t M, int64_t N_g, int64_t K_g, void *out_bf16,
+                              int64_t ldo, cudaStream_t stream);
+
 /* Grouped W8A8 GEMM for MoE experts (a6): for each expert e the rows
  * [group_offsets[e], group_offsets[e+1]) of aq/sa/out are multiplied by expert e's weight.
  *   wq             [E][N][ldw] uint8 codes (expert stride N * ldw)
@@ -192,6 +214,33 @@ int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, i
  * activated gate/up output, quantized 1x128 like every activation here). */
 int fp8q_silu_mul_quant(const void *h_bf16, int64_t R, int64_t I, int64_t ldh, void *q_e4m3,
                         int64_t ldq, float *sa, int64_t lds, cudaStream_t stream);
+
+/* Inverse RoPE + 1x128 quant: the front end of the attention output projection (wo_a), whose
+ * output feeds the per-head-group GEMM fp8q_gemm_w8a8_block_diag.
+ *   o_bf16     [T][H][D] bf16, heads contiguous, token stride ldo (elements), read
+ *   positions  [T] int64, DEVICE memory: each token's position, read when rope_dim > 0
+ *   cos_cache, sin_cache
+ *              [max_pos][rope_dim / 2] fp32, DEVICE memory (16-byte aligned), read
+ *   q_e4m3     [T][ldq] uint8 codes of y (below) along the flattened H*D row, written
+ *   sa         fp32 scales sa[kb * lds + t], one per 128-group of y, written for t < T only
+ * y: the last rope_dim dims of each head are rotated by -theta_i in pairs (a, b) = (2i, 2i + 1)
+ * (interleaved = 1) or (i, i + rope_dim / 2) (interleaved = 0), with c = cos[p][i] and
+ * s = sin[p][i]: y_a = bf16(fp32(x_a c) + fp32(x_b s)), y_b = bf16(fp32(x_b c) - fp32(x_a s)),
+ * each product and sum one IEEE fp32 rounding; the first D - rope_dim dims pass through.
+ * scale_fmt FP8Q_SCALE_F32: s = fp32(amax / 448) (1 for an all-zero group); FP8Q_SCALE_E8M0:
+ * s = the smallest power of two >= fp32(amax / 448) (the MX scale of the GEMM that follows),
+ * stored as its fp32 value.  Codes are RNE-saturating E4M3 of y / s.
+ * D % 8 == 0, rope_dim % 8 == 0 (% 16 when interleaved == 0), rope_dim <= D, H*D % 128 == 0,
+ * H*D <= 2^24.  A token whose position is outside [0, max_pos) is not written and records
+ * FP8Q_ERR_RANGE in the device error word (fp8q_check_device_error).  Bit-exact against the
+ * CPU oracle.  Source: vLLM PR 54894 analysis, section 3 (inverse_rope_group_quant(o [T, heads,
+ * head_dim], positions, cos cache, sin cache, num_groups, quant_group_size=128) fuses the
+ * inverse RoPE with the FP8 quantization so that the rotated bf16 values never reach memory). */
+int fp8q_inverse_rope_quant(const void *o_bf16, int64_t ldo, const int64_t *positions,
+                            const float *cos_cache, const float *sin_cache, int64_t max_pos,
+                            int64_t T, int64_t H, int64_t D, int64_t rope_dim, int interleaved,
+                            int scale_fmt, void *q_e4m3, int64_t ldq, float *sa, int64_t lds,
+                            cudaStream_t stream);
 
 /* Per-token (full-row) quantization, optionally fused with RMSNorm: one fp32 scale per row of K
  * (the "group size 0 = per token" mode).  Applied to a weight W [N, K] it gives the

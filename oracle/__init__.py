@@ -236,6 +236,27 @@ def grouped_gemm_w8a8_block(aq, sa, wq, sw, group_offsets, sw_fmt: int = SCALE_F
     return ref, absref
 
 
+def gemm_w8a8_block_diag(aq, sa, wq, sw, sw_fmt: int = SCALE_F32, rows=None):
+    """Block-diagonal reference [DSv4-WOA sections 2-3: a batched GEMM over head groups]:
+    wq [G, N_g, K_g], sw [G, N_g/128, K_g/128]; group g multiplies the K-slice
+    [g K_g, (g+1) K_g) of aq (scales: sa's K-blocks [g K_g/128, ...)) by wq[g] and fills the
+    output columns [g N_g, (g+1) N_g).  Each group is one call of the plain block GEMM."""
+    aq = _c(aq, np.uint8)
+    sa = _c(sa, np.float32)
+    G, N_g, K_g = wq.shape
+    KB = K_g // 128
+    M = aq.shape[0]
+    nrows = M if rows is None else len(rows)
+    ref = np.empty((nrows, G * N_g), dtype=np.float64)
+    absref = np.empty((nrows, G * N_g), dtype=np.float64)
+    for g in range(G):
+        r, a = gemm_w8a8_block(aq[:, g * K_g:(g + 1) * K_g], sa[g * KB:(g + 1) * KB], wq[g],
+                               sw[g], sw_fmt, rows)
+        ref[:, g * N_g:(g + 1) * N_g] = r
+        absref[:, g * N_g:(g + 1) * N_g] = a
+    return ref, absref
+
+
 def exp_f32(x: float) -> float:
     """e^x in fp32 by the method of reading R8 (Cody-Waite reduction, degree-7 Taylor)."""
     return float(lib().oracle_exp_f32(float(x)))

@@ -33,7 +33,7 @@ def test_exports_match_header(L):
 
 
 def test_status_strings(L):
-    for s in range(9):
+    for s in range(10):
         assert len(_lib.status_string(s)) >= 2
     assert _lib.status_string(99) == "unknown status"
 
@@ -165,3 +165,53 @@ def test_silu_mul_quant_host_checks(L):
     assert f(FAKE, 4, 128, 260, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_ALIGN   # ldh % 8
     assert f(None, 4, 128, 256, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_NULL
     assert f(None, 0, 128, 256, None, 128, None, 4, None) == _lib.FP8Q_OK
+
+
+def test_inverse_rope_quant_host_checks(L):
+    f = L.fp8q_inverse_rope_quant
+    ok = dict(o=FAKE, ldo=1024, pos=FAKE, cos=FAKE, sin=FAKE, max_pos=64, T=8, H=2, D=512, R=64,
+              il=1, fmt=0, q=FAKE, ldq=1024, sa=FAKE, lds=8)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["o"], a["ldo"], a["pos"], a["cos"], a["sin"], a["max_pos"], a["T"], a["H"],
+                 a["D"], a["R"], a["il"], a["fmt"], a["q"], a["ldq"], a["sa"], a["lds"], None)
+    assert call(fmt=2) == _lib.FP8Q_ERR_ARG
+    assert call(il=2) == _lib.FP8Q_ERR_ARG
+    assert call(D=100, ldo=200, ldq=208) == _lib.FP8Q_ERR_SHAPE          # D % 8
+    assert call(H=1, D=192, ldo=192, ldq=192) == _lib.FP8Q_ERR_SHAPE      # H*D % 128
+    assert call(R=60) == _lib.FP8Q_ERR_SHAPE                              # rope_dim % 8
+    assert call(R=520) == _lib.FP8Q_ERR_SHAPE                             # rope_dim > D
+    assert call(R=40, il=0) == _lib.FP8Q_ERR_SHAPE                        # halves: % 16
+    assert call(ldo=1000) == _lib.FP8Q_ERR_SHAPE
+    assert call(lds=4) == _lib.FP8Q_ERR_SHAPE
+    assert call(max_pos=0) == _lib.FP8Q_ERR_SHAPE
+    assert call(pos=None) == _lib.FP8Q_ERR_NULL
+    assert call(cos=FAKE + 4) == _lib.FP8Q_ERR_ALIGN
+    assert call(pos=FAKE + 4) == _lib.FP8Q_ERR_ALIGN
+    assert call(ldo=1028) == _lib.FP8Q_ERR_ALIGN
+    assert call(T=0, o=None, q=None, sa=None, pos=None) == _lib.FP8Q_OK
+    import torch
+    if not torch.cuda.is_available():   # valid arguments reach the device check (never launched)
+        assert call() == _lib.FP8Q_ERR_ARCH
+        assert call(R=0, pos=None, cos=None, sin=None, max_pos=0) == _lib.FP8Q_ERR_ARCH
+
+
+def test_block_diag_gemm_host_checks(L):
+    g = L.fp8q_gemm_w8a8_block_diag
+    ok = dict(aq=FAKE, lda=1024, sa=FAKE, lds=64, wq=FAKE, ldw=512, sw=FAKE, fmt=0, G=2, M=64,
+              N_g=256, K_g=512, out=FAKE, ldo=512)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["aq"], a["lda"], a["sa"], a["lds"], a["wq"], a["ldw"], a["sw"], a["fmt"],
+                 a["G"], a["M"], a["N_g"], a["K_g"], a["out"], a["ldo"], None)
+    assert call(N_g=128, ldo=256) == _lib.FP8Q_ERR_SHAPE                  # N_g % 256
+    assert call(G=0) == _lib.FP8Q_ERR_SHAPE
+    assert call(lda=768) == _lib.FP8Q_ERR_SHAPE                           # lda < G K_g
+    assert call(ldo=256) == _lib.FP8Q_ERR_SHAPE                           # ldo < G N_g
+    assert call(K_g=200, ldw=208) == _lib.FP8Q_ERR_SHAPE
+    assert call(fmt=3) == _lib.FP8Q_ERR_ARG
+    assert call(sw=None) == _lib.FP8Q_ERR_NULL
+    assert call(lda=1032) == _lib.FP8Q_ERR_ALIGN
+    assert call(M=0, aq=None, sa=None, out=None) == _lib.FP8Q_OK

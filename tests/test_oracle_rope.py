@@ -138,3 +138,31 @@ def test_no_rotary_dims_reduces_to_token_quant():
     q, sa = oracle.inverse_rope_quant(o, np.zeros(5, np.int64), cos, sin, 0)
     q2, sa2 = oracle.quant_token_1x128(o.reshape(5, 512))
     assert np.array_equal(q, q2) and np.array_equal(sa, sa2)
+
+
+@pytest.mark.parametrize("fmt", [oracle.SCALE_F32, oracle.SCALE_E8M0])
+def test_block_diag_gemm_equals_dense_gemm_with_block_diagonal_weight(fmt):
+    """The per-group GEMM is the plain GEMM with the groups' weights on the block diagonal of
+    one [G N_g, G K_g] matrix (zero codes elsewhere add exact zeros)."""
+    G, M, N_g, K_g = 3, 20, 256, 256
+    a = inputs.bf16_bits_to_f32(inputs.randn_bf16((M, G * K_g), 40.0, 41, 0))
+    aq = oracle.e4m3_encode(a).reshape(M, G * K_g)
+    sa = np.abs(inputs.bf16_bits_to_f32(inputs.randn_bf16((G * K_g // 128, M), 0.01, 41, 1)))
+    sa += np.float32(1e-4)
+    w = inputs.randn_bf16((G, N_g, K_g), 0.02, 41, 2)
+    wq = np.empty((G, N_g, K_g), np.uint8)
+    sw = []
+    for g in range(G):
+        wq[g], s = oracle.quant_weight_block(w[g], fmt)
+        sw.append(s)
+    sw = np.stack(sw)
+    ref, absref = oracle.gemm_w8a8_block_diag(aq, sa, wq, sw, fmt)
+    wfull = np.zeros((G * N_g, G * K_g), np.uint8)
+    swfull = np.full((G * N_g // 128, G * K_g // 128), 1.0 if fmt == oracle.SCALE_F32 else 127,
+                     np.float32 if fmt == oracle.SCALE_F32 else np.uint8)
+    for g in range(G):
+        wfull[g * N_g:(g + 1) * N_g, g * K_g:(g + 1) * K_g] = wq[g]
+        swfull[g * N_g // 128:(g + 1) * N_g // 128, g * K_g // 128:(g + 1) * K_g // 128] = sw[g]
+    ref2, absref2 = oracle.gemm_w8a8_block(aq, sa, wfull, swfull, fmt)
+    assert np.array_equal(ref, ref2) and np.array_equal(absref, absref2)
+    assert np.abs(ref).max() > 0
