@@ -420,7 +420,47 @@ def measure_rows(fq, device, steps, warmup, pk):
     rows["wo_a_chain"] = {"ms": ms, "TFLOP/s": fl / ms / 1e9,
                           "workload": f"inverse RoPE quant -> {G}-group GEMM, {T} tokens",
                           "launches": 2}
+    # the same GEMM with the scales applied by the tensor core (both scale sets powers of two)
+    ms, _ = timed_loop(lambda: fq.gemm_w8a8_mx(q_d, sa_d, wq, sw, out=out_d), steps, warmup,
+                       flush)
+    rows["gemm_mx_wo_a"] = {"ms": ms, "TFLOP/s": fl / ms / 1e9,
+                            "frac_fp8_sustained": fl / ms / 1e9 / (2.0 * pk["bf16_sustained"]),
+                            "workload": f"{G} head groups: [{T}, {K_g}] x [{N_g}, {K_g}] each, "
+                                        "hardware block scaling"}
+
+    def wo_a_chain_mx():
+        fq.inverse_rope_quant(o_d, pos_d, cos_d, sin_d, 64, True, fq.FP8Q_SCALE_E8M0,
+                              out_q=q_d, out_sa=sa_d)
+        fq.gemm_w8a8_mx(q_d, sa_d, wq, sw, out=out_d)
+    ms, _ = timed_loop(wo_a_chain_mx, steps, warmup, flush)
+    rows["wo_a_chain_mx"] = {"ms": ms, "TFLOP/s": fl / ms / 1e9,
+                             "workload": f"inverse RoPE quant -> {G}-group MX GEMM, {T} tokens",
+                             "launches": 2}
     del o_d, pos_d, cos_d, sin_d, W, wq, sw, q_d, sa_d, out_d
+    torch.cuda.empty_cache()
+
+    # the prefill GEMM with power-of-two scales on both operands, hardware block scaling
+    pf = inputs.prefill_linear()
+    X = dev_bf16(pf["X"], device)
+    W = dev_bf16(pf["W"], device)
+    Mp, Kp = X.shape
+    Np = W.shape[0]
+    aq, sa = fq.inverse_rope_quant(X.view(Mp, 1, Kp), None, None, None, 0, True,
+                                   fq.FP8Q_SCALE_E8M0)
+    wq, sw = fq.quant_weight_block(W, "e8m0")
+    out = torch.empty((Mp, Np), dtype=torch.bfloat16, device=device)
+    fl = 2.0 * Mp * Np * Kp
+    ms, _ = timed_loop(lambda: fq.gemm_w8a8_mx(aq, sa, wq, sw, out=out), steps, warmup)
+    rows["gemm_mx_prefill"] = {"ms": ms, "TFLOP/s": fl / ms / 1e9,
+                               "frac_fp8_sustained": fl / ms / 1e9 / (2.0 * pk["bf16_sustained"]),
+                               "workload": f"M={Mp} N={Np} K={Kp}, E8M0 scales, hardware block "
+                                           "scaling"}
+    sw32 = torch.ldexp(torch.ones_like(sw, dtype=torch.float32), sw.to(torch.int32) - 127)
+    ms, _ = timed_loop(lambda: fq.gemm_w8a8_block(aq, sa, wq, sw32, out=out), steps, warmup)
+    rows["gemm_sw_promotion_prefill_pow2"] = {
+        "ms": ms, "TFLOP/s": fl / ms / 1e9,
+        "workload": f"M={Mp} N={Np} K={Kp}, the same power-of-two scales, software promotion"}
+    del X, W, aq, sa, wq, sw, sw32, out
     torch.cuda.empty_cache()
     return rows
 
@@ -692,6 +732,20 @@ def run_ncu_case(name):
         out = torch.empty((R, 1536), dtype=torch.bfloat16, device=dev)
         fn = lambda: fq.grouped_gemm_w8a8_block(aq, sa, wq.view(128, 1536, 2048),
                                                 sw.view(128, 12, 16), offd, out=out)
+    elif name in ("inverse_rope_wo_a", "inverse_rope_wo_a_f32"):   # o [8192, 32, 512]: 268 MB in
+        o = randn((8192, 32, 512), 1.0)
+        pos = torch.randint(0, 16384, (8192,), generator=g, device=dev)
+        cs = torch.rand((16384, 32), generator=g, device=dev)
+        sn = torch.rand((16384, 32), generator=g, device=dev)
+        fmt = "f32" if name.endswith("f32") else "e8m0"
+        fn = lambda: fq.inverse_rope_quant(o, pos, cs, sn, 64, True, fmt)
+    elif name == "gemm_diag_wo_a":       # 4 head groups: [8192, 4096] x [1024, 4096] each
+        o = randn((8192, 32, 512), 1.0)
+        aq, sa = fq.inverse_rope_quant(o, None, None, None, 0)
+        wq, sw = fq.quant_weight_block(randn((4096, 4096), 0.02), "e8m0")
+        out = torch.empty((8192, 4096), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm_w8a8_block_diag(aq, sa, wq.view(4, 1024, 4096),
+                                             sw.view(4, 8, 32), out=out)
     else:
         raise SystemExit(f"unknown --ncu-case {name}")
     torch.cuda.synchronize()

@@ -16,7 +16,7 @@ import torch
 
 from . import _lib
 from ._lib import (FP8Q_ERR_ALIGN, FP8Q_ERR_ARCH, FP8Q_ERR_ARG, FP8Q_ERR_LAUNCH, FP8Q_ERR_NULL,
-                   FP8Q_ERR_RANGE, FP8Q_ERR_SHAPE, FP8Q_ERR_TIMEOUT, FP8Q_OK, FP8Q_SCALE_E8M0, FP8Q_SCALE_F32,
+                   FP8Q_ERR_NOT_POW2, FP8Q_ERR_RANGE, FP8Q_ERR_SHAPE, FP8Q_ERR_TIMEOUT, FP8Q_OK, FP8Q_SCALE_E8M0, FP8Q_SCALE_F32,
                    Fp8qError)
 
 import ctypes
@@ -24,7 +24,7 @@ import ctypes
 __all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
            "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant", "inverse_rope_quant",
-           "gemm_w8a8_block_diag",
+           "gemm_w8a8_block_diag", "gemm_w8a8_mx",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -221,6 +221,29 @@ def gemm_w8a8_block_diag(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, s
                                               _ptr(wq), wq.stride(1), _ptr(sw), f, G, M, N_g,
                                               K_g, _ptr(o), _ld(o), _stream(stream))
     _lib.check(st, "fp8q_gemm_w8a8_block_diag")
+    return o
+
+
+def gemm_w8a8_mx(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,
+                 out=None, stream=None):
+    """Hardware block-scaled GEMM for power-of-two scales: codes aq [M, G*K_g] with fp32
+    power-of-two scales sa [G*K_g/128, lds], weights wq [N, K] (G = 1) or [G, N_g, K_g] with E8M0
+    bytes sw [N/128, K/128] or [G, N_g/128, K_g/128] -> bf16 [M, G*N_g]."""
+    if sw.dtype != torch.uint8:
+        raise ValueError("sw must hold E8M0 bytes (torch.uint8)")
+    if wq.dim() == 2:
+        G, (N_g, K_g) = 1, wq.shape
+        ldw = _ld(wq)
+    else:
+        G, N_g, K_g = wq.shape
+        if wq.stride(0) != N_g * wq.stride(1) or wq.stride(2) != 1:
+            raise ValueError("wq must be [G, N_g, ldw] with group stride N_g * ldw")
+        ldw = wq.stride(1)
+    M = aq.shape[0]
+    o = torch.empty((M, G * N_g), dtype=torch.bfloat16, device=aq.device) if out is None else out
+    st = _lib.lib().fp8q_gemm_w8a8_mx(_ptr(aq), _ld(aq), _ptr(sa), sa.stride(0), _ptr(wq), ldw,
+                                      _ptr(sw), G, M, N_g, K_g, _ptr(o), _ld(o), _stream(stream))
+    _lib.check(st, "fp8q_gemm_w8a8_mx")
     return o
 
 

@@ -18,6 +18,7 @@ FP8Q_ERR_TIMEOUT = 6
 FP8Q_ERR_ARG = 7
 FP8Q_ERR_TOO_LARGE = 8
 FP8Q_ERR_RANGE = 9
+FP8Q_ERR_NOT_POW2 = 10
 
 FP8Q_SCALE_F32 = 0
 FP8Q_SCALE_E8M0 = 1
@@ -44,6 +45,8 @@ SIGNATURES = {
                                      _P, _I64, _P, _I64, _P]),
     "fp8q_gemm_w8a8_block_diag": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64, _I64,
                                        _I64, _P, _I64, _P]),
+    "fp8q_gemm_w8a8_mx": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _P,
+                               _I64, _P]),
     "fp8q_quant_rowwise": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "fp8q_gemm_w8a8_rowwise": (_I, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I64, _P]),
     "fp8q_check_device_error": (_I, [_P]),

@@ -72,6 +72,8 @@ int device_state(DeviceState **out) {
             cudaSuccess ||
         cudaFuncSetAttribute(fp8q::k_gemm_w8a8_rowwise,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fp8q::kGemmSmemDense) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_gemm_w8a8_mx, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fp8q::kGemmSmemDense) != cudaSuccess)
       return FP8Q_ERR_LAUNCH;
     st.attrs_set = true;
@@ -232,6 +234,7 @@ const char *fp8q_status_string(int status) {
     case FP8Q_ERR_LAUNCH: return "CUDA runtime or launch failure";
     case FP8Q_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (outputs incomplete)";
     case FP8Q_ERR_ARG: return "enum argument out of range";
+    case FP8Q_ERR_NOT_POW2: return "a scale given to the hardware block-scaled GEMM is not a power of two (outputs invalid)";
     case FP8Q_ERR_RANGE: return "an index input (a RoPE position) was outside its table; that row was not written";
     case FP8Q_ERR_TOO_LARGE: return "problem needs more split-K scratch than the library's static 24 MiB buffer (use fp8q_gemm_w8a8_block_splitk with a workspace, or fewer splits)";
     default: return "unknown status";
@@ -600,6 +603,48 @@ int fp8q_gemm_w8a8_rowwise(const void *aq, int64_t lda, const float *sa, const v
   const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
   fp8q::k_gemm_w8a8_rowwise<<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemDense, stream>>>(tm_a,
                                                                                        tm_b, a);
+  return launch_status();
+}
+
+int fp8q_gemm_w8a8_mx(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                      const void *wq, int64_t ldw, const void *sw_e8m0, int64_t G, int64_t M,
+                      int64_t N_g, int64_t K_g, void *out_bf16, int64_t ldo,
+                      cudaStream_t stream) {
+  if (G <= 0 || G > (1 << 16) || N_g <= 0 || N_g % 128 || K_g <= 0 || K_g % 128)
+    return FP8Q_ERR_SHAPE;
+  if (G > 1 && N_g % fp8q::kBN) return FP8Q_ERR_SHAPE;
+  if (N_g > (1 << 30) / G || K_g > (1 << 30) / G || M < 0 || M > INT32_MAX - 256)
+    return FP8Q_ERR_SHAPE;
+  const int64_t N = G * N_g;
+  if (lda < G * K_g || ldw < K_g || ldo < N || lds < M) return FP8Q_ERR_SHAPE;
+  if (M == 0) return FP8Q_OK;
+  if (!aq || !sa || !wq || !sw_e8m0 || !out_bf16) return FP8Q_ERR_NULL;
+  if (!aligned16(aq) || !aligned16(wq) || !aligned16(out_bf16) ||
+      (reinterpret_cast<uintptr_t>(sa) & 3u) || lda % 16 || ldw % 16 || ldo % 8)
+    return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  if ((rc = get_encoder()) != FP8Q_OK) return rc;
+  CUtensorMap tm_a, tm_b;
+  if ((rc = make_u8_map(&tm_a, aq, M, G * K_g, lda, fp8q::kBM)) != FP8Q_OK) return rc;
+  if ((rc = make_u8_map(&tm_b, wq, N, K_g, ldw, fp8q::kBN)) != FP8Q_OK) return rc;
+  fp8q::MxArgs a;
+  a.sa = sa;
+  a.lds = lds;
+  a.sw = static_cast<const uint8_t *>(sw_e8m0);
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.K = static_cast<int>(K_g);
+  a.out = static_cast<uint16_t *>(out_bf16);
+  a.ldo = ldo;
+  a.num_n = static_cast<int>((N + fp8q::kBN - 1) / fp8q::kBN);
+  a.num_m = static_cast<int>((M + fp8q::kBM - 1) / fp8q::kBM);
+  a.n_tiles_per_group = G > 1 ? static_cast<int>(N_g / fp8q::kBN) : 0;
+  const int64_t tiles = static_cast<int64_t>(a.num_m) * a.num_n;
+  const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+  fp8q::k_gemm_w8a8_mx<<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemDense, stream>>>(tm_a, tm_b,
+                                                                                  a);
   return launch_status();
 }
 

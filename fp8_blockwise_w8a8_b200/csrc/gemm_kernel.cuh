@@ -193,20 +193,14 @@ __device__ __forceinline__ void promote8(float2 *acc, const uint32_t (&r)[16], f
 // bf16 conversion and store of 32 columns (v[j] = columns 2j, 2j + 1 of chunk c4) of this
 // thread's row, through the warp's swizzled staging buffer so that each global store
 // instruction writes 64-byte row segments.
-__device__ __forceinline__ void store_chunk32(const float2 (&v)[16], uint32_t stage_u32, int lane,
-                                              uint16_t *out_base, const Tile &tl, int q, int c4,
-                                              bool col_ok, int64_t ldo) {
+__device__ __forceinline__ void store_packed32(const uint32_t (&pk)[16], uint32_t stage_u32,
+                                               int lane, uint16_t *out_base, const Tile &tl, int q,
+                                               int c4, bool col_ok, int64_t ldo) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    uint32_t pk[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const __nv_bfloat162 v2 = __floats2bfloat162_rn(v[4 * j + u].x, v[4 * j + u].y);
-      pk[u] = *reinterpret_cast<const uint32_t *>(&v2);
-    }
     const int phys = j ^ ((lane >> 1) & 3);
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(stage_u32 + lane * 64 + phys * 16),
-                 "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                 "r"(pk[4 * j]), "r"(pk[4 * j + 1]), "r"(pk[4 * j + 2]), "r"(pk[4 * j + 3])
                  : "memory");
   }
   __syncwarp();
@@ -224,6 +218,18 @@ __device__ __forceinline__ void store_chunk32(const float2 (&v)[16], uint32_t st
       *reinterpret_cast<uint4 *>(out_base + static_cast<int64_t>(grow) * ldo + 32 * c4 + 8 * c) = w;
   }
   __syncwarp();
+}
+
+__device__ __forceinline__ void store_chunk32(const float2 (&v)[16], uint32_t stage_u32, int lane,
+                                              uint16_t *out_base, const Tile &tl, int q, int c4,
+                                              bool col_ok, int64_t ldo) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const __nv_bfloat162 v2 = __floats2bfloat162_rn(v[u].x, v[u].y);
+    pk[u] = *reinterpret_cast<const uint32_t *>(&v2);
+  }
+  store_packed32(pk, stage_u32, lane, out_base, tl, q, c4, col_ok, ldo);
 }
 
 template <bool GROUPED>
@@ -716,6 +722,309 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_swempty + 8 * tp);  // done with this tile's weight scales
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Hardware block-scaled GEMM for power-of-two (E8M0) scales:
+//   out[m, n] = bf16( sum_kb 2^ea[m, kb] * 2^ew[n / 128, kb] * P_kb[m, n] )
+// tcgen05.mma kind::mxf8f6f4.block_scale applies one UE8M0 scale per 32 K-elements of each row of
+// A and each column of B inside the tensor core; the 128-group scale of a K-block is given to all
+// four of its 32-element sub-blocks.  All of K accumulates in one 256-column TMEM buffer, so the
+// epilogue only converts: it moves the whole tile to registers, hands the buffer back to the MMA
+// and then writes bf16 while the next tile accumulates.
+// Scale factors in TMEM: SFA in 4 columns (row m at lane m % 32 of every sub-partition, column
+// m / 32), SFB in 8 (column n at lane n % 32, column n / 32).  Each 32-bit cell holds the scales
+// of four consecutive K-blocks, one per byte; the instruction's scale-factor ID picks the byte.
+// So one group of three tcgen05.cp (SFA, SFB 0-127, SFB 128-255) serves four K-blocks; two such
+// slots (TMEM columns 256 + 16 j) alternate between groups.  Roles:
+//   warp 0      TMA producer, as in k_gemm_w8a8_block
+//   warp 1      MMA issuer: at the first K-block of a group the three copies from the group's
+//               shared scale tiles, then per K-block 4 block-scaled MMAs; after the group's last
+//               MMA a commit frees the group's slot (shared tiles and TMEM columns)
+//   warp 2      scale producer: per group converts the activation scales (fp32 powers of two;
+//               anything else records FP8Q_ERR_NOT_POW2) and the tile's weight-scale bytes into
+//               the 32 x 16-byte shared tiles tcgen05.cp reads; the next group's global loads are
+//               issued as soon as the current group is written
+//   warps 4-11  epilogue
+// Block-diagonal head groups work as in k_gemm_w8a8_block (Tile::a_kb).
+// ---------------------------------------------------------------------------------------------
+struct MxArgs {
+  const float *sa;       // K-block-major fp32 powers of two, sa[kb * lds + m]
+  int64_t lds;
+  const uint8_t *sw;     // E8M0 bytes [N/128][K/128]
+  int M, N, K;           // K: per group when n_tiles_per_group > 0
+  uint16_t *out;
+  int64_t ldo;
+  int num_n, num_m;
+  int n_tiles_per_group;
+};
+
+constexpr int kErrNotPow2 = 10;  // FP8Q_ERR_NOT_POW2
+constexpr int kSfGroup = 4;                            // K-blocks per scale-factor group
+constexpr int kSfTileBytes = 32 * 16;                  // one tcgen05.cp source: 32 rows x 16 B
+constexpr int kSfSlotBytes = 3 * kSfTileBytes;         // SFA, SFB columns 0-127, SFB 128-255
+constexpr int kOffSf = kOffSa;                         // [2 slots][3][32][16] B
+static_assert(kOffSf + 2 * kSfSlotBytes <= kOffBar, "scale-factor tiles overlap barriers");
+// Block-scaled instruction descriptor: A, B E4M3 (bits 7-9, 10-12 = 0), K-major, N >> 3 in bits
+// 17-22, scale format UE8M0 (bit 23), M >> 4 in bits 24-28, K = 32 (bit 31 = 0); the scale-factor
+// IDs (bits 4-5 for B, 29-30 for A) are set per K-block by mx_idesc.
+constexpr uint32_t kIdescMx = (static_cast<uint32_t>(kBN >> 3) << 17) | (1u << 23) |
+                              (static_cast<uint32_t>(kBM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t mx_idesc(uint32_t sf_id) {
+  return kIdescMx | (sf_id << 4) | (sf_id << 29);
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte tile, rows contiguous, no swizzle: 8-row core
+// groups 128 bytes apart (stride byte offset), leading byte offset 16 (a single 16-byte column),
+// descriptor version 1 (bit 46), layout 0.
+__device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(16 >> 4) << 16) |
+         (static_cast<uint64_t>(128 >> 4) << 32) | (static_cast<uint64_t>(1) << 46);
+}
+
+// E8M0 byte of an fp32 power of two (2^-127 .. 2^127); other values record kErrNotPow2.
+__device__ __forceinline__ uint32_t e8m0_of_pow2(float v) {
+  const uint32_t b = __float_as_uint(v);
+  const uint32_t ex = (b >> 23) & 0xFFu, mant = b & 0x7FFFFFu;
+  if (b >> 31 || ex == 0xFFu || (ex != 0u && mant != 0u) || (ex == 0u && mant != 0x400000u)) {
+    record_error(kErrNotPow2);
+    return 127u;
+  }
+  return ex;  // 2^-127 (0x00400000) has exponent field 0, its E8M0 byte
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm_w8a8_mx(const __grid_constant__ CUtensorMap tm_a,
+                   const __grid_constant__ CUtensorMap tm_b, const MxArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar_full = sbase + kOffBar;              // [kStages]
+  const uint32_t bar_empty = bar_full + 8 * kStages;      // [kStages]
+  const uint32_t bar_tfull = bar_empty + 8 * kStages;
+  const uint32_t bar_tempty = bar_tfull + 16;
+  const uint32_t bar_done = bar_tempty + 16;
+  const uint32_t bar_sffull = bar_done + 8;               // [2]
+  const uint32_t bar_sfempty = bar_sffull + 16;           // [2]
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+  const int KB = args.K / kBK;
+  const int NB = args.N / 128;
+  GemmArgs ga{};
+  ga.num_m = args.num_m;
+  ga.num_n = args.num_n;
+  ga.M = args.M;
+  ga.K = args.K;
+  ga.n_tiles_per_group = args.n_tiles_per_group;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_sffull + 8 * i, 1);
+      mbar_init(bar_sfempty + 8 * i, 1);
+    }
+    mbar_init(bar_tfull, 1);
+    mbar_init(bar_tempty, 8);
+    mbar_init(bar_done, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total_tiles = args.num_m * args.num_n;
+
+  if (warp < 4) {
+    reg_dealloc<kProducerRegs>();
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_b);
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+          const Tile tl = dense_tile(ga, t);
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            if (!wait_one(bar_empty + 8 * s, ph ^ 1u, s_abort)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar_full + 8 * s, kStageBytes);
+            tma_load_2d(sbase + kOffA + s * kTileABytes, &tm_a, (tl.a_kb + kb) * kBK, tl.m0,
+                        bar_full + 8 * s);
+            tma_load_2d(sbase + kOffB + s * kTileBBytes, &tm_b, kb * kBK, tl.b_row,
+                        bar_full + 8 * s);
+          }
+        }
+        for (uint32_t s = 0; s < kStages && s < it; ++s) {
+          const uint32_t last = s + ((it - 1 - s) / kStages) * kStages;  // last fill of stage s
+          wait_drain(bar_full + 8 * s, (last / kStages) & 1u);
+        }
+      }
+      __syncwarp();
+    } else if (warp == 2) {
+      // ---------------------------------------------------------------- scale producer
+      float qa[kSfGroup][4];        // the next group's activation scales (rows lane + 32 c)
+      uint32_t qb[kSfGroup][2];     // and weight-scale bytes of the tile's two 128-column halves
+      int lt = blockIdx.x, lg = 0;  // the next group to load: tile, first K-block
+      auto load_group = [&]() {
+        if (lt >= total_tiles) return;
+        const Tile tl = dense_tile(ga, lt);
+#pragma unroll
+        for (int j = 0; j < kSfGroup; ++j) {
+          const bool in = lg + j < KB;
+          const float *sa_kb = args.sa + static_cast<int64_t>(tl.a_kb + lg + j) * args.lds;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int m = tl.m0 + lane + 32 * c;
+            qa[j][c] = (in && m < args.M) ? __ldg(sa_kb + m) : 1.0f;
+          }
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int nb = tl.n0 / 128 + hh;
+            qb[j][hh] = (in && nb < NB) ? __ldg(args.sw + static_cast<int64_t>(nb) * KB + lg + j)
+                                        : 127u;
+          }
+        }
+        lg += kSfGroup;
+        if (lg >= KB) {
+          lg = 0;
+          lt += gridDim.x;
+        }
+      };
+      load_group();
+      uint32_t gi = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        for (int g0 = 0; g0 < KB; g0 += kSfGroup, ++gi) {
+          const uint32_t j = gi & 1u, ph = (gi >> 1) & 1u;
+          // the MMAs of the group that last used this slot have completed
+          if (!wait_warp(bar_sfempty + 8 * j, ph ^ 1u, s_abort)) { ok = false; break; }
+          uint8_t *tile = smem + kOffSf + j * kSfSlotBytes;
+          uint32_t w[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            w[c] = e8m0_of_pow2(qa[0][c]) | (e8m0_of_pow2(qa[1][c]) << 8) |
+                   (e8m0_of_pow2(qa[2][c]) << 16) | (e8m0_of_pow2(qa[3][c]) << 24);
+          *reinterpret_cast<uint4 *>(tile + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint32_t bw =
+                qb[0][hh] | (qb[1][hh] << 8) | (qb[2][hh] << 16) | (qb[3][hh] << 24);
+            *reinterpret_cast<uint4 *>(tile + (1 + hh) * kSfTileBytes + lane * 16) =
+                make_uint4(bw, bw, bw, bw);
+          }
+          fence_proxy_async_shared();  // generic-proxy writes -> the tensor core's reads
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_sffull + 8 * j);
+          load_group();
+        }
+      }
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        uint32_t it = 0, tile_it = 0, gi = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++tile_it) {
+          // the epilogue has moved the previous tile out of the accumulator
+          if (!wait_one(bar_tempty, (tile_it & 1u) ^ 1u, s_abort)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t tsf = 0;
+          for (int kb = 0; kb < KB; ++kb, ++it) {
+            const uint32_t sfj = static_cast<uint32_t>(kb % kSfGroup);
+            if (sfj == 0) {
+              const uint32_t j = gi & 1u, ph = (gi >> 1) & 1u;
+              if (!wait_one(bar_sffull + 8 * j, ph, s_abort)) { ok = false; break; }
+              tc_fence_after();
+              tsf = tmem_base + 256 + 16 * j;
+              const uint32_t sft = sbase + kOffSf + j * kSfSlotBytes;
+              tmem_cp_32x128b_x4(tsf, sdesc_sf(sft));
+              tmem_cp_32x128b_x4(tsf + 4, sdesc_sf(sft + kSfTileBytes));
+              tmem_cp_32x128b_x4(tsf + 8, sdesc_sf(sft + 2 * kSfTileBytes));
+            }
+            const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            if (!wait_one(bar_full + 8 * s, ph, s_abort)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t ad = sdesc_k128(sbase + kOffA + s * kTileABytes);
+            const uint64_t bd = sdesc_k128(sbase + kOffB + s * kTileBBytes);
+            const uint32_t idesc = mx_idesc(sfj);
+            const uint32_t tsfa = tsf | (sfj << 30), tsfb = (tsf + 4) | (sfj << 30);
+#pragma unroll
+            for (int kk = 0; kk < kBK / 32; ++kk)
+              mma_mxf8f6f4(tmem_base, ad + 2 * kk, bd + 2 * kk, idesc, tsfa, tsfb,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(bar_empty + 8 * s);
+            if (sfj == kSfGroup - 1 || kb == KB - 1) {
+              mma_commit(bar_sfempty + 8 * (gi & 1u));  // the group's scale slot is free
+              ++gi;
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar_tfull);
+        }
+        // Every MMA and copy has completed before TMEM is released.
+        mma_commit(bar_done);
+        wait_drain(bar_done, 0);
+      }
+      __syncwarp();
+    }
+  } else {
+    reg_alloc<kEpilogueRegs>();
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;         // TMEM lane quarter = rows 32q .. 32q + 31 of the tile
+    const int h = (warp - 4) >> 2;  // column half of the 256-wide tile
+    uint8_t *stage = smem + kOffStaging + (warp - 4) * kStagingBytesPerWarp;
+    const uint32_t stage_u32 = smem_u32(stage);
+    uint32_t tile_it = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tile_it) {
+      const Tile tl = dense_tile(ga, t);
+      const bool col_ok = tl.n0 / 128 + h < NB;
+      if (!wait_warp(bar_tfull, tile_it & 1u, s_abort)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + h * 128;
+      // the tile's 128 columns: eight 16-column loads in flight together, one wait
+      uint32_t r[8][16];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) tmem_ld_32x32b_x16(taddr + 16 * c, r[c]);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) tmem_ld_wait(r[c]);
+      // the whole tile is in registers: the accumulator goes back to the MMA
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_tempty);
+      uint32_t pk[4][16];
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const __nv_bfloat162 v2 = __floats2bfloat162_rn(__uint_as_float(r[c][2 * j]),
+                                                          __uint_as_float(r[c][2 * j + 1]));
+          pk[c / 2][8 * (c & 1) + j] = *reinterpret_cast<const uint32_t *>(&v2);
+        }
+      uint16_t *out_base = args.out + static_cast<int64_t>(tl.n0 + 128 * h);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        store_packed32(pk[c4], stage_u32, lane, out_base, tl, q, c4, col_ok, args.ldo);
     }
     tc_fence_before();
   }

@@ -173,6 +173,28 @@ __device__ __forceinline__ void mma_f8f6f4(uint32_t tmem_d, uint64_t adesc, uint
       : "memory");
 }
 
+// D (+)= A x B with block scaling, kind::mxf8f6f4 (E4M3 operands, one UE8M0 scale per 32 K-elements
+// of each row of A and each column of B, read from tensor memory at tsfa / tsfb; the scale IDs in
+// the instruction descriptor pick the byte of each 32-bit TMEM cell).
+__device__ __forceinline__ void mma_mxf8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Copy 32 rows x 128 bits from shared memory (matrix descriptor sdesc) into TMEM lanes 0-31,
+// columns taddr .. taddr + 3, replicated into the other three 32-lane sub-partitions.  Executes in
+// issue order with the tcgen05.mma instructions of the same thread.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 operation issued so far by this thread completes.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

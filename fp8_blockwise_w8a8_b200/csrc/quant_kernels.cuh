@@ -700,6 +700,12 @@ __global__ void __launch_bounds__(512) k_inverse_rope_quant(
   const int grp = lane / LPB, sub = lane % LPB;
   if (FMT == kScaleF32) build_scale_tab(tab, threadIdx.x, blockDim.x);
   __syncthreads();
+  // Offset inside its head of each chunk this lane owns at the first step, and the advance per
+  // step (BPS blocks) modulo D: the offsets then follow without a division per step.
+  int d_first[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) d_first[c] = (grp * 128 + (sub + LPB * c) * 8) % D;
+  const int d_step = (BPS * 128) % D;
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
   for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < T; m += stride) {
@@ -717,16 +723,21 @@ __global__ void __launch_bounds__(512) k_inverse_rope_quant(
     uint4 xn[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) xn[c] = ld_stream_v4(xr + bl * 128 + (sub + LPB * c) * 8);
+    int d0c[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) d0c[c] = d_first[c];
     for (int b0 = 0; b0 < KB; b0 += BPS) {
       const int b = b0 + grp;
       const bool active = b < KB;
       uint4 v[CPL];
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
-        const int k0 = bl * 128 + (sub + LPB * c) * 8;
-        const int d0 = k0 % D;
+        // while active, xn[c] holds block b and d0 is its chunk's offset inside the head
+        const int k0 = b * 128 + (sub + LPB * c) * 8;
+        const int d0 = d0c[c];
+        d0c[c] = d0 + d_step >= D ? d0 + d_step - D : d0 + d_step;
         v[c] = xn[c];
-        if (d0 >= pass) {
+        if (active && d0 >= pass) {
           const int j0 = d0 - pass;
           if (INTERLEAVED) {
             v[c] = inv_rope8_pairs(xn[c], ldg_f4(cs + j0 / 2), ldg_f4(sn + j0 / 2));

@@ -68,7 +68,8 @@ typedef enum {
   FP8Q_ERR_TIMEOUT = 6, /* (device error word) a kernel gave up on a bounded wait */
   FP8Q_ERR_ARG = 7,     /* an enum argument is out of range */
   FP8Q_ERR_TOO_LARGE = 8, /* the problem does not fit the library's static split-K scratch */
-  FP8Q_ERR_RANGE = 9      /* (device error word) a RoPE position was outside [0, max_pos) */
+  FP8Q_ERR_RANGE = 9,     /* (device error word) a RoPE position was outside [0, max_pos) */
+  FP8Q_ERR_NOT_POW2 = 10  /* (device error word) an MX-GEMM activation scale is not 2^e */
 } fp8q_status;
 
 typedef enum {
@@ -187,6 +188,28 @@ int fp8q_gemm_w8a8_block_diag(const void *aq, int64_t lda, const float *sa, int6
                               const void *wq, int64_t ldw, const void *sw, int sw_fmt,
                               int64_t G, int64_t M, int64_t N_g, int64_t K_g, void *out_bf16,
                               int64_t ldo, cudaStream_t stream);
+
+/* W8A8 GEMM with hardware block scaling for power-of-two (E8M0) scales, dense (G = 1) or
+ * block-diagonal over G head groups (as fp8q_gemm_w8a8_block_diag):
+ *   out[m][g N_g + n] = sum over kb of sa[(g KB_g + kb) lds + m] * 2^(sw[g][n/128][kb] - 127)
+ *                       * (dot product of the 128 codes of K-block kb)
+ * The tensor core applies both scales (tcgen05.mma kind::mxf8f6f4.block_scale, the 128-group
+ * scale given to each of its four 32-element sub-blocks) and accumulates all of K in fp32; no
+ * software promotion.  The sum is the one fp8q_gemm_w8a8_block computes, within the same
+ * tolerance.
+ *   aq       [M][lda] uint8 codes, lda >= G K_g
+ *   sa       fp32 activation scales, K-block-major sa[kb * lds + m]; every value must be a power
+ *            of two in [2^-127, 2^127] (what FP8Q_SCALE_E8M0 quantizers write); any other value
+ *            records FP8Q_ERR_NOT_POW2 in the device error word and the outputs are invalid
+ *   wq       [G][N_g][ldw] uint8 codes; sw_e8m0 [G][N_g/128][K_g/128] E8M0 bytes
+ *   out      [M][ldo] bf16, ldo >= G N_g
+ * N_g % 128 == 0 (% 256 when G > 1), K_g % 128 == 0.  Source: vLLM PR 54894 analysis, sections 1-3
+ * (E8M0 scales; batched_gemm_a8w8_mxscale(o_fp8, weight, o_scale, e8m0_scale) consumes the
+ * inverse-RoPE quant's output with MX scales on both operands). */
+int fp8q_gemm_w8a8_mx(const void *aq, int64_t lda, const float *sa, int64_t lds,
+                      const void *wq, int64_t ldw, const void *sw_e8m0, int64_t G, int64_t M,
+                      int64_t N_g, int64_t K_g, void *out_bf16, int64_t ldo,
+                      cudaStream_t stream);
 
 /* Grouped W8A8 GEMM for MoE experts (a6): for each expert e the rows
  * [group_offsets[e], group_offsets[e+1]) of aq/sa/out are multiplied by expert e's weight.

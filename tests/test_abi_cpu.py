@@ -33,7 +33,7 @@ def test_exports_match_header(L):
 
 
 def test_status_strings(L):
-    for s in range(10):
+    for s in range(11):
         assert len(_lib.status_string(s)) >= 2
     assert _lib.status_string(99) == "unknown status"
 
@@ -214,4 +214,24 @@ def test_block_diag_gemm_host_checks(L):
     assert call(fmt=3) == _lib.FP8Q_ERR_ARG
     assert call(sw=None) == _lib.FP8Q_ERR_NULL
     assert call(lda=1032) == _lib.FP8Q_ERR_ALIGN
+    assert call(M=0, aq=None, sa=None, out=None) == _lib.FP8Q_OK
+
+
+def test_mx_gemm_host_checks(L):
+    g = L.fp8q_gemm_w8a8_mx
+    ok = dict(aq=FAKE, lda=1024, sa=FAKE, lds=64, wq=FAKE, ldw=512, sw=FAKE, G=2, M=64, N_g=256,
+              K_g=512, out=FAKE, ldo=512)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return g(a["aq"], a["lda"], a["sa"], a["lds"], a["wq"], a["ldw"], a["sw"], a["G"],
+                 a["M"], a["N_g"], a["K_g"], a["out"], a["ldo"], None)
+    assert call(N_g=128, ldo=256) == _lib.FP8Q_ERR_SHAPE                  # groups: N_g % 256
+    assert call(G=1, N_g=100, ldo=128) == _lib.FP8Q_ERR_SHAPE             # N % 128
+    assert call(K_g=200, ldw=208) == _lib.FP8Q_ERR_SHAPE
+    assert call(lda=768) == _lib.FP8Q_ERR_SHAPE
+    assert call(lds=32) == _lib.FP8Q_ERR_SHAPE
+    assert call(sw=None) == _lib.FP8Q_ERR_NULL
+    assert call(sa=FAKE + 2) == _lib.FP8Q_ERR_ALIGN
+    assert call(ldo=516) == _lib.FP8Q_ERR_ALIGN
     assert call(M=0, aq=None, sa=None, out=None) == _lib.FP8Q_OK
