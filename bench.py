@@ -746,6 +746,12 @@ def run_ncu_case(name):
         out = torch.empty((8192, 4096), dtype=torch.bfloat16, device=dev)
         fn = lambda: fq.gemm_w8a8_block_diag(aq, sa, wq.view(4, 1024, 4096),
                                              sw.view(4, 8, 32), out=out)
+    elif name == "gemm_mx_prefill":      # the prefill GEMM with E8M0 scales, hardware block scaling
+        x = randn((M_, K_), 1.0)
+        aq, sa = fq.inverse_rope_quant(x.view(M_, 1, K_), None, None, None, 0, True, "e8m0")
+        wq, sw = fq.quant_weight_block(randn((N_, K_), 0.02), "e8m0")
+        out = torch.empty((M_, N_), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm_w8a8_mx(aq, sa, wq, sw, out=out)
     else:
         raise SystemExit(f"unknown --ncu-case {name}")
     torch.cuda.synchronize()

@@ -158,3 +158,28 @@ def test_token_zero_rows_and_sign_of_zero():
     _token_case(x)
     g = np.full(256, 0x3F80, np.uint16)
     _token_case(x, g, 1e-6)
+
+
+@pytest.mark.parametrize("K", [640, 768, 1920, 2048, 3968])
+@pytest.mark.parametrize("M", [1, 37, 301])
+def test_token_rows_sharing_a_warp(K, M):
+    """Rows of fewer than 32 blocks: several rows per warp (32 // (K / 128) of them), a last
+    row group that is cut short by M, with and without RMSNorm."""
+    x = inputs.randn_bf16((M, K), 1.0, 93, K + M)
+    g = inputs.to_bf16_bits(np.random.default_rng(K).uniform(0.5, 1.5, K).astype(np.float32))
+    _token_case(x, g, 1e-6)
+    _token_case(x, None)
+
+
+def test_token_strided_rows():
+    M, K = 70, 1024
+    x = inputs.randn_bf16((M, K + 64), 1.0, 94, 0)
+    xs = dev_bf16(x)[:, :K]
+    g = inputs.to_bf16_bits(np.random.default_rng(5).uniform(0.5, 1.5, K).astype(np.float32))
+    for gamma in (g, None):
+        q, sa = fq.rmsnorm_quant_token(xs, None if gamma is None else dev_bf16(gamma), 1e-6)
+        assert fq.check_device_error() == 0
+        q_ref, sa_ref = oracle.rmsnorm_quant_token(np.ascontiguousarray(x[:, :K]), gamma, 1e-6,
+                                                   lds=sa.shape[1])
+        assert np.array_equal(q.cpu().numpy(), q_ref)
+        assert np.array_equal(sa.cpu().numpy()[:, :M], sa_ref[:, :M])
