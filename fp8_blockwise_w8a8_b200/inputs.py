@@ -24,6 +24,10 @@ bf16 tensors are returned as numpy ``uint16`` bit patterns (host) or torch ``bfl
                    of each head the rotary part; positions ~ U[0, 16384); cos/sin caches
                    [16384, 32] of the angle p * 10000^(-2i/64), computed in float64 and rounded
                    to fp32; 4 head groups, W_wo_a [4, 1024, 8 * 512] ~ N(0, 0.02); seed 5
+* FP8 KV cache     QKV activations [8192 tokens, (32 + 2 x 8) heads x 128]: Q ~ N(0,1), K ~ N(0,1)
+                   with 4 channels per head x 8, V ~ N(0, 0.5); a paged cache of 1024 blocks x 16
+                   slots; each token gets a distinct random slot, 2 % of them -1 (padding, not
+                   cached); seed 6
 """
 import numpy as np
 import torch
@@ -151,3 +155,21 @@ def wo_a(tokens: int = 8192, heads: int = 32, head_dim: int = 512, rope_dim: int
     if with_weight:
         out["W"] = randn_bf16((groups, out_per_group, heads // groups * head_dim), 0.02, seed, 2)
     return out
+
+
+def kv_cache(tokens: int = 8192, q_heads: int = 32, kv_heads: int = 8, head_dim: int = 128,
+             num_blocks: int = 1024, block_size: int = 16):
+    seed = 6
+    r = rng_for(seed, 1)
+    D = head_dim
+    q = r.standard_normal((tokens, q_heads * D)).astype(np.float32)
+    k = r.standard_normal((tokens, kv_heads, D)).astype(np.float32)
+    outl = r.choice(D, size=4, replace=False)
+    k[:, :, outl] *= 8.0
+    v = (0.5 * r.standard_normal((tokens, kv_heads * D))).astype(np.float32)
+    qkv = to_bf16_bits(np.concatenate([q, k.reshape(tokens, -1), v], axis=1))
+    num_slots = num_blocks * block_size
+    slots = r.permutation(num_slots)[:tokens].astype(np.int64)
+    slots[r.random(tokens) < 0.02] = -1
+    return {"qkv": qkv, "slots": slots, "num_slots": num_slots, "Hq": q_heads, "Hkv": kv_heads,
+            "D": D}

@@ -66,6 +66,12 @@ def lib():
         L.oracle_inverse_rope_quant.argtypes = [P, P, P, P, I64, I64, I64, I64, ctypes.c_int,
                                                 ctypes.c_int, P, P, I64]
         L.oracle_inverse_rope_quant.restype = None
+        L.oracle_qkv_amax.argtypes = [P, I64, I64, I64, I64, I64, P]
+        L.oracle_qkv_amax.restype = None
+        L.oracle_qkv_scales.argtypes = [P, P]
+        L.oracle_qkv_scales.restype = None
+        L.oracle_kv_cache_write.argtypes = [P, I64, I64, I64, I64, I64, P, P, P, I64, P, P]
+        L.oracle_kv_cache_write.restype = None
         L.oracle_quant_rowwise.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64, P]
         L.oracle_quant_rowwise.restype = None
         L.oracle_gemm_w8a8_rowwise_rows.argtypes = [P, I64, P, P, I64, P, I64, I64, P, I64, P, P]
@@ -316,6 +322,38 @@ def inverse_rope_quant(o_bf16: np.ndarray, positions, cos_cache, sin_cache, rope
     lib().oracle_inverse_rope_quant(_ptr(o), _ptr(pos), _ptr(c), _ptr(sn), T, H, D, rope_dim,
                                     int(interleaved), int(fmt), _ptr(q), _ptr(sa), lds)
     return q, sa
+
+
+def qkv_amax(qkv_bf16: np.ndarray, Hq: int, Hkv: int, D: int) -> np.ndarray:
+    """Per-tensor absolute maxima (Q, K, V) of a QKV activation [T, (Hq + 2 Hkv) D] (R10)."""
+    x = _c(qkv_bf16, np.uint16)
+    a = np.zeros(3, np.float32)
+    lib().oracle_qkv_amax(_ptr(x), x.shape[0], x.shape[1], Hq, Hkv, D, _ptr(a))
+    return a
+
+
+def qkv_scales(amax3) -> np.ndarray:
+    """Per-tensor scales of reading R10: amax / 448 in fp32, 1 for an all-zero tensor."""
+    a = _c(np.asarray(amax3, np.float32), np.float32)
+    s = np.zeros(3, np.float32)
+    lib().oracle_qkv_scales(_ptr(a), _ptr(s))
+    return s
+
+
+def kv_cache_write(qkv_bf16: np.ndarray, Hq: int, Hkv: int, D: int, slots, scales3,
+                   k_cache: np.ndarray, v_cache: np.ndarray) -> np.ndarray:
+    """Writes K and V codes into rows slots[t] of k_cache / v_cache (uint8 [num_slots, Hkv D],
+    updated in place; negative slots skipped) and returns the Q codes [T, Hq D]."""
+    x = _c(qkv_bf16, np.uint16)
+    T = x.shape[0]
+    sl = _c(np.asarray(slots, np.int64), np.int64)
+    sc = _c(np.asarray(scales3, np.float32), np.float32)
+    assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
+    assert k_cache.dtype == np.uint8 and v_cache.dtype == np.uint8
+    q = np.zeros((T, Hq * D), np.uint8)
+    lib().oracle_kv_cache_write(_ptr(x), T, x.shape[1], Hq, Hkv, D, _ptr(sl), _ptr(sc), _ptr(q),
+                                Hq * D, _ptr(k_cache), _ptr(v_cache))
+    return q
 
 
 def quant_rowwise(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6):

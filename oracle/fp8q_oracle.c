@@ -62,6 +62,13 @@
  *       heads x head_dim row of each token, scales K-block-major as R5 (each head group's
  *       K-blocks are then contiguous).  The scale is R1's fp32 amax/448, or, since the GEMM that
  *       follows on the page takes MX (E8M0) scales, R2's power of two, stored as its fp32 value.
+ *   R10 FP8 KV cache with per-step QKV scale recalibration [FP8-RL abstract, item (ii)]: each
+ *       step, one fp32 scale per tensor (Q, K, V of a layer) is recomputed from the step's QKV
+ *       activations with R1's rule, s = amax / 448 over the whole tensor (0 -> 1); K and V
+ *       are then stored in the cache as E4M3 codes RNEsat(x / s) (R1's element rule) at the
+ *       slots given per token (a negative slot: the token is not cached), and Q is quantized
+ *       the same way for the attention that reads the cache.  The QKV row of a token holds
+ *       Hq heads of Q, then Hkv of K, then Hkv of V, each of D values.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math -fopenmp.
  * fp32 arithmetic below relies on FLT_EVAL_METHOD == 0 (SSE on x86-64), so every float
@@ -470,6 +477,52 @@ void oracle_inverse_rope_quant(const uint16_t *o, const int64_t *pos, const floa
                 for (int j = 0; j < 128; ++j) qg[j] = oracle_e4m3_encode(y[j] / s);
                 sa[kb * lds + t] = s;
             }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* FP8 KV cache: per-step QKV scale recalibration and cache write [FP8-RL (ii)], reading R10    */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Absolute maxima of the Q, K and V parts of qkv bf16 [T][ld] (row = Hq*D of Q, Hkv*D of K,
+ * Hkv*D of V) into amax3[0..2]. */
+void oracle_qkv_amax(const uint16_t *qkv, int64_t T, int64_t ld, int64_t Hq, int64_t Hkv,
+                     int64_t D, float *amax3) {
+    int64_t width[3] = {Hq * D, Hkv * D, Hkv * D};
+    int64_t start = 0;
+    for (int part = 0; part < 3; ++part) {
+        float amax = 0.0f;
+        for (int64_t t = 0; t < T; ++t)
+            for (int64_t c = 0; c < width[part]; ++c) {
+                float a = fabsf(bf16_to_f32(qkv[t * ld + start + c]));
+                if (a > amax) amax = a;
+            }
+        amax3[part] = amax;
+        start += width[part];
+    }
+}
+
+/* The per-tensor scales of reading R10 from the maxima. */
+void oracle_qkv_scales(const float *amax3, float *scale3) {
+    for (int part = 0; part < 3; ++part) scale3[part] = scale_f32_from_amax(amax3[part]);
+}
+
+/* Quantize every token's Q into q_out [T][ldq] and write its K and V codes into row slots[t] of
+ * k_cache / v_cache ([num_slots][Hkv*D] each); slots[t] < 0 leaves the caches untouched. */
+void oracle_kv_cache_write(const uint16_t *qkv, int64_t T, int64_t ld, int64_t Hq, int64_t Hkv,
+                           int64_t D, const int64_t *slots, const float *scale3, uint8_t *q_out,
+                           int64_t ldq, uint8_t *k_cache, uint8_t *v_cache) {
+    int64_t wq = Hq * D, wkv = Hkv * D;
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *row = qkv + t * ld;
+        for (int64_t c = 0; c < wq; ++c)
+            q_out[t * ldq + c] = oracle_e4m3_encode(bf16_to_f32(row[c]) / scale3[0]);
+        if (slots[t] < 0) continue;
+        for (int64_t c = 0; c < wkv; ++c) {
+            k_cache[slots[t] * wkv + c] = oracle_e4m3_encode(bf16_to_f32(row[wq + c]) / scale3[1]);
+            v_cache[slots[t] * wkv + c] =
+                oracle_e4m3_encode(bf16_to_f32(row[wq + wkv + c]) / scale3[2]);
         }
     }
 }
