@@ -439,6 +439,37 @@ def measure_rows(fq, device, steps, warmup, pk):
     del o_d, pos_d, cos_d, sin_d, W, wq, sw, q_d, sa_d, out_d
     torch.cuda.empty_cache()
 
+    # FP8 KV cache: per-step recalibration of the per-tensor QKV scales, then the cache write
+    kv = inputs.kv_cache()
+    Hq, Hkv, Dh = kv["Hq"], kv["Hkv"], kv["D"]
+    qkv = dev_bf16(kv["qkv"], device)
+    T = qkv.shape[0]
+    slots = torch.from_numpy(kv["slots"]).to(device)
+    kc = torch.zeros((kv["num_slots"], Hkv * Dh), dtype=torch.uint8, device=device)
+    vc = torch.zeros_like(kc)
+    amax3 = torch.empty(3, dtype=torch.float32, device=device)
+    sc3 = torch.empty(3, dtype=torch.float32, device=device)
+    qo = torch.empty((T, Hq * Dh), dtype=torch.uint8, device=device)
+    ms, _ = timed_loop(lambda: fq.qkv_scales(qkv, Hq, Hkv, Dh, out_amax=amax3, out_scales=sc3),
+                       steps, warmup, flush)
+    byts = qkv.numel() * 2
+    rows["kv_qkv_scales_prefill"] = {"ms": ms, "GB/s": byts / ms / 1e6, "frac": byts / ms / 1e6 / hbm,
+                                     "workload": f"QKV [{T}, {qkv.shape[1]}] -> 3 scales",
+                                     "launches": 3}
+    cached = int((kv["slots"] >= 0).sum())
+    byts = qkv.numel() * 2 + T * 8 + T * Hq * Dh + cached * 2 * Hkv * Dh
+    ms, _ = timed_loop(lambda: fq.kv_cache_write(qkv, Hq, Hkv, Dh, slots, sc3, kc, vc, out_q=qo),
+                       steps, warmup, flush)
+    rows["kv_cache_write_prefill"] = {
+        "ms": ms, "GB/s": byts / ms / 1e6, "frac": byts / ms / 1e6 / hbm,
+        "workload": f"{T} tokens, Q {Hq}x{Dh} quantized, K and V {Hkv}x{Dh} to cache slots"}
+    dq = qkv[:256]
+    ms, _ = timed_loop(lambda: fq.kv_cache_write(dq, Hq, Hkv, Dh, slots[:256], sc3, kc, vc,
+                                                 out_q=qo[:256]), steps, warmup, flush)
+    rows["kv_cache_write_decode"] = {"ms": ms, "workload": "256 decode tokens (launch-bound)"}
+    del kv, qkv, slots, kc, vc, qo
+    torch.cuda.empty_cache()
+
     # the prefill GEMM with power-of-two scales on both operands, hardware block scaling
     pf = inputs.prefill_linear()
     X = dev_bf16(pf["X"], device)

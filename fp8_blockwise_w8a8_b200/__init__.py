@@ -24,7 +24,7 @@ import ctypes
 __all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
            "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant", "inverse_rope_quant",
-           "gemm_w8a8_block_diag", "gemm_w8a8_mx",
+           "gemm_w8a8_block_diag", "gemm_w8a8_mx", "qkv_scales", "kv_cache_write",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -245,6 +245,43 @@ def gemm_w8a8_mx(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, sw: torch
                                       _ptr(sw), G, M, N_g, K_g, _ptr(o), _ld(o), _stream(stream))
     _lib.check(st, "fp8q_gemm_w8a8_mx")
     return o
+
+
+def qkv_scales(qkv: torch.Tensor, Hq: int, Hkv: int, D: int, out_amax=None, out_scales=None,
+               stream=None):
+    """Per-step recalibration of the FP8 KV-cache scales: QKV activations bf16
+    [T, (Hq + 2 Hkv) D] -> (amax fp32 [3], scales fp32 [3]) for Q, K, V."""
+    T = qkv.shape[0]
+    a = torch.empty(3, dtype=torch.float32, device=qkv.device) if out_amax is None else out_amax
+    s = torch.empty(3, dtype=torch.float32, device=qkv.device) if out_scales is None else out_scales
+    st = _lib.lib().fp8q_qkv_scales(_ptr(qkv), T, _ld(qkv), Hq, Hkv, D, _ptr(a), _ptr(s),
+                                    _stream(stream))
+    _lib.check(st, "fp8q_qkv_scales")
+    return a, s
+
+
+def kv_cache_write(qkv: torch.Tensor, Hq: int, Hkv: int, D: int, slots: torch.Tensor,
+                   scales: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   out_q=None, quantize_q: bool = True, stream=None):
+    """Quantize Q (returned, uint8 [T, Hq D], unless quantize_q is False) and write the E4M3
+    codes of K and V into rows slots[t] of k_cache / v_cache (uint8, [num_slots, Hkv D] or any
+    contiguous view of it, e.g. [blocks, block_size, Hkv, D])."""
+    T = qkv.shape[0]
+    for c, name in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        if c.dtype != torch.uint8 or not c.is_contiguous() or c.numel() % (Hkv * D):
+            raise ValueError(f"{name} must be a contiguous uint8 tensor of whole Hkv*D rows")
+    if slots.dtype != torch.int64 or slots.numel() != T or not slots.is_contiguous():
+        raise ValueError("slots must be a contiguous int64 tensor of T entries")
+    num_slots = k_cache.numel() // (Hkv * D)
+    q = None
+    if quantize_q:
+        q = torch.empty((T, Hq * D), dtype=torch.uint8, device=qkv.device) if out_q is None else out_q
+    st = _lib.lib().fp8q_kv_cache_write(_ptr(qkv), T, _ld(qkv), Hq, Hkv, D, _ptr(slots),
+                                        num_slots, _ptr(scales), _ptr(q),
+                                        q.stride(0) if q is not None else 0, _ptr(k_cache),
+                                        _ptr(v_cache), _stream(stream))
+    _lib.check(st, "fp8q_kv_cache_write")
+    return q
 
 
 def quant_rowwise(x: torch.Tensor, gamma=None, eps: float = 1e-6, out_q=None, out_s=None,

@@ -47,6 +47,9 @@ SIGNATURES = {
                                        _I64, _P, _I64, _P]),
     "fp8q_gemm_w8a8_mx": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _P,
                                _I64, _P]),
+    "fp8q_qkv_scales": (_I, [_P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P]),
+    "fp8q_kv_cache_write": (_I, [_P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P,
+                                 _P]),
     "fp8q_quant_rowwise": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "fp8q_gemm_w8a8_rowwise": (_I, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I64, _P]),
     "fp8q_check_device_error": (_I, [_P]),

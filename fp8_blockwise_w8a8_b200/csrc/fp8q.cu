@@ -235,7 +235,7 @@ const char *fp8q_status_string(int status) {
     case FP8Q_ERR_TIMEOUT: return "a kernel gave up on a bounded wait (outputs incomplete)";
     case FP8Q_ERR_ARG: return "enum argument out of range";
     case FP8Q_ERR_NOT_POW2: return "a scale given to the hardware block-scaled GEMM is not a power of two (outputs invalid)";
-    case FP8Q_ERR_RANGE: return "an index input (a RoPE position) was outside its table; that row was not written";
+    case FP8Q_ERR_RANGE: return "an index or scale input was outside its valid range (a RoPE position, a cache slot, a non-positive or non-finite scale); the affected rows were not written";
     case FP8Q_ERR_TOO_LARGE: return "problem needs more split-K scratch than the library's static 24 MiB buffer (use fp8q_gemm_w8a8_block_splitk with a workspace, or fewer splits)";
     default: return "unknown status";
   }
@@ -567,6 +567,59 @@ int fp8q_inverse_rope_quant(const void *o_bf16, int64_t ldo, const int64_t *posi
                                      cos_cache, sin_cache, max_pos, T, static_cast<int>(D),
                                      static_cast<int>(rope_dim), static_cast<int>(K),
                                      static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
+  return launch_status();
+}
+
+int fp8q_qkv_scales(const void *qkv_bf16, int64_t T, int64_t ld, int64_t Hq, int64_t Hkv,
+                    int64_t D, float *amax3, float *scale3, cudaStream_t stream) {
+  if (T < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || D % 8) return FP8Q_ERR_SHAPE;
+  if ((Hq + 2 * Hkv) * D > (1 << 24) || ld < (Hq + 2 * Hkv) * D) return FP8Q_ERR_SHAPE;
+  if (!amax3 || !scale3 || (T > 0 && !qkv_bf16)) return FP8Q_ERR_NULL;
+  if ((T > 0 && !aligned16(qkv_bf16)) || ld % 8 || (reinterpret_cast<uintptr_t>(amax3) & 3u) ||
+      (reinterpret_cast<uintptr_t>(scale3) & 3u))
+    return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  if (cudaMemsetAsync(amax3, 0, 3 * sizeof(float), stream) != cudaSuccess) return FP8Q_ERR_LAUNCH;
+  if (T > 0) {
+    const int64_t need = (T + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(st->sms) * 8;
+    const int grid = static_cast<int>(need < cap ? need : cap);
+    fp8q::k_qkv_amax<<<grid, 256, 0, stream>>>(
+        static_cast<const uint16_t *>(qkv_bf16), ld, T, static_cast<int>(Hq * D / 8),
+        static_cast<int>(Hkv * D / 8), static_cast<int>(Hkv * D / 8),
+        reinterpret_cast<uint32_t *>(amax3));
+    const int lrc = launch_status();
+    if (lrc != FP8Q_OK) return lrc;
+  }
+  fp8q::k_qkv_finalize<<<1, 32, 0, stream>>>(reinterpret_cast<const uint32_t *>(amax3), scale3);
+  return launch_status();
+}
+
+int fp8q_kv_cache_write(const void *qkv_bf16, int64_t T, int64_t ld, int64_t Hq, int64_t Hkv,
+                        int64_t D, const int64_t *slots, int64_t num_slots, const float *scale3,
+                        void *q_e4m3, int64_t ldq, void *k_cache, void *v_cache,
+                        cudaStream_t stream) {
+  if (T < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || D % 16 || num_slots < 0) return FP8Q_ERR_SHAPE;
+  if ((Hq + 2 * Hkv) * D > (1 << 24) || ld < (Hq + 2 * Hkv) * D) return FP8Q_ERR_SHAPE;
+  if (q_e4m3 && ldq < Hq * D) return FP8Q_ERR_SHAPE;
+  if (T == 0) return FP8Q_OK;
+  if (!qkv_bf16 || !slots || !scale3 || !k_cache || !v_cache) return FP8Q_ERR_NULL;
+  if (!aligned16(qkv_bf16) || ld % 8 || (reinterpret_cast<uintptr_t>(slots) & 7u) ||
+      (reinterpret_cast<uintptr_t>(scale3) & 3u) || (reinterpret_cast<uintptr_t>(k_cache) & 7u) ||
+      (reinterpret_cast<uintptr_t>(v_cache) & 7u) ||
+      (q_e4m3 && ((reinterpret_cast<uintptr_t>(q_e4m3) & 7u) || ldq % 8)))
+    return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  const int64_t cap = static_cast<int64_t>(st->sms) * 16;
+  const int grid = static_cast<int>(T < cap ? T : cap);
+  fp8q::k_kv_cache_write<<<grid, fp8q::kKvThreads, 0, stream>>>(
+      static_cast<const uint16_t *>(qkv_bf16), ld, T, static_cast<int>(Hq * D / 8),
+      static_cast<int>(Hkv * D / 8), slots, num_slots, scale3, static_cast<uint8_t *>(q_e4m3),
+      ldq, static_cast<uint8_t *>(k_cache), static_cast<uint8_t *>(v_cache));
   return launch_status();
 }
 

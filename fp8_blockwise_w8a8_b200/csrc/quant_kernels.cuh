@@ -786,4 +786,125 @@ __global__ void __launch_bounds__(512) k_inverse_rope_quant(
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// FP8 KV cache with per-step QKV scale recalibration.  A token's QKV row holds Hq heads of Q, then
+// Hkv of K, then Hkv of V (D values each).  k_qkv_amax reduces |x| over each of the three parts
+// (warp, then CTA, then one atomicMax per part on the fp32 bit pattern, which orders non-negative
+// floats like their values); k_qkv_finalize turns the maxima into s = amax / 448 (1 for zero).
+// k_kv_cache_write quantizes Q into a dense buffer and K, V into the cache rows named by the
+// token's slot, with the bracket quantizer for an arbitrary fp32 scale (no tie shortcut: every
+// ambiguous bracket takes the exact fp64 quotient).
+// ---------------------------------------------------------------------------------------------
+constexpr int kErrRangeKv = 9;  // FP8Q_ERR_RANGE
+
+__device__ __forceinline__ QParams qparams_scale(float s) {
+  QParams p;
+  p.s = s;
+  p.tie = false;
+  p.fast = s >= 0x1.0p-60f && s <= 0x1.0p+100f;
+  const float r = rcp_approx(p.fast ? s : 1.0f);
+  const float lo = __fmul_rn(r, 0x1.ffffc0p-1f), hi = __fmul_rn(r, 0x1.000020p+0f);
+  p.lo2 = make_float2(lo, lo);
+  p.hi2 = make_float2(hi, hi);
+  return p;
+}
+
+// Grid: any number of CTAs of 256 threads; warps take rows, lanes 16-byte chunks of a row.
+__global__ void __launch_bounds__(256) k_qkv_amax(const uint16_t *__restrict__ qkv, int64_t ld,
+                                                  int64_t T, int cq, int ck, int cv,
+                                                  uint32_t *__restrict__ amax3) {
+  __shared__ float red[8][3];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int cw = cq + ck + cv;  // 16-byte chunks per row; Q chunks [0, cq), K [cq, cq + ck)
+  uint32_t m[3] = {0u, 0u, 0u};
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * 8;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * 8 + warp; t < T; t += wstride) {
+    const uint16_t *row = qkv + t * ld;
+#pragma unroll 8
+    for (int c = lane; c < cw; c += 32) {
+      const uint4 v = ld_stream_v4(row + c * 8);
+      const int part = c < cq ? 0 : (c < cq + ck ? 1 : 2);
+      const uint32_t a = absmax_uint4(0u, v);
+      m[0] = part == 0 ? absmax_bf16x2(m[0], a) : m[0];
+      m[1] = part == 1 ? absmax_bf16x2(m[1], a) : m[1];
+      m[2] = part == 2 ? absmax_bf16x2(m[2], a) : m[2];
+    }
+  }
+  float f[3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    f[i] = absmax_finish(m[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) f[i] = fmaxf(f[i], __shfl_xor_sync(0xffffffffu, f[i], o));
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) red[warp][i] = f[i];
+  }
+  __syncthreads();
+  if (threadIdx.x < 3) {
+    float v = red[0][threadIdx.x];
+    for (int w = 1; w < 8; ++w) v = fmaxf(v, red[w][threadIdx.x]);
+    atomicMax(amax3 + threadIdx.x, __float_as_uint(v));
+  }
+}
+
+__global__ void k_qkv_finalize(const uint32_t *__restrict__ amax3, float *__restrict__ scale3) {
+  if (threadIdx.x < 3) {
+    const float a = __uint_as_float(amax3[threadIdx.x]);
+    scale3[threadIdx.x] = a == 0.0f ? 1.0f : __fdiv_rn(a, 448.0f);
+  }
+}
+
+// Grid: CTAs of 128 threads, one token at a time per CTA; each thread loads up to 8 of the
+// token's 16-byte chunks before it converts any, so a token's loads are all in flight together.
+// A slot outside [0, num_slots) other than a negative one, or a scale that is not positive and
+// finite, records FP8Q_ERR_RANGE; the token's cache rows (for a bad scale: that part) are not
+// written.
+constexpr int kKvThreads = 128, kKvBatch = 8;
+__global__ void __launch_bounds__(kKvThreads) k_kv_cache_write(
+    const uint16_t *__restrict__ qkv, int64_t ld, int64_t T, int cq, int ckv,
+    const int64_t *__restrict__ slots, int64_t num_slots, const float *__restrict__ scale3,
+    uint8_t *__restrict__ q_out, int64_t ldq, uint8_t *__restrict__ k_cache,
+    uint8_t *__restrict__ v_cache) {
+  const float sq = __ldg(scale3), sk = __ldg(scale3 + 1), sv = __ldg(scale3 + 2);
+  const bool okq = sq > 0.0f && sq <= 0x1.fffffep+127f, okk = sk > 0.0f && sk <= 0x1.fffffep+127f,
+             okv = sv > 0.0f && sv <= 0x1.fffffep+127f;
+  const QParams pq = qparams_scale(okq ? sq : 1.0f), pk = qparams_scale(okk ? sk : 1.0f),
+                pv = qparams_scale(okv ? sv : 1.0f);
+  if (!(okq && okk && okv) && blockIdx.x == 0 && threadIdx.x == 0) record_error(kErrRangeKv);
+  const int cw = cq + 2 * ckv;
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const uint16_t *row = qkv + t * ld;
+    const int64_t slot = __ldg(slots + t);
+    const bool cached = slot >= 0 && slot < num_slots;
+    if (slot >= num_slots && threadIdx.x == 0) record_error(kErrRangeKv);
+    const bool do_q = q_out != nullptr && okq, do_k = cached && okk, do_v = cached && okv;
+    for (int base = 0; base < cw; base += kKvBatch * kKvThreads) {
+      uint4 v[kKvBatch];
+#pragma unroll
+      for (int j = 0; j < kKvBatch; ++j) {
+        const int c = base + j * kKvThreads + threadIdx.x;
+        const bool want = c < cq ? do_q : (c < cq + ckv ? do_k : do_v);
+        if (c < cw && want) v[j] = ld_stream_v4(row + c * 8);
+      }
+#pragma unroll
+      for (int j = 0; j < kKvBatch; ++j) {
+        const int c = base + j * kKvThreads + threadIdx.x;
+        if (c >= cw) continue;
+        if (c < cq) {
+          if (do_q) *reinterpret_cast<uint2 *>(q_out + t * ldq + c * 8) = quant8_f32(v[j], pq);
+        } else if (c < cq + ckv) {
+          if (do_k)
+            *reinterpret_cast<uint2 *>(k_cache + slot * (ckv * 8) + (c - cq) * 8) =
+                quant8_f32(v[j], pk);
+        } else if (do_v) {
+          *reinterpret_cast<uint2 *>(v_cache + slot * (ckv * 8) + (c - cq - ckv) * 8) =
+              quant8_f32(v[j], pv);
+        }
+      }
+    }
+  }
+}
+
 }  // namespace fp8q

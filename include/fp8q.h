@@ -68,7 +68,7 @@ typedef enum {
   FP8Q_ERR_TIMEOUT = 6, /* (device error word) a kernel gave up on a bounded wait */
   FP8Q_ERR_ARG = 7,     /* an enum argument is out of range */
   FP8Q_ERR_TOO_LARGE = 8, /* the problem does not fit the library's static split-K scratch */
-  FP8Q_ERR_RANGE = 9,     /* (device error word) a RoPE position was outside [0, max_pos) */
+  FP8Q_ERR_RANGE = 9,     /* (device error word) a position, cache slot or scale out of range */
   FP8Q_ERR_NOT_POW2 = 10  /* (device error word) an MX-GEMM activation scale is not 2^e */
 } fp8q_status;
 
@@ -210,6 +210,37 @@ int fp8q_gemm_w8a8_mx(const void *aq, int64_t lda, const float *sa, int64_t lds,
                       const void *wq, int64_t ldw, const void *sw_e8m0, int64_t G, int64_t M,
                       int64_t N_g, int64_t K_g, void *out_bf16, int64_t ldo,
                       cudaStream_t stream);
+
+/* FP8 KV cache, step 1: per-step recalibration of the per-tensor QKV scales.
+ *   qkv_bf16  [T][ld] bf16, read: each token's row holds Hq heads of Q, then Hkv heads of K, then
+ *             Hkv heads of V, D values per head (D % 8 == 0)
+ *   amax3     [3] fp32, DEVICE memory, written: max |x| over all of Q, of K, of V
+ *   scale3    [3] fp32, DEVICE memory, written: s = amax / 448 (IEEE fp32), 1 for an all-zero part
+ * Three stream operations: a memset of amax3, the reduction (one atomicMax per CTA and part on
+ * the fp32 bit pattern: the result does not depend on the order), and a one-warp finalize.  T may
+ * be 0 (scales 1).  Bit-exact against the CPU oracle.  Source: FP8-RL abstract, item (ii) (FP8
+ * KV cache with per-step QKV scale recalibration). */
+int fp8q_qkv_scales(const void *qkv_bf16, int64_t T, int64_t ld, int64_t Hq, int64_t Hkv,
+                    int64_t D, float *amax3, float *scale3, cudaStream_t stream);
+
+/* FP8 KV cache, step 2: quantize Q and write K and V into the cache.
+ *   qkv_bf16  as fp8q_qkv_scales (D % 16 == 0)
+ *   slots     [T] int64, DEVICE memory: the cache row of each token; a negative slot means the
+ *             token is not cached (padding); a slot >= num_slots records FP8Q_ERR_RANGE and the
+ *             token's cache rows are not written
+ *   scale3    [3] fp32, DEVICE memory: the per-tensor scales (from fp8q_qkv_scales, or the
+ *             caller's); a scale that is not positive and finite records FP8Q_ERR_RANGE and that
+ *             part is not written
+ *   q_e4m3    [T][ldq] uint8 codes of Q, written; may be NULL (Q not quantized)
+ *   k_cache, v_cache
+ *             [num_slots][Hkv * D] uint8 each (a paged cache [blocks][block_size][Hkv][D] seen
+ *             as slot-major rows), rows slots[t] written, all others untouched
+ * Codes are RNE-saturating E4M3 of x / s (one IEEE fp32 division), bit-exact against the CPU
+ * oracle.  Source: FP8-RL abstract, item (ii). */
+int fp8q_kv_cache_write(const void *qkv_bf16, int64_t T, int64_t ld, int64_t Hq, int64_t Hkv,
+                        int64_t D, const int64_t *slots, int64_t num_slots, const float *scale3,
+                        void *q_e4m3, int64_t ldq, void *k_cache, void *v_cache,
+                        cudaStream_t stream);
 
 /* Grouped W8A8 GEMM for MoE experts (a6): for each expert e the rows
  * [group_offsets[e], group_offsets[e+1]) of aq/sa/out are multiplied by expert e's weight.

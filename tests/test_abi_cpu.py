@@ -235,3 +235,27 @@ def test_mx_gemm_host_checks(L):
     assert call(sa=FAKE + 2) == _lib.FP8Q_ERR_ALIGN
     assert call(ldo=516) == _lib.FP8Q_ERR_ALIGN
     assert call(M=0, aq=None, sa=None, out=None) == _lib.FP8Q_OK
+
+
+def test_kv_cache_host_checks(L):
+    f = L.fp8q_qkv_scales
+    assert f(FAKE, 8, 6144, 32, 8, 100, FAKE, FAKE, None) == _lib.FP8Q_ERR_SHAPE     # D % 8
+    assert f(FAKE, 8, 6000, 32, 8, 128, FAKE, FAKE, None) == _lib.FP8Q_ERR_SHAPE     # ld
+    assert f(FAKE, 8, 6144, 32, 8, 128, None, FAKE, None) == _lib.FP8Q_ERR_NULL
+    assert f(FAKE, 8, 6148, 32, 8, 128, FAKE, FAKE, None) == _lib.FP8Q_ERR_ALIGN     # ld % 8
+    w = L.fp8q_kv_cache_write
+    ok = dict(x=FAKE, T=8, ld=6144, Hq=32, Hkv=8, D=128, slots=FAKE, ns=64, s=FAKE, q=FAKE,
+              ldq=4096, k=FAKE, v=FAKE)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return w(a["x"], a["T"], a["ld"], a["Hq"], a["Hkv"], a["D"], a["slots"], a["ns"], a["s"],
+                 a["q"], a["ldq"], a["k"], a["v"], None)
+    assert call(D=72, ld=72 * 48, ldq=72 * 32) == _lib.FP8Q_ERR_SHAPE            # D % 16
+    assert call(ldq=4000) == _lib.FP8Q_ERR_SHAPE
+    assert call(ns=-1) == _lib.FP8Q_ERR_SHAPE
+    assert call(slots=None) == _lib.FP8Q_ERR_NULL
+    assert call(k=None) == _lib.FP8Q_ERR_NULL
+    assert call(slots=FAKE + 4) == _lib.FP8Q_ERR_ALIGN
+    assert call(q=FAKE + 4) == _lib.FP8Q_ERR_ALIGN
+    assert call(T=0, x=None, slots=None, s=None, q=None, k=None, v=None) == _lib.FP8Q_OK
