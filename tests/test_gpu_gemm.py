@@ -81,6 +81,18 @@ def test_single_nonzero_k_block():
     _run_dense(aq, sa, wq, sw, 0)
 
 
+@pytest.mark.parametrize("M,N,K,fmt", [(1000, 9600, 512, oracle.SCALE_F32),
+                                       (300, 10240, 256, oracle.SCALE_E8M0),
+                                       (512, 19200, 384, oracle.SCALE_F32)])
+def test_many_tiles_ragged(M, N, K, fmt):
+    """More tiles than SMs (several tiles per persistent CTA), M not a multiple of 128 or 256 and N
+    ending in a half 256-column tile, both scale formats."""
+    a = inputs.randn_bf16((M, K), 1.0, 42, M + N + K)
+    w = inputs.randn_bf16((N, K), 0.02, 43, M + N + K)
+    rows = sorted({0, 127, 128, 255, 256, M // 2, M - 1})
+    _run_dense(*_quantize(a, w, fmt, lds=(M + 7) // 8 * 8), fmt, rows=rows, pad=8)
+
+
 def test_decode_full_size_sampled_rows():
     d = inputs.decode_linear()
     aq, sa, wq, sw = _quantize(d["A"], d["W"], 0)
