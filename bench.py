@@ -233,7 +233,22 @@ def measure_rows(fq, device, steps, warmup, pk):
                       "frac": byts / ms / 1e6 / hbm, "launches": len(ws),
                       "workload": "36 layers x {q,k,v,o,gate,up,down}, 6.946 G bf16 weights"}
         del ss
-    del ws, qs
+    del qs
+    torch.cuda.empty_cache()
+    # the same sweep as one batched launch over all 252 weights
+    for fmt, name in (("f32", "a1_requant_sweep_f32_batched"),
+                      ("e8m0", "a2_requant_sweep_e8m0_batched")):
+        batch = fq.WeightBatch(ws, fmt)
+        sbytes = sum(s.numel() * s.element_size() for s in batch.s)
+        ms, _ = timed_loop(batch.run, max(3, steps // 4), max(1, warmup // 2))
+        byts = elems * 3 + sbytes
+        rows[name] = {"ms": ms, "bytes": byts, "GB/s": byts / ms / 1e6,
+                      "frac": byts / ms / 1e6 / hbm, "launches": 1,
+                      "workload": "36 layers x {q,k,v,o,gate,up,down}, 6.946 G bf16 weights, "
+                                  "one launch"}
+        del batch
+        torch.cuda.empty_cache()
+    del ws
     torch.cuda.empty_cache()
 
     # decode: token quant of A [128, 4096] and GEMM with W [12288, 4096]

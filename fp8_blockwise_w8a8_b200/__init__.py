@@ -12,6 +12,7 @@ library or a non-sm_100 device raises.
     gemm_w8a8_block_splitk(aq, sa, wq, sw, ...) -> bf16 [M, N], K split over CTAs (small M)
     grouped_gemm_w8a8_block(aq, sa, wq, sw, offsets, fmt) -> bf16 [M, N]
 """
+import numpy as np
 import torch
 
 from . import _lib
@@ -24,7 +25,7 @@ import ctypes
 __all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
            "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant", "inverse_rope_quant",
-           "gemm_w8a8_block_diag", "gemm_w8a8_mx", "qkv_scales", "kv_cache_write",
+           "gemm_w8a8_block_diag", "gemm_w8a8_mx", "qkv_scales", "kv_cache_write", "WeightBatch",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -64,6 +65,44 @@ def quant_weight_block(w: torch.Tensor, fmt="f32", out_q=None, out_s=None, strea
                                             _stream(stream))
     _lib.check(st, "fp8q_quant_weight_block")
     return q, s
+
+
+class WeightBatch:
+    """A fixed list of bf16 weights [N_i, K_i] requantized together in one launch
+    (fp8q_quant_weight_block_batched).  Builds the output codes and scales once and a device
+    table of descriptors; run() requantizes every weight into them (e.g. once per step, after
+    the weights changed in place)."""
+
+    _DESC = np.dtype([("w", "<u8"), ("q", "<u8"), ("s", "<u8"), ("N", "<i8"), ("K", "<i8"),
+                      ("ldw", "<i8"), ("ldq", "<i8"), ("off", "<i8")])
+
+    def __init__(self, weights, fmt="f32"):
+        self.fmt = scale_format(fmt)
+        self.weights = list(weights)
+        if not self.weights:
+            raise ValueError("empty weight list")
+        dev = self.weights[0].device
+        sdt = torch.float32 if self.fmt == FP8Q_SCALE_F32 else torch.uint8
+        self.q, self.s = [], []
+        desc = np.zeros(len(self.weights), self._DESC)
+        off = 0
+        for i, w in enumerate(self.weights):
+            N, K = w.shape
+            q = torch.empty((N, K), dtype=torch.uint8, device=dev)
+            sc = torch.empty((N // 128, K // 128), dtype=sdt, device=dev)
+            self.q.append(q)
+            self.s.append(sc)
+            desc[i] = (w.data_ptr(), q.data_ptr(), sc.data_ptr(), N, K, _ld(w), _ld(q), off)
+            off += (N // 128) * (K // 128)
+        self.total_blocks = off
+        self.desc = torch.from_numpy(desc.view(np.uint8).copy()).to(dev)
+
+    def run(self, stream=None):
+        st = _lib.lib().fp8q_quant_weight_block_batched(_ptr(self.desc), len(self.weights),
+                                                        self.total_blocks, self.fmt,
+                                                        _stream(stream))
+        _lib.check(st, "fp8q_quant_weight_block_batched")
+        return self.q, self.s
 
 
 def rmsnorm_quant_token(x: torch.Tensor, gamma=None, eps: float = 1e-6, lds=None, out_q=None,

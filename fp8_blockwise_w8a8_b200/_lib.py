@@ -48,6 +48,7 @@ SIGNATURES = {
     "fp8q_gemm_w8a8_mx": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I64, _I64, _I64, _I64, _P,
                                _I64, _P]),
     "fp8q_qkv_scales": (_I, [_P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P]),
+    "fp8q_quant_weight_block_batched": (_I, [_P, _I64, _I64, _I, _P]),
     "fp8q_kv_cache_write": (_I, [_P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _P, _P, _I64, _P, _P,
                                  _P]),
     "fp8q_quant_rowwise": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P, _P]),

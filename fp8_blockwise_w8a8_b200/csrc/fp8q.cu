@@ -268,6 +268,31 @@ int fp8q_quant_weight_block(const void *w_bf16, int64_t N, int64_t K, int64_t ld
   return launch_status();
 }
 
+static_assert(sizeof(fp8q_weight_desc) == sizeof(fp8q::WeightDesc),
+              "fp8q_weight_desc and the kernel's descriptor must match");
+
+int fp8q_quant_weight_block_batched(const fp8q_weight_desc *descs, int64_t count,
+                                    int64_t total_blocks, int sw_fmt, cudaStream_t stream) {
+  if (sw_fmt != FP8Q_SCALE_F32 && sw_fmt != FP8Q_SCALE_E8M0) return FP8Q_ERR_ARG;
+  if (count < 0 || count > fp8q::kMaxBatchMatrices || total_blocks < 0) return FP8Q_ERR_SHAPE;
+  if (count == 0 || total_blocks == 0) return FP8Q_OK;
+  if (!descs) return FP8Q_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(descs) & 7u) return FP8Q_ERR_ALIGN;
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  const int64_t cap = static_cast<int64_t>(st->sms) * 4;
+  const int grid = static_cast<int>(total_blocks < cap ? total_blocks : cap);
+  const auto *d = reinterpret_cast<const fp8q::WeightDesc *>(descs);
+  if (sw_fmt == FP8Q_SCALE_F32)
+    fp8q::k_quant_weight_block_batched<fp8q::kScaleF32><<<grid, 256, 0, stream>>>(
+        d, static_cast<int>(count), total_blocks);
+  else
+    fp8q::k_quant_weight_block_batched<fp8q::kScaleE8M0><<<grid, 256, 0, stream>>>(
+        d, static_cast<int>(count), total_blocks);
+  return launch_status();
+}
+
 int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
                              int64_t K, int64_t ldx, void *xq_e4m3, int64_t ldq, float *sa,
                              int64_t lds, cudaStream_t stream) {

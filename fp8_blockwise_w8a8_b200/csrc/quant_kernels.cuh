@@ -170,6 +170,50 @@ __device__ __forceinline__ uint2 quant8_pow2(const uint4 v, const float2 inv2) {
 // chunk (t % 16) of rows (t / 16) + 16 i, i = 0..7, so every load and store instruction of a
 // warp covers two full 256-byte (load) / 128-byte (store) row segments.
 // ---------------------------------------------------------------------------------------------
+// One 128x128 block: quantize w[128][ldw] (the block's top-left element) into q[128][ldq] and write
+// its scale to *scale (fp32 or one E8M0 byte).  All 256 threads of the CTA take part; red is 8
+// floats of shared memory.
+template <int FMT>
+__device__ __forceinline__ void quant_weight_one_block(const uint16_t *__restrict__ w, int64_t ldw,
+                                                       uint8_t *__restrict__ q, int64_t ldq,
+                                                       void *scale, float *red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r0 = tid >> 4;
+  const int c8 = (tid & 15) * 8;
+  const uint16_t *src = w + r0 * ldw + c8;
+  uint4 v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = ld_stream_v4(src + static_cast<int64_t>(i) * 16 * ldw);
+  uint32_t m2 = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m2 = absmax_uint4(m2, v[i]);
+  float amax = absmax_finish(m2);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) amax = fmaxf(amax, red[i]);
+  __syncthreads();  // red[] is rewritten by the next block
+  uint8_t *dst = q + r0 * ldq + c8;
+  if (FMT == kScaleF32) {
+    const QParams p = qparams_f32(amax);
+    if (tid == 0) *static_cast<float *>(scale) = p.s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<uint2 *>(dst + static_cast<int64_t>(i) * 16 * ldq) = quant8_f32(v[i], p);
+  } else {
+    const int e = e8m0_exponent(amax);
+    if (tid == 0) *static_cast<uint8_t *>(scale) = static_cast<uint8_t>(e + 127);
+    const float inv = pow2_f32(-e);
+    const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<uint2 *>(dst + static_cast<int64_t>(i) * 16 * ldq) = quant8_pow2(v[i], inv2);
+  }
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(256, 4) k_quant_weight_block(const uint16_t *__restrict__ w,
                                                             int64_t ldw, uint8_t *__restrict__ q,
@@ -213,6 +257,53 @@ __global__ void __launch_bounds__(256, 4) k_quant_weight_block(const uint16_t *_
       for (int i = 0; i < 8; ++i)
         *reinterpret_cast<uint2 *>(dst + static_cast<int64_t>(i) * 16 * ldq) = quant8_pow2(v[i], inv2);
     }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// All the weights of a step in one launch.  Matrix i of the batch owns the blocks
+// [block_offset_i, block_offset_{i+1}) of one global numbering; persistent CTAs walk that
+// numbering with a stride of the grid, keeping the current matrix (the offsets are held in shared
+// memory and only ever move forward).  A descriptor that breaks the shape or alignment rules, or a
+// block outside its matrix, records FP8Q_ERR_SHAPE and is skipped.
+// ---------------------------------------------------------------------------------------------
+struct WeightDesc {
+  const uint16_t *w;
+  uint8_t *q;
+  void *s;
+  int64_t N, K, ldw, ldq, block_offset;
+};
+constexpr int kMaxBatchMatrices = 2048;
+constexpr int kErrShapeDev = 2;  // FP8Q_ERR_SHAPE
+
+template <int FMT>
+__global__ void __launch_bounds__(256, 4) k_quant_weight_block_batched(
+    const WeightDesc *__restrict__ d, int count, int64_t total) {
+  __shared__ float red[8];
+  __shared__ int64_t s_off[kMaxBatchMatrices + 1];
+  for (int i = threadIdx.x; i < count; i += blockDim.x) s_off[i] = d[i].block_offset;
+  if (threadIdx.x == 0) s_off[count] = total;
+  __syncthreads();
+  int cur = 0;
+  for (int64_t g = blockIdx.x; g < total; g += gridDim.x) {
+    while (cur + 1 < count && g >= s_off[cur + 1]) ++cur;
+    const WeightDesc md = d[cur];
+    const int64_t local = g - s_off[cur];
+    const bool shape_ok = md.N > 0 && md.K > 0 && md.N % 128 == 0 && md.K % 128 == 0 &&
+                          md.ldw >= md.K && md.ldq >= md.K && md.ldw % 8 == 0 && md.ldq % 16 == 0 &&
+                          (reinterpret_cast<uintptr_t>(md.w) & 15u) == 0 &&
+                          (reinterpret_cast<uintptr_t>(md.q) & 15u) == 0 && md.s != nullptr &&
+                          (FMT != kScaleF32 || (reinterpret_cast<uintptr_t>(md.s) & 3u) == 0);
+    const int64_t KB = md.K / 128;
+    if (!shape_ok || local < 0 || local >= (md.N / 128) * KB) {
+      if (threadIdx.x == 0) record_error(kErrShapeDev);
+      continue;
+    }
+    const int64_t nb = local / KB, kb = local - nb * KB;
+    void *scale = FMT == kScaleF32 ? static_cast<void *>(static_cast<float *>(md.s) + local)
+                                   : static_cast<void *>(static_cast<uint8_t *>(md.s) + local);
+    quant_weight_one_block<FMT>(md.w + nb * 128 * md.ldw + kb * 128, md.ldw,
+                                md.q + nb * 128 * md.ldq + kb * 128, md.ldq, scale, red);
   }
 }
 

@@ -87,6 +87,28 @@ int fp8q_quant_weight_block(const void *w_bf16, int64_t N, int64_t K, int64_t ld
                             void *wq_e4m3, int64_t ldq, void *sw, int sw_fmt,
                             cudaStream_t stream);
 
+/* One matrix of a batched weight requantization (fp8q_quant_weight_block_batched): the arguments
+ * of fp8q_quant_weight_block for that matrix, plus the index of its first 128x128 block in the
+ * batch's block numbering (the sum of (N/128)(K/128) over the matrices before it). */
+typedef struct {
+  const void *w;          /* bf16 [N][ldw], read */
+  void *q;                /* uint8 [N][ldq], written */
+  void *s;                /* [N/128][K/128] fp32 or E8M0 scales, written */
+  int64_t N, K, ldw, ldq; /* as fp8q_quant_weight_block */
+  int64_t block_offset;   /* first block of this matrix in the batch numbering */
+} fp8q_weight_desc;
+
+/* Batched a1 / a2: every matrix of `descs` (DEVICE memory, count <= 2048, block_offset ascending,
+ * total_blocks = the sum of all matrices' blocks) requantized in one launch, with the arithmetic
+ * and outputs of fp8q_quant_weight_block.  The descriptors are read on the device: one that
+ * breaks that call's shape or alignment rules (or block numbering that does not match the
+ * matrices) records FP8Q_ERR_SHAPE in the device error word and its blocks are skipped.
+ * Source: FP8-RL abstract, item (i) (the policy's weights change every step, so all of them are
+ * requantized every step). */
+int fp8q_quant_weight_block_batched(const fp8q_weight_desc *descs, int64_t count,
+                                    int64_t total_blocks, int sw_fmt, cudaStream_t stream);
+
+
 /* Per-token 1x128 activation quantization, optionally fused with RMSNorm (a3 / a4).
  *   x_bf16      [M][ldx] bf16, read
  *   gamma_bf16  [K] bf16 RMSNorm weight, or NULL for plain token quant (no normalisation)

@@ -259,3 +259,13 @@ def test_kv_cache_host_checks(L):
     assert call(slots=FAKE + 4) == _lib.FP8Q_ERR_ALIGN
     assert call(q=FAKE + 4) == _lib.FP8Q_ERR_ALIGN
     assert call(T=0, x=None, slots=None, s=None, q=None, k=None, v=None) == _lib.FP8Q_OK
+
+
+def test_weight_batch_host_checks(L):
+    f = L.fp8q_quant_weight_block_batched
+    assert f(FAKE, 3, 100, 5, None) == _lib.FP8Q_ERR_ARG
+    assert f(FAKE, 4096, 100, 0, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(FAKE, 3, -1, 0, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(None, 3, 100, 0, None) == _lib.FP8Q_ERR_NULL
+    assert f(FAKE + 4, 3, 100, 0, None) == _lib.FP8Q_ERR_ALIGN
+    assert f(None, 0, 0, 1, None) == _lib.FP8Q_OK

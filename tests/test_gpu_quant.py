@@ -183,3 +183,48 @@ def test_token_strided_rows():
                                                    lds=sa.shape[1])
         assert np.array_equal(q.cpu().numpy(), q_ref)
         assert np.array_equal(sa.cpu().numpy()[:, :M], sa_ref[:, :M])
+
+
+# --- batched requant ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [oracle.SCALE_F32, oracle.SCALE_E8M0])
+def test_weight_batch_mixed_shapes(fmt):
+    shapes = [(128, 128), (256, 384), (1024, 4096), (384, 128), (4096, 512), (128, 1152)]
+    ws = [inputs.randn_bf16(s, 0.02 * (i + 1), 95, i) for i, s in enumerate(shapes)]
+    ws[2] = np.concatenate([ws[2], np.zeros((1024, 64), np.uint16)], axis=1)   # strided rows
+    dev = [dev_bf16(w) for w in ws]
+    dev[2] = dev[2][:, :4096]
+    batch = fq.WeightBatch(dev, fmt)
+    qs, ss = batch.run()
+    assert fq.check_device_error() == 0
+    for w, q, s_ in zip(ws, qs, ss):
+        N, K = q.shape
+        q_ref, s_ref = oracle.quant_weight_block(np.ascontiguousarray(w[:, :K]), fmt)
+        assert np.array_equal(q.cpu().numpy(), q_ref)
+        assert np.array_equal(s_.cpu().numpy(), s_ref)
+
+
+def test_weight_batch_sweep_layer_matches_per_matrix_calls():
+    ws = [inputs.sweep_matrix(0, i, "cuda") for i in range(len(inputs.SWEEP_MATRICES))]
+    for fmt in ("f32", "e8m0"):
+        qs, ss = fq.WeightBatch(ws, fmt).run()
+        assert fq.check_device_error() == 0
+        for w, q, s_ in zip(ws, qs, ss):
+            q1, s1 = fq.quant_weight_block(w, fmt)
+            assert torch.equal(q, q1) and torch.equal(s_, s1)
+
+
+def test_weight_batch_bad_descriptor_is_reported_and_skipped():
+    ws = [dev_bf16(inputs.randn_bf16((256, 256), 0.02, 96, i)) for i in range(3)]
+    batch = fq.WeightBatch(ws, "f32")
+    desc = batch.desc.cpu().numpy().view(fq.WeightBatch._DESC).copy()
+    desc[1]["K"] = 200                       # not a multiple of 128
+    batch.desc = torch.from_numpy(desc.view(np.uint8).copy()).cuda()
+    for q in batch.q:
+        q.fill_(0xEE)
+    qs, ss = batch.run()
+    assert fq.check_device_error() == fq.FP8Q_ERR_SHAPE
+    assert (qs[1] == 0xEE).all()
+    for i in (0, 2):
+        q_ref, s_ref = oracle.quant_weight_block(ws[i].cpu().view(torch.int16).numpy().view(np.uint16), 0)
+        assert np.array_equal(qs[i].cpu().numpy(), q_ref) and np.array_equal(ss[i].cpu().numpy(), s_ref)
