@@ -1057,18 +1057,29 @@ __global__ void __launch_bounds__(kReduceThreads)
   if (row >= M || col >= N) return;
   const int h = g >> 3, c0 = (g & 7) * 4;
   const float4 *p = ws + static_cast<size_t>(t) * splits * (2 * 32 * 128) + (h * 32 + c0) * 128 + r;
+  // The partials of up to four splits are loaded together, then added in split order.
   float4 sum[4];
+  for (int j0 = 0; j0 < splits; j0 += 4) {
+    float4 v[4][4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) sum[i] = __ldcg(p + i * 128);
-  for (int j = 1; j < splits; ++j) {
-    const float4 *pj = p + static_cast<size_t>(j) * (2 * 32 * 128);
-    float4 v[4];
+    for (int jj = 0; jj < 4; ++jj) {
+      if (j0 + jj < splits) {
+        const float4 *pj = p + static_cast<size_t>(j0 + jj) * (2 * 32 * 128);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = __ldcg(pj + i * 128);
+        for (int i = 0; i < 4; ++i) v[jj][i] = __ldcg(pj + i * 128);
+      }
+    }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      sum[i] = make_float4(__fadd_rn(sum[i].x, v[i].x), __fadd_rn(sum[i].y, v[i].y),
-                           __fadd_rn(sum[i].z, v[i].z), __fadd_rn(sum[i].w, v[i].w));
+    for (int jj = 0; jj < 4; ++jj) {
+      if (j0 + jj < splits) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          sum[i] = j0 + jj == 0
+                       ? v[jj][i]
+                       : make_float4(__fadd_rn(sum[i].x, v[jj][i].x), __fadd_rn(sum[i].y, v[jj][i].y),
+                                     __fadd_rn(sum[i].z, v[jj][i].z), __fadd_rn(sum[i].w, v[jj][i].w));
+      }
+    }
   }
   uint32_t pk[8];
 #pragma unroll
