@@ -25,7 +25,7 @@ import ctypes
 __all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
            "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant", "inverse_rope_quant",
-           "gemm_w8a8_block_diag", "gemm_w8a8_mx", "qkv_scales", "kv_cache_write", "WeightBatch",
+           "gemm_w8a8_block_diag", "gemm_w8a8_mx", "qkv_scales", "kv_cache_write", "WeightBatch", "selftest_timeout",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -347,6 +347,13 @@ def gemm_w8a8_rowwise(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, sw: 
                                            _ptr(sw), M, N, K, _ptr(o), _ld(o), _stream(stream))
     _lib.check(st, "fp8q_gemm_w8a8_rowwise")
     return o
+
+
+def selftest_timeout(limit_ns: int = 1_000_000, stream=None):
+    """Launch the bounded-wait self-test kernel (a wait that nothing completes, given up after
+    limit_ns); fp8q_check_device_error then reports FP8Q_ERR_TIMEOUT."""
+    st = _lib.lib().fp8q_selftest_timeout(int(limit_ns), _stream(stream))
+    _lib.check(st, "fp8q_selftest_timeout")
 
 
 def check_device_error(stream=None) -> int:

@@ -726,6 +726,15 @@ int fp8q_gemm_w8a8_mx(const void *aq, int64_t lda, const float *sa, int64_t lds,
   return launch_status();
 }
 
+int fp8q_selftest_timeout(int64_t limit_ns, cudaStream_t stream) {
+  if (limit_ns <= 0 || limit_ns > 100000000) return FP8Q_ERR_ARG;  // (0, 100 ms]
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  fp8q::k_selftest_timeout<<<1, 128, 0, stream>>>(static_cast<uint64_t>(limit_ns));
+  return launch_status();
+}
+
 int fp8q_check_device_error(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return FP8Q_ERR_LAUNCH;
   int v = 0;

@@ -289,14 +289,15 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[64]) {
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
 
 // Bounded wait by one thread.  Returns false on abort (another role gave up) or timeout.
-__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                         uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         record_error(6 /* FP8Q_ERR_TIMEOUT */);
         return false;
@@ -306,7 +307,8 @@ __device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile
 }
 
 // Bounded wait by a whole warp with a warp-uniform outcome.
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const int lane = threadIdx.x & 31;
   uint64_t t0 = 0;
   for (uint32_t n = 0;; ++n) {
@@ -319,7 +321,7 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
         if (t0 == 0) t0 = now;
         if (*abort_flag) {
           stop = 1;
-        } else if (now - t0 > kWaitLimitNs) {
+        } else if (now - t0 > limit_ns) {
           *abort_flag = 1;
           record_error(6 /* FP8Q_ERR_TIMEOUT */);
           stop = 1;

@@ -998,4 +998,47 @@ __global__ void __launch_bounds__(kKvThreads) k_kv_cache_write(
   }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Self-test of the bounded-wait teardown: the GEMM kernels' roles and helpers, run against a
+// barrier that nothing ever arrives on.  Warp 1 allocates TMEM; thread 0 waits on the barrier
+// with a short limit, gives up, records FP8Q_ERR_TIMEOUT and raises the abort flag; warps 2-3
+// wait (warp-wide) on another barrier that nothing arrives on and leave on the abort flag; TMEM
+// is released and the kernel returns.  No fault, no trap: the context stays usable.
+// ---------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(128, 1) k_selftest_timeout(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort_store;
+  volatile int *s_abort = &s_abort_store;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t b0 = smem_u32(&bars[0]), b1 = smem_u32(&bars[1]);
+  if (threadIdx.x == 0) {
+    mbar_init(b0, 1);
+    mbar_init(b1, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&s_tmem), 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = s_tmem;
+  if (warp == 0) {
+    if (lane == 0) wait_one(b0, 0, s_abort, limit_ns);   // never completes: times out
+    __syncwarp();
+  } else if (warp >= 2) {
+    // a longer limit: these warps leave because of the abort flag, not their own limit
+    wait_warp(b1, 0, s_abort, 10 * limit_ns);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 32);
+  }
+}
+
 }  // namespace fp8q

@@ -347,6 +347,13 @@ int fp8q_gemm_w8a8_rowwise(const void *aq, int64_t lda, const float *sa, const v
                            int64_t ldw, const float *sw, int64_t M, int64_t N, int64_t K,
                            void *out_bf16, int64_t ldo, cudaStream_t stream);
 
+/* Self-test of the bounded-wait path: launches one small kernel that allocates TMEM, waits on a
+ * barrier nothing arrives on with the limit limit_ns (0 < limit_ns <= 100 ms), gives up, records
+ * FP8Q_ERR_TIMEOUT in the device error word, stops its other warps through the abort flag and
+ * releases TMEM, as the GEMM kernels do on a timeout.  A following fp8q_check_device_error
+ * returns FP8Q_ERR_TIMEOUT; the context stays usable.  For tests. */
+int fp8q_selftest_timeout(int64_t limit_ns, cudaStream_t stream);
+
 /* Synchronize `stream`, then read and clear the device error word of the current device.
  * Returns FP8Q_OK, FP8Q_ERR_TIMEOUT (a kernel gave up on a bounded wait since the last call;
  * its outputs are incomplete) or FP8Q_ERR_LAUNCH (the synchronize failed). */

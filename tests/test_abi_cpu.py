@@ -269,3 +269,12 @@ def test_weight_batch_host_checks(L):
     assert f(None, 3, 100, 0, None) == _lib.FP8Q_ERR_NULL
     assert f(FAKE + 4, 3, 100, 0, None) == _lib.FP8Q_ERR_ALIGN
     assert f(None, 0, 0, 1, None) == _lib.FP8Q_OK
+
+
+def test_selftest_timeout_host_checks(L):
+    f = L.fp8q_selftest_timeout
+    assert f(0, None) == _lib.FP8Q_ERR_ARG
+    assert f(200_000_000, None) == _lib.FP8Q_ERR_ARG
+    import torch
+    if not torch.cuda.is_available():
+        assert f(1_000_000, None) == _lib.FP8Q_ERR_ARCH
