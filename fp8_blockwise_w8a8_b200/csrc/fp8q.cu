@@ -52,12 +52,18 @@ int device_state(DeviceState **out) {
   }
   if (!st.is_sm100) return FP8Q_ERR_ARCH;
   if (!st.attrs_set) {
-    if (cudaFuncSetAttribute(fp8q::k_gemm_w8a8_block<false>,
+    if (cudaFuncSetAttribute(fp8q::k_gemm_w8a8_block<false, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fp8q::kGemmSmemDense) != cudaSuccess ||
-        cudaFuncSetAttribute(fp8q::k_gemm_w8a8_block<true>,
+        cudaFuncSetAttribute(fp8q::k_gemm_w8a8_block<true, false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fp8q::kGemmSmemGrouped) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_gemm_w8a8_block<false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fp8q::BlockLayout<true>::smemDense) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_gemm_w8a8_block<true, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             fp8q::BlockLayout<true>::smemGrouped) != cudaSuccess ||
         cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
             cudaSuccess ||
@@ -107,6 +113,19 @@ int make_u8_map(CUtensorMap *map, const void *base, int64_t rows, int64_t cols, 
                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_LAUNCH;
+}
+
+// 2-D bf16 tensor map over a row-major [rows][ld] output, box = 32 rows x 64 columns (128 bytes),
+// 128-byte swizzle: the tile-store target of the block GEMM.
+int make_bf16_out_map(CUtensorMap *map, void *base, int64_t rows, int64_t cols, int64_t ld) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld * 2)};
+  const cuuint32_t box[2] = {64, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FP8Q_OK : FP8Q_ERR_LAUNCH;
 }
 
@@ -204,12 +223,26 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
   const int64_t tiles = (static_cast<int64_t>(a.num_m) + (grouped ? E : 0)) * a.num_n;
   const int64_t units = tiles * splits;
   const int grid = static_cast<int>(units < st->sms ? units : st->sms);
-  if (grouped)
-    fp8q::k_gemm_w8a8_block<true><<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemGrouped, stream>>>(
-        tm_a, tm_b, a);
+  // Tile stores by TMA when a CTA runs several tiles (the store then overlaps the next tile); one
+  // tile per CTA keeps the deeper 4-stage operand ring instead.
+  const bool ts = splits == 1 && tiles > st->sms;
+  CUtensorMap tm_out;
+  if (ts && (rc = make_bf16_out_map(&tm_out, out, M, N, ldo)) != FP8Q_OK) return rc;
+  if (!ts) tm_out = tm_a;  // unused
+  if (grouped && ts)
+    fp8q::k_gemm_w8a8_block<true, true><<<grid, fp8q::kGemmThreads,
+                                          fp8q::BlockLayout<true>::smemGrouped, stream>>>(
+        tm_a, tm_b, tm_out, a);
+  else if (grouped)
+    fp8q::k_gemm_w8a8_block<true, false><<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemGrouped,
+                                           stream>>>(tm_a, tm_b, tm_out, a);
+  else if (ts)
+    fp8q::k_gemm_w8a8_block<false, true><<<grid, fp8q::kGemmThreads,
+                                           fp8q::BlockLayout<true>::smemDense, stream>>>(
+        tm_a, tm_b, tm_out, a);
   else
-    fp8q::k_gemm_w8a8_block<false><<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemDense, stream>>>(
-        tm_a, tm_b, a);
+    fp8q::k_gemm_w8a8_block<false, false><<<grid, fp8q::kGemmThreads, fp8q::kGemmSmemDense,
+                                            stream>>>(tm_a, tm_b, tm_out, a);
   if (splits > 1 && !grouped) {
     if ((rc = launch_status()) != FP8Q_OK) return rc;
     fp8q::k_splitk_reduce<<<static_cast<unsigned>(tiles * 8), fp8q::kReduceThreads, 0, stream>>>(

@@ -63,6 +63,27 @@ constexpr int kOffGroups = kOffMisc + 16;          // grouped: offsets[E+1], til
 constexpr int kGemmSmemDense = kOffGroups + 1024;  // + alignment slack
 constexpr int kGemmSmemGrouped = kOffGroups + 2 * (kMaxExperts + 1) * 4 + 1024;
 
+// Shared-memory layout of k_gemm_w8a8_block.  With TS (tile stores by TMA) the operand ring has 3
+// stages and each epilogue warp a whole 8 KB output slot (its 32 rows x 128 columns of bf16), so
+// a finished tile leaves through the TMA engine while the warps promote the next one.
+template <bool TS> struct BlockLayout {
+  static constexpr int stages = TS ? 3 : kStages;
+  static constexpr int offA = 0;
+  static constexpr int offB = offA + stages * kTileABytes;
+  static constexpr int offStaging = offB + stages * kTileBBytes;
+  static constexpr int stagingPerWarp = TS ? 8192 : kStagingBytesPerWarp;
+  static constexpr int offSa = offStaging + 8 * stagingPerWarp;
+  static constexpr int offSw = offSa + kSaStages * kBM * 4;
+  static constexpr int offBar = offSw + 2 * 2 * kMaxKB * 4;
+  static constexpr int numBars = 2 * stages + 4 + 1 + 2 * kSaStages + 4;
+  static constexpr int offMisc = offBar + numBars * 8;
+  static constexpr int offGroups = offMisc + 16;
+  static constexpr int smemDense = offGroups + 1024;
+  static constexpr int smemGrouped = offGroups + 2 * (kMaxExperts + 1) * 4 + 1024;
+};
+static_assert(BlockLayout<true>::smemGrouped <= 227 * 1024, "TMA-store layout exceeds shared memory");
+static_assert(BlockLayout<false>::smemGrouped == kGemmSmemGrouped, "layouts differ");
+
 // Instruction descriptor, kind::f8f6f4: D fp32 (bits 4-5 = 1), A and B E4M3 (bits 7-9, 10-12
 // = 0), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
 constexpr uint32_t kIdesc = (1u << 4) | (static_cast<uint32_t>(kBN >> 3) << 17) |
@@ -232,35 +253,37 @@ __device__ __forceinline__ void store_chunk32(const float2 (&v)[16], uint32_t st
   store_packed32(pk, stage_u32, lane, out_base, tl, q, c4, col_ok, ldo);
 }
 
-template <bool GROUPED>
+template <bool GROUPED, bool TS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm_w8a8_block(const __grid_constant__ CUtensorMap tm_a,
-                      const __grid_constant__ CUtensorMap tm_b, const GemmArgs args) {
+                      const __grid_constant__ CUtensorMap tm_b,
+                      const __grid_constant__ CUtensorMap tm_out, const GemmArgs args) {
+  using L = BlockLayout<TS>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar_full = sbase + kOffBar;              // [kStages]
-  const uint32_t bar_empty = bar_full + 8 * kStages;      // [kStages]
-  const uint32_t bar_tfull = bar_empty + 8 * kStages;     // [2]
+  const uint32_t bar_full = sbase + L::offBar;              // [L::stages]
+  const uint32_t bar_empty = bar_full + 8 * L::stages;      // [L::stages]
+  const uint32_t bar_tfull = bar_empty + 8 * L::stages;     // [2]
   const uint32_t bar_tempty = bar_tfull + 16;             // [2]
   const uint32_t bar_done = bar_tempty + 16;
   const uint32_t bar_safull = bar_done + 8;                   // [kSaStages]
   const uint32_t bar_saempty = bar_safull + 8 * kSaStages;    // [kSaStages]
   const uint32_t bar_swfull = bar_saempty + 8 * kSaStages;    // [2]
   const uint32_t bar_swempty = bar_swfull + 16;               // [2]
-  float *s_sa = reinterpret_cast<float *>(smem + kOffSa);
-  float *s_sw = reinterpret_cast<float *>(smem + kOffSw);
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + kOffMisc);
-  volatile int *s_abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
-  int *s_off = reinterpret_cast<int *>(smem + kOffGroups);
+  float *s_sa = reinterpret_cast<float *>(smem + L::offSa);
+  float *s_sw = reinterpret_cast<float *>(smem + L::offSw);
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(smem + L::offMisc);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(smem + L::offMisc + 4);
+  int *s_off = reinterpret_cast<int *>(smem + L::offGroups);
   int *s_prefix = s_off + (kMaxExperts + 1);
 
   const int KB = args.K / kBK;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < L::stages; ++i) {
       mbar_init(bar_full + 8 * i, 1);
       mbar_init(bar_empty + 8 * i, 1);
     }
@@ -325,20 +348,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const Tile tl = GROUPED ? grouped_tile(args, s_off, s_prefix, un.t) : dense_tile(args, un.t);
           bool ok = true;
           for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
-            const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            const uint32_t s = it % L::stages, ph = (it / L::stages) & 1u;
             if (!wait_one(bar_empty + 8 * s, ph ^ 1u, s_abort)) { ok = false; break; }
             mbar_arrive_expect_tx(bar_full + 8 * s, kStageBytes);
-            tma_load_2d(sbase + kOffA + s * kTileABytes, &tm_a, (tl.a_kb + kb) * kBK, tl.m0,
+            tma_load_2d(sbase + L::offA + s * kTileABytes, &tm_a, (tl.a_kb + kb) * kBK, tl.m0,
                         bar_full + 8 * s);
-            tma_load_2d(sbase + kOffB + s * kTileBBytes, &tm_b, kb * kBK, tl.b_row,
+            tma_load_2d(sbase + L::offB + s * kTileBBytes, &tm_b, kb * kBK, tl.b_row,
                         bar_full + 8 * s);
           }
           if (!ok) break;
         }
         // Drain: every issued load has landed before the CTA can exit.
-        for (uint32_t s = 0; s < kStages && s < it; ++s) {
-          const uint32_t last = s + ((it - 1 - s) / kStages) * kStages;  // last fill of stage s
-          wait_drain(bar_full + 8 * s, (last / kStages) & 1u);
+        for (uint32_t s = 0; s < L::stages && s < it; ++s) {
+          const uint32_t last = s + ((it - 1 - s) / L::stages) * L::stages;  // last fill of stage s
+          wait_drain(bar_full + 8 * s, (last / L::stages) & 1u);
         }
       }
       __syncwarp();
@@ -400,13 +423,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           bool ok = true;
           for (int kb = un.kb0; kb < un.kb1; ++kb, ++it) {
             if ((it & 1u) != mine) continue;
-            const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            const uint32_t s = it % L::stages, ph = (it / L::stages) & 1u;
             const uint32_t b = it & 1u, bph = (it >> 1) & 1u;
             if (!wait_one(bar_tempty + 8 * b, bph ^ 1u, s_abort)) { ok = false; break; }
             if (!wait_one(bar_full + 8 * s, ph, s_abort)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t ad = sdesc_k128(sbase + kOffA + s * kTileABytes);
-            const uint64_t bd = sdesc_k128(sbase + kOffB + s * kTileBBytes);
+            const uint64_t ad = sdesc_k128(sbase + L::offA + s * kTileABytes);
+            const uint64_t bd = sdesc_k128(sbase + L::offB + s * kTileBBytes);
             const uint32_t d = tmem_base + b * kBN;
 #pragma unroll
             for (int kk = 0; kk < kBK / 32; ++kk)  // 32-byte steps inside the 128-byte row
@@ -428,7 +451,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;         // TMEM lane quarter = rows 32q .. 32q + 31 of the tile
     const int h = (warp - 4) >> 2;  // column half of the 256-wide tile
     const int NB = args.N / 128;
-    uint8_t *stage = smem + kOffStaging + (warp - 4) * kStagingBytesPerWarp;
+    uint8_t *stage = smem + L::offStaging + (warp - 4) * L::stagingPerWarp;
     const uint32_t stage_u32 = smem_u32(stage);
     uint32_t it = 0, tile_it = 0;
     bool ok = true;
@@ -520,10 +543,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                              acc[2 * c + 1].y));
         continue;
       }
+      if constexpr (TS) {
+        if (!GROUPED || tl.row_end >= tl.m0 + kBM) {
+          // The tile's bf16 rows go to this warp's slot as two 32 x 64 boxes (128-byte swizzle)
+          // and out through the TMA engine; the warp goes on to the next tile.
+          if (lane == 0) bulk_wait_read0();  // the slot's previous stores have read it
+          __syncwarp();
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[4 * cc + u].x, acc[4 * cc + u].y);
+              pk[u] = *reinterpret_cast<const uint32_t *>(&v2);
+            }
+            const uint32_t addr = stage_u32 + (cc >> 3) * 4096 + lane * 128 +
+                                  ((static_cast<uint32_t>(cc & 7) ^ static_cast<uint32_t>(lane & 7)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[0]),
+                         "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                         : "memory");
+          }
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) {
+            const int y = tl.m0 + 32 * q;
+#pragma unroll
+            for (int bx = 0; bx < 2; ++bx) {
+              const int x = tl.n0 + 128 * h + 64 * bx;
+              if (x < args.N && y < args.M) tma_store_2d(&tm_out, x, y, stage_u32 + bx * 4096);
+            }
+            bulk_commit();
+          }
+          continue;
+        }
+        if (lane == 0) bulk_wait_read0();  // the masked path below reuses the slot
+        __syncwarp();
+      }
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4)
         store_chunk32(*reinterpret_cast<const float2(*)[16]>(acc + 16 * c4), stage_u32, lane,
                       out_base, tl, q, c4, col_ok, args.ldo);
+    }
+    if constexpr (TS) {
+      if (lane == 0) bulk_wait0();  // every tile store of this warp has completed
+      __syncwarp();
     }
     tc_fence_before();
   }
