@@ -544,9 +544,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         continue;
       }
       if constexpr (TS) {
-        if (!GROUPED || tl.row_end >= tl.m0 + kBM) {
-          // The tile's bf16 rows go to this warp's slot as two 32 x 64 boxes (128-byte swizzle)
-          // and out through the TMA engine; the warp goes on to the next tile.
+        if (!GROUPED || tl.row_end >= tl.m0 + 32 * q + 32) {  // this warp's 32 rows are all in
+          // This warp's bf16 rows go to its slot as two 32 x 64 boxes (128-byte swizzle) and out
+          // through the TMA engine; the warp goes on to the next tile.  Grouped: a warp whose rows
+          // an expert's end cuts takes the masked path below.
           if (lane == 0) bulk_wait_read0();  // the slot's previous stores have read it
           __syncwarp();
 #pragma unroll
