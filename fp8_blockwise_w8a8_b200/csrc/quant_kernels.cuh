@@ -444,6 +444,53 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
   __syncthreads();
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
+  if (!NORM) {
+    // Plain 1x128 quant: the warp walks (row, step) units; the next unit's loads (of the same row
+    // or the warp's next row) are in flight while the current one is converted, so a new row
+    // starts without waiting for its data.
+    int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp;
+    int b0 = 0;
+    uint4 v0[CPL], v1[CPL];
+    auto load_unit = [&](int64_t mm, int bb0, uint4 (&dst)[CPL]) {
+      if (mm < M) {
+        const int bb = bb0 + grp < KB ? bb0 + grp : bb0;
+        const uint16_t *src = x + mm * ldx + bb * 128;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) dst[c] = ld_stream_v4(src + (sub + LPB * c) * 8);
+      }
+    };
+    load_unit(m, b0, v0);
+    while (m < M) {
+      int64_t m1 = m;
+      int b1 = b0 + BPS;
+      if (b1 >= KB) {
+        b1 = 0;
+        m1 += stride;
+      }
+      load_unit(m1, b1, v1);
+      const int b = b0 + grp;
+      const bool active = b < KB;
+      uint32_t mx = 0u;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) mx = absmax_uint4(mx, v0[c]);
+#pragma unroll
+      for (int o = LPB / 2; o > 0; o >>= 1)
+        mx = absmax_bf16x2(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const QParams p = qparams_tab(absmax_finish(mx), tab);
+      uint8_t *qb = q + m * ldq + b * 128;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        const uint2 codes = quant8_f32(v0[c], p);
+        if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
+      }
+      if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) v0[c] = v1[c];
+      m = m1;
+      b0 = b1;
+    }
+    return;
+  }
   for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < M; m += stride) {
     const uint16_t *xr = x + m * ldx;
     const int64_t next = m + stride;
