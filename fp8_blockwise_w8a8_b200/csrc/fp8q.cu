@@ -361,7 +361,9 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   }
   if (best_wpc == 0) return FP8Q_ERR_SHAPE;
   const int wpc = best_wpc, smem = best_smem;
-  const int64_t need = (M + wpc - 1) / wpc;
+  // the plain kernel spreads (row, step) units over the warps, the fused one whole rows
+  const int64_t units = norm ? M : M * ((K / 128 + 7) / 8);
+  const int64_t need = (units + wpc - 1) / wpc;
   const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
   const int grid = static_cast<int>(need < cap ? need : cap);
   const auto *x = static_cast<const uint16_t *>(x_bf16);
@@ -370,6 +372,9 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   if (norm)
     fp8q::k_rmsnorm_quant_token<true><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, lds);
+  else if (M < static_cast<int64_t>(grid) * wpc)  // fewer rows than warps: spread the steps
+    fp8q::k_rmsnorm_quant_token<false, true><<<grid, 32 * wpc, smem, stream>>>(
+        x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds);
   else
     fp8q::k_rmsnorm_quant_token<false><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds);

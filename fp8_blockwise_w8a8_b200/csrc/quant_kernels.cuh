@@ -416,7 +416,7 @@ __host__ __device__ constexpr int token_smem_bytes(int K, bool norm, int wpc) {
   return static_cast<int>(sizeof(ScaleTab)) + (norm ? K * 4 + wpc * (K / 128) * 8 : 0);
 }
 
-template <bool NORM>
+template <bool NORM, bool SPREAD = false>
 __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
     int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ sa, int64_t lds) {
@@ -445,11 +445,21 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
   if (!NORM) {
-    // Plain 1x128 quant: the warp walks (row, step) units; the next unit's loads (of the same row
-    // or the warp's next row) are in flight while the current one is converted, so a new row
-    // starts without waiting for its data.
-    int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp;
-    int b0 = 0;
+    // Plain 1x128 quant over (row, step) units, a step being BPS blocks of one row; the next
+    // unit's loads are in flight while the current one is converted.  With at least as many rows
+    // as warps, a warp takes whole rows (its steps in order, then the row `stride` further on).
+    // With fewer rows (SPREAD, which the launch picks when M < stride), the warps take every
+    // stride-th unit, so a few rows still occupy them all.
+    const int S = (KB + BPS - 1) / BPS;  // steps per row
+    const int64_t u0 = static_cast<int64_t>(blockIdx.x) * wpc + warp;
+    int64_t m = u0, Sq = 0;              // SPREAD: the unit stride is Sq rows and Sr steps
+    int b0 = 0, Sr = 0;
+    if constexpr (SPREAD) {
+      m = u0 / S;
+      b0 = static_cast<int>(u0 - m * S) * BPS;
+      Sq = stride / S;
+      Sr = static_cast<int>(stride - Sq * S);
+    }
     uint4 v0[CPL], v1[CPL];
     auto load_unit = [&](int64_t mm, int bb0, uint4 (&dst)[CPL]) {
       if (mm < M) {
@@ -463,7 +473,14 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     while (m < M) {
       int64_t m1 = m;
       int b1 = b0 + BPS;
-      if (b1 >= KB) {
+      if constexpr (SPREAD) {
+        m1 = m + Sq;
+        b1 = b0 + Sr * BPS;
+        if (b1 >= S * BPS) {
+          b1 -= S * BPS;
+          ++m1;
+        }
+      } else if (b1 >= KB) {
         b1 = 0;
         m1 += stride;
       }
