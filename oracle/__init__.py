@@ -74,6 +74,9 @@ def lib():
         L.oracle_kv_cache_write.restype = None
         L.oracle_quant_rowwise.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64, P]
         L.oracle_quant_rowwise.restype = None
+        L.oracle_add_rmsnorm_quant.argtypes = [P, I64, P, I64, P, ctypes.c_float, I64, I64,
+                                               ctypes.c_int, P, I64, P, I64]
+        L.oracle_add_rmsnorm_quant.restype = None
         L.oracle_gemm_w8a8_rowwise_rows.argtypes = [P, I64, P, P, I64, P, I64, I64, P, I64, P, P]
         L.oracle_gemm_w8a8_rowwise_rows.restype = None
         L.oracle_e4m3_encode_array.argtypes = [P, I64, P]
@@ -367,6 +370,29 @@ def quant_rowwise(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6):
     lib().oracle_quant_rowwise(_ptr(x), None if g is None else _ptr(g), float(eps), R, K, K,
                                _ptr(q), K, _ptr(s))
     return q, s
+
+
+def add_rmsnorm_quant(x_bf16: np.ndarray, res_bf16: np.ndarray, gamma_bf16: np.ndarray,
+                      eps: float = 1e-6, per_token: bool = False, lds: int = None):
+    """Residual add + RMSNorm + quant, reading R11: h = bf16(fp32(x) + fp32(res)); returns
+    (h, codes, scales) -- h the updated residual, scales [K/128, lds] K-block-major (1x128 groups)
+    or [M] (per_token).  The inputs are not modified."""
+    x = _c(x_bf16, np.uint16)
+    h = np.array(_c(res_bf16, np.uint16), copy=True)
+    g = _c(gamma_bf16, np.uint16)
+    M, K = x.shape
+    if h.shape != (M, K):
+        raise ValueError("x and res differ in shape")
+    q = np.empty((M, K), np.uint8)
+    if per_token:
+        lds = 0
+        sa = np.empty(M, np.float32)
+    else:
+        lds = M if lds is None else lds
+        sa = np.zeros((K // 128, lds), np.float32)
+    lib().oracle_add_rmsnorm_quant(_ptr(x), K, _ptr(h), K, _ptr(g), float(eps), M, K,
+                                   1 if per_token else 0, _ptr(q), K, _ptr(sa), lds)
+    return h, q, sa
 
 
 def gemm_w8a8_rowwise(aq, sa, wq, sw, rows=None):

@@ -69,6 +69,11 @@
  *       slots given per token (a negative slot: the token is not cached), and Q is quantized
  *       the same way for the attention that reads the cache.  The QKV row of a token holds
  *       Hq heads of Q, then Hkv of K, then Hkv of V, each of D values.
+ *   R11 residual add ahead of the RMSNorm front end [SGL-RMSQ section 1: the fused kernel the
+ *       page calls is the AMD library's add_rmsnorm_quant; the call it prints passes no
+ *       residual]: h_k = bf16_RNE( fp32(x_k) + fp32(res_k) ), the value an unfused bf16 add
+ *       writes; h replaces res (the updated residual stream, as a pre-norm block carries it),
+ *       and the RMSNorm and quant of R4 (1x128 groups) or R7 (one scale per row) run on h.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math -fopenmp.
  * fp32 arithmetic below relies on FLT_EVAL_METHOD == 0 (SSE on x86-64), so every float
@@ -555,6 +560,32 @@ void oracle_quant_rowwise(const uint16_t *x, const uint16_t *gamma, float eps, i
         s[m] = sc;
     }
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Residual add + RMSNorm + quant, reading R11                                                  */
+/* ------------------------------------------------------------------------------------------ */
+
+/* res[m, k] <- bf16_RNE(fp32(x[m, k]) + fp32(res[m, k])) for every row, then the RMSNorm front
+ * end on the updated res: 1x128 groups with K-block-major scales sa[kb * lds + m]
+ * (per_token == 0, reading R4) or one scale per row in sa[m] (per_token != 0, reading R7). */
+void oracle_add_rmsnorm_quant(const uint16_t *x, int64_t ldx, uint16_t *res, int64_t ldr,
+                              const uint16_t *gamma, float eps, int64_t M, int64_t K,
+                              int per_token, uint8_t *q, int64_t ldq, float *sa, int64_t lds) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            float sum = bf16_to_f32(x[m * ldx + k]) + bf16_to_f32(res[m * ldr + k]);
+            res[m * ldr + k] = f32_to_bf16_rne(sum);
+        }
+    if (per_token)
+        oracle_quant_rowwise(res, gamma, eps, M, K, ldr, q, ldq, sa);
+    else
+        oracle_rmsnorm_quant_token(res, gamma, eps, M, K, ldr, q, ldq, sa, lds);
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Per-channel GEMM [SGL-RMSQ section 3], reading R7                                           */
+/* ------------------------------------------------------------------------------------------ */
 
 /* Per-channel GEMM reference on a subset of rows, reading R7: ref = sa[m] * sw[n] * P and
  * absref = sa[m] * sw[n] * sum_k |dec(a) * dec(w)|, in fp64 (P is exact: 8-bit products). */
