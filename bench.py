@@ -307,11 +307,26 @@ def measure_rows(fq, device, steps, warmup, pk):
                                            "frac": byts / ms / 1e6 / hbm,
                                            "workload": "W [24576, 4096], one scale per output channel"}
     ms, _ = timed_loop(lambda: fq.quant_rowwise(x, gam, d["eps"], out_q=aq, out_s=sa), steps,
-                       warmup)
+                       warmup, flush)
     byts = M_ * K_ * 3 + M_ * 4 + K_ * 2
     rows["ptpc_rmsnorm_quant_prefill_X"] = {"ms": ms, "GB/s": byts / ms / 1e6,
                                             "frac": byts / ms / 1e6 / hbm,
                                             "workload": "X [8192, 4096], RMSNorm + one scale per token"}
+    # residual add + RMSNorm + quant: x and the residual read, the new residual written, codes
+    res = dev_bf16(inputs.randn_bf16((M_, K_), 1.0, 2, 7), device)
+    for per_token, tag in ((False, "1x128"), (True, "per_token")):
+        aq2 = torch.empty((M_, K_), dtype=torch.uint8, device=device)
+        sa2 = (torch.empty((M_,), dtype=torch.float32, device=device) if per_token else
+               torch.empty((K_ // 128, M_), dtype=torch.float32, device=device))
+        ms, _ = timed_loop(lambda: fq.add_rmsnorm_quant(x, res, gam, d["eps"], per_token,
+                                                        out_q=aq2, out_sa=sa2), steps, warmup,
+                           flush)
+        byts = M_ * K_ * 7 + sa2.numel() * 4 + K_ * 2
+        rows[f"add_rmsnorm_quant_{tag}_prefill_X"] = {
+            "ms": ms, "GB/s": byts / ms / 1e6, "frac": byts / ms / 1e6 / hbm,
+            "workload": f"X, residual [8192, 4096] -> residual, codes ({tag} scales)"}
+        del aq2, sa2
+    del res
     ms, _ = timed_loop(lambda: fq.gemm_w8a8_rowwise(aq, sa, wq, sw, out=out), steps, warmup)
     rows["ptpc_gemm_prefill"] = {"ms": ms, "TFLOP/s": FLOPS / ms / 1e9,
                                  "frac_fp8_sustained": FLOPS / ms / 1e9 / (2.0 * pk["bf16_sustained"]),

@@ -22,10 +22,11 @@ from ._lib import (FP8Q_ERR_ALIGN, FP8Q_ERR_ARCH, FP8Q_ERR_ARG, FP8Q_ERR_LAUNCH,
 
 import ctypes
 
-__all__ = ["quant_weight_block", "rmsnorm_quant_token", "gemm_w8a8_block",
+__all__ = ["quant_weight_block", "rmsnorm_quant_token", "add_rmsnorm_quant", "gemm_w8a8_block",
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
            "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant", "inverse_rope_quant",
-           "gemm_w8a8_block_diag", "gemm_w8a8_mx", "qkv_scales", "kv_cache_write", "WeightBatch", "selftest_timeout",
+           "gemm_w8a8_block_diag", "gemm_w8a8_mx", "qkv_scales", "kv_cache_write", "WeightBatch",
+           "selftest_timeout",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -334,6 +335,30 @@ def quant_rowwise(x: torch.Tensor, gamma=None, eps: float = 1e-6, out_q=None, ou
                                        _ld(q), _ptr(s), _stream(stream))
     _lib.check(st, "fp8q_quant_rowwise")
     return q, s
+
+
+def add_rmsnorm_quant(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor,
+                      eps: float = 1e-6, per_token: bool = False, out_q=None, out_sa=None,
+                      lds: int = None, stream=None):
+    """Residual add + RMSNorm + quant: residual <- bf16(x + residual) (in place), then the codes
+    of RMSNorm(residual) with 1x128 scales (sa fp32 [K/128, lds], K-block-major) or, per_token,
+    one scale per row (sa fp32 [M]).  Returns (codes, sa)."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if out_q is None else out_q
+    if per_token:
+        sa = torch.empty((M,), dtype=torch.float32, device=x.device) if out_sa is None else out_sa
+        lds = 0
+    else:
+        if lds is None:
+            lds = max(4, (M + 3) // 4 * 4)
+        sa = (torch.empty((K // 128, lds), dtype=torch.float32, device=x.device)
+              if out_sa is None else out_sa)
+        lds = sa.stride(0)
+    st = _lib.lib().fp8q_add_rmsnorm_quant(_ptr(x), _ld(x), _ptr(residual), _ld(residual),
+                                           _ptr(gamma), float(eps), M, K, 1 if per_token else 0,
+                                           _ptr(q), _ld(q), _ptr(sa), lds, _stream(stream))
+    _lib.check(st, "fp8q_add_rmsnorm_quant")
+    return q, sa
 
 
 def gemm_w8a8_rowwise(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor, sw: torch.Tensor,

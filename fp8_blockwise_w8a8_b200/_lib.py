@@ -53,6 +53,8 @@ SIGNATURES = {
                                  _P]),
     "fp8q_quant_rowwise": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "fp8q_gemm_w8a8_rowwise": (_I, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I64, _P]),
+    "fp8q_add_rmsnorm_quant": (_I, [_P, _I64, _P, _I64, _P, ctypes.c_float, _I64, _I64, _I, _P,
+                                    _I64, _P, _I64, _P]),
     "fp8q_selftest_timeout": (_I, [_I64, _P]),
     "fp8q_check_device_error": (_I, [_P]),
     "fp8q_status_string": (ctypes.c_char_p, [_I]),

@@ -76,6 +76,12 @@ int device_state(DeviceState **out) {
         cudaFuncSetAttribute(fp8q::k_quant_rowwise<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
             cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<true, false, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_quant_rowwise<true, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
         cudaFuncSetAttribute(fp8q::k_gemm_w8a8_rowwise,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fp8q::kGemmSmemDense) != cudaSuccess ||
@@ -371,13 +377,13 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   auto *q = static_cast<uint8_t *>(xq_e4m3);
   if (norm)
     fp8q::k_rmsnorm_quant_token<true><<<grid, 32 * wpc, smem, stream>>>(
-        x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, lds);
+        x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
   else if (M < static_cast<int64_t>(grid) * wpc)  // fewer rows than warps: spread the steps
     fp8q::k_rmsnorm_quant_token<false, true><<<grid, 32 * wpc, smem, stream>>>(
-        x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds);
+        x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
   else
     fp8q::k_rmsnorm_quant_token<false><<<grid, 32 * wpc, smem, stream>>>(
-        x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds);
+        x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
   return launch_status();
 }
 
@@ -542,11 +548,69 @@ int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, in
   const auto *g = static_cast<const uint16_t *>(gamma_bf16);
   auto *q = static_cast<uint8_t *>(q_e4m3);
   if (norm)
-    fp8q::k_quant_rowwise<true><<<grid, 32 * wpc, smem, stream>>>(x, ldx, g, eps, M,
-                                                                   static_cast<int>(K), q, ldq, s);
+    fp8q::k_quant_rowwise<true><<<grid, 32 * wpc, smem, stream>>>(
+        x, ldx, g, eps, M, static_cast<int>(K), q, ldq, s, nullptr, 0);
   else
-    fp8q::k_quant_rowwise<false><<<grid, 32 * wpc, smem, stream>>>(x, ldx, nullptr, eps, M,
-                                                                    static_cast<int>(K), q, ldq, s);
+    fp8q::k_quant_rowwise<false><<<grid, 32 * wpc, smem, stream>>>(
+        x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, s, nullptr, 0);
+  return launch_status();
+}
+
+int fp8q_add_rmsnorm_quant(const void *x_bf16, int64_t ldx, void *residual_bf16, int64_t ldr,
+                           const void *gamma_bf16, float eps, int64_t M, int64_t K, int per_token,
+                           void *q_e4m3, int64_t ldq, float *sa, int64_t lds,
+                           cudaStream_t stream) {
+  if (M < 0 || K <= 0 || K % 128 || K > kMaxTokenK) return FP8Q_ERR_SHAPE;
+  if (per_token != 0 && per_token != 1) return FP8Q_ERR_ARG;
+  if (ldx < K || ldr < K || ldq < K || (!per_token && lds < M)) return FP8Q_ERR_SHAPE;
+  if (M == 0) return FP8Q_OK;
+  if (!x_bf16 || !residual_bf16 || !gamma_bf16 || !q_e4m3 || !sa) return FP8Q_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(residual_bf16) || !aligned16(gamma_bf16) ||
+      !aligned16(q_e4m3) || ldx % 8 || ldr % 8 || ldq % 16 ||
+      (per_token ? (reinterpret_cast<uintptr_t>(sa) & 3u) != 0 : (!aligned16(sa) || lds % 4)))
+    return FP8Q_ERR_ALIGN;
+  {  // x is read while the residual is written: the two row ranges must not overlap
+    const auto xb = reinterpret_cast<uintptr_t>(x_bf16), rb = reinterpret_cast<uintptr_t>(residual_bf16);
+    const uintptr_t xe = xb + static_cast<uintptr_t>(((M - 1) * ldx + K) * 2);
+    const uintptr_t re = rb + static_cast<uintptr_t>(((M - 1) * ldr + K) * 2);
+    if (xb < re && rb < xe) return FP8Q_ERR_ARG;
+  }
+  DeviceState *st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != FP8Q_OK) return rc;
+  const int budget = 227 * 1024;
+  int best_wpc = 0, best_ctas = 0, best_smem = 0;
+  for (int wpc : {16, 12, 8, 4, 2, 1}) {
+    const int smem = fp8q::token_smem_bytes(static_cast<int>(K), true, wpc);
+    if (smem > budget) continue;
+    int per_sm = 0;
+    if (per_token)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_quant_rowwise<true, true>,
+                                                    32 * wpc, smem);
+    else
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+          &per_sm, fp8q::k_rmsnorm_quant_token<true, false, true>, 32 * wpc, smem);
+    if (per_sm * wpc > best_ctas * best_wpc) {
+      best_wpc = wpc;
+      best_ctas = per_sm;
+      best_smem = smem;
+    }
+  }
+  if (best_wpc == 0) return FP8Q_ERR_SHAPE;
+  const int wpc = best_wpc, smem = best_smem;
+  const int64_t need = (M + wpc - 1) / wpc;
+  const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  const auto *x = static_cast<const uint16_t *>(x_bf16);
+  auto *res = static_cast<uint16_t *>(residual_bf16);
+  const auto *g = static_cast<const uint16_t *>(gamma_bf16);
+  auto *q = static_cast<uint8_t *>(q_e4m3);
+  if (per_token)
+    fp8q::k_quant_rowwise<true, true><<<grid, 32 * wpc, smem, stream>>>(
+        x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, res, ldr);
+  else
+    fp8q::k_rmsnorm_quant_token<true, false, true><<<grid, 32 * wpc, smem, stream>>>(
+        x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, lds, res, ldr);
   return launch_status();
 }
 

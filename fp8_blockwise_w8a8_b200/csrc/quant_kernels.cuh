@@ -411,15 +411,38 @@ __device__ __forceinline__ double block_sumsq(const uint16_t *blk) {
   return acc;
 }
 
+// Residual add of one row, coalesced (lane l takes 16-byte chunks l, l + 32, ...):
+// res <- h = bf16_RNE(fp32(x) + fp32(res)).  The res lines just read stay in L1 for the passes
+// over h that follow (after a __syncwarp).
+__device__ __forceinline__ void row_add_residual(const uint16_t *xr, uint16_t *rr, int K, int lane) {
+  const int KC = K >> 3;
+#pragma unroll 2
+  for (int j = lane; j < KC; j += 32) {
+    const uint4 a = *reinterpret_cast<const uint4 *>(xr + j * 8);
+    const uint4 b = *reinterpret_cast<const uint4 *>(rr + j * 8);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+    uint32_t h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 s2 = f2_add_rn(unpack_bf16x2(wa[i]), unpack_bf16x2(wb[i]));
+      h[i] = pack_bf16x2(s2.x, s2.y);
+    }
+    *reinterpret_cast<uint4 *>(rr + j * 8) = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+}
+
 // Shared-memory bytes of the token kernel.
 __host__ __device__ constexpr int token_smem_bytes(int K, bool norm, int wpc) {
   return static_cast<int>(sizeof(ScaleTab)) + (norm ? K * 4 + wpc * (K / 128) * 8 : 0);
 }
 
-template <bool NORM, bool SPREAD = false>
+// ADD (with NORM): each row is first replaced by h = bf16(fp32(x) + fp32(res)) in res (row
+// stride ldr), and h is what gets normalised and quantized.
+template <bool NORM, bool SPREAD = false, bool ADD = false>
 __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
-    int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ sa, int64_t lds) {
+    int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ sa, int64_t lds,
+    uint16_t *res, int64_t ldr) {
   constexpr int LPB = NORM ? 8 : 4;        // lanes per 128-block
   constexpr int CPL = 16 / LPB;            // 16-byte chunks per lane
   constexpr int BPS = 32 / LPB;            // blocks per warp step
@@ -509,16 +532,26 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     return;
   }
   for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < M; m += stride) {
-    const uint16_t *xr = x + m * ldx;
+    uint16_t *rr = ADD ? res + m * ldr : nullptr;
+    // the row that is normalised and quantized: x, or h (written over res in the first pass)
+    const uint16_t *xr = ADD ? rr : x + m * ldx;
     const int64_t next = m + stride;
     if (next < M) {
       const char *nr = reinterpret_cast<const char *>(x + next * ldx);
       for (int off = lane * 128; off < K * 2; off += 32 * 128) prefetch_l2(nr + off);
+      if (ADD) {
+        const char *nh = reinterpret_cast<const char *>(res + next * ldr);
+        for (int off = lane * 128; off < K * 2; off += 32 * 128) prefetch_l2(nh + off);
+      }
     }
 
     float r = 1.0f;
     if (NORM) {
       // Sum of squares in fp64: each lane takes its own 128-blocks in ascending k ...
+      if (ADD) {
+        row_add_residual(x + m * ldx, rr, K, lane);
+        __syncwarp();  // every lane's h stores before the reads below
+      }
       for (int b = lane; b < KB; b += 32) wsum[b] = block_sumsq(xr + b * 128);
       __syncwarp();
       // ... then lane 0 adds the block sums in ascending block order.
@@ -585,10 +618,13 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
 // over the row finds its absolute maximum (of y with RMSNorm) and a second pass writes the codes.
 // Both passes read the row through L1 (the row was prefetched into L2 during the previous one).
 // ---------------------------------------------------------------------------------------------
-template <bool NORM>
+// ADD (with NORM): as in k_rmsnorm_quant_token, each row is first replaced by
+// h = bf16(fp32(x) + fp32(res)) in res, and h is normalised and quantized.
+template <bool NORM, bool ADD = false>
 __global__ void __launch_bounds__(512) k_quant_rowwise(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
-    int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_out) {
+    int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ s_out,
+    uint16_t *res, int64_t ldr) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int wpc = blockDim.x >> 5;
@@ -610,14 +646,23 @@ __global__ void __launch_bounds__(512) k_quant_rowwise(
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
   for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < M; m += stride) {
-    const uint16_t *xr = x + m * ldx;
+    uint16_t *rr = ADD ? res + m * ldr : nullptr;
+    const uint16_t *xr = ADD ? rr : x + m * ldx;   // the row that is normalised and quantized
     const int64_t next = m + stride;
     if (next < M) {
       const char *nr = reinterpret_cast<const char *>(x + next * ldx);
       for (int off = lane * 128; off < K * 2; off += 32 * 128) prefetch_l2(nr + off);
+      if (ADD) {
+        const char *nh = reinterpret_cast<const char *>(res + next * ldr);
+        for (int off = lane * 128; off < K * 2; off += 32 * 128) prefetch_l2(nh + off);
+      }
     }
     float r = 1.0f;
     if (NORM) {
+      if (ADD) {
+        row_add_residual(x + m * ldx, rr, K, lane);
+        __syncwarp();  // every lane's h stores before the reads below
+      }
       for (int b = lane; b < KB; b += 32) wsum[b] = block_sumsq(xr + b * 128);
       __syncwarp();
       if (lane == 0) {

@@ -334,6 +334,27 @@ int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, in
                        int64_t K, int64_t ldx, void *q_e4m3, int64_t ldq, float *s,
                        cudaStream_t stream);
 
+/* Residual add + RMSNorm + quantization in one pass over each row (the fused add-RMSNorm-quant of
+ * a pre-norm block; the updated residual stream is written back):
+ *   x_bf16        [M][ldx] bf16, read (the sub-layer output)
+ *   residual_bf16 [M][ldr] bf16, read and overwritten with h = bf16_RNE(fp32(x) + fp32(residual))
+ *   gamma_bf16    [K] bf16 RMSNorm weight (required); eps as fp8q_rmsnorm_quant_token
+ *   per_token     0: 1x128 groups, sa [K/128][lds] K-block-major as fp8q_rmsnorm_quant_token
+ *                 (lds >= M, lds % 4 == 0, 16-byte aligned); 1: one scale per row, sa [M]
+ *                 (4-byte aligned; lds unused), as fp8q_quant_rowwise
+ *   q_e4m3        [M][ldq] uint8 codes of RMSNorm(h), written
+ * The norm and quant arithmetic are those of fp8q_rmsnorm_quant_token / fp8q_quant_rowwise, on h.
+ * The x and residual row ranges must not overlap (FP8Q_ERR_ARG otherwise); ldx, ldr % 8 == 0,
+ * ldq % 16 == 0, K % 128 == 0, K <= 16384; per_token other than 0 or 1 is FP8Q_ERR_ARG.
+ * Bit-exact (codes, scales and the new residual) against the CPU oracle.  Source: SGLang PR 21403
+ * analysis, section 1 (the fused kernel it calls is the AMD library's add_rmsnorm_quant, with
+ * weight, epsilon and group_size 0 = per token; the call it prints passes no residual, so the
+ * residual add is the reading above: what an unfused bf16 add writes). */
+int fp8q_add_rmsnorm_quant(const void *x_bf16, int64_t ldx, void *residual_bf16, int64_t ldr,
+                           const void *gamma_bf16, float eps, int64_t M, int64_t K, int per_token,
+                           void *q_e4m3, int64_t ldq, float *sa, int64_t lds,
+                           cudaStream_t stream);
+
 /* Per-token x per-channel W8A8 GEMM:
  *   out[m, n] = bf16( P[m, n] * fp32(sa[m] * sw[n]) ),  P = fp32 tensor-core dot product over K
  * with no per-K-block promotion (the scales are constant along K).

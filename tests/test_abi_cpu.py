@@ -157,6 +157,35 @@ def test_rowwise_host_checks(L):
     assert call(M=0, aq=None, sa=None, out=None) == _lib.FP8Q_OK
 
 
+def test_add_rmsnorm_quant_host_checks(L):
+    f = L.fp8q_add_rmsnorm_quant
+    R2 = FAKE + (1 << 24)                 # a residual that does not overlap x
+    ok = dict(x=FAKE, ldx=256, res=R2, ldr=256, g=FAKE, M=8, K=256, pt=0, q=FAKE, ldq=256,
+              sa=FAKE, lds=8)
+
+    def call(**kw):
+        b = dict(ok, **kw)
+        return f(b["x"], b["ldx"], b["res"], b["ldr"], b["g"], 1e-6, b["M"], b["K"], b["pt"],
+                 b["q"], b["ldq"], b["sa"], b["lds"], None)
+    assert call(K=200, ldx=208, ldr=208, ldq=208) == _lib.FP8Q_ERR_SHAPE   # K % 128
+    assert call(K=32768, ldx=32768, ldr=32768, ldq=32768) == _lib.FP8Q_ERR_SHAPE
+    assert call(lds=4) == _lib.FP8Q_ERR_SHAPE                              # lds < M
+    assert call(ldr=128) == _lib.FP8Q_ERR_SHAPE                            # ldr < K
+    assert call(pt=2) == _lib.FP8Q_ERR_ARG
+    assert call(g=None) == _lib.FP8Q_ERR_NULL                              # gamma is required
+    assert call(res=None) == _lib.FP8Q_ERR_NULL
+    assert call(ldr=260) == _lib.FP8Q_ERR_ALIGN
+    assert call(res=R2 + 4) == _lib.FP8Q_ERR_ALIGN
+    assert call(lds=10) == _lib.FP8Q_ERR_ALIGN                             # 1x128: lds % 4
+    assert call(pt=1, lds=0, sa=FAKE + 2) == _lib.FP8Q_ERR_ALIGN
+    assert call(res=FAKE + 256) == _lib.FP8Q_ERR_ARG                       # x and res overlap
+    assert call(M=0, x=None, res=None, g=None, q=None, sa=None) == _lib.FP8Q_OK
+    import torch
+    if not torch.cuda.is_available():     # valid arguments reach the device query
+        assert call() == _lib.FP8Q_ERR_ARCH
+        assert call(pt=1, lds=0) == _lib.FP8Q_ERR_ARCH
+
+
 def test_silu_mul_quant_host_checks(L):
     f = L.fp8q_silu_mul_quant
     assert f(FAKE, 4, 100, 200, FAKE, 112, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE   # I % 128
