@@ -171,6 +171,15 @@ def test_token_rows_sharing_a_warp(K, M):
     _token_case(x, None)
 
 
+@pytest.mark.parametrize("M,K", [(2000, 3072), (1111, 5120), (150, 16384)])
+def test_token_plain_fewer_rows_than_warps(M, K):
+    """Fewer rows than warps: the plain kernel spreads the (row, step) units of all rows over the
+    warps, with a unit stride that is not a whole number of rows (a carry from a row's last step
+    into the next row) on the full grid."""
+    x = inputs.randn_bf16((M, K), 1.0, 95, K + M)
+    _token_case(x)
+
+
 def test_token_strided_rows():
     M, K = 70, 1024
     x = inputs.randn_bf16((M, K + 64), 1.0, 94, 0)
