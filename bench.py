@@ -271,6 +271,20 @@ def measure_rows(fq, device, steps, warmup, pk):
     hbm = pk["hbm"]
     fp8_peak = 2.0 * pk["bf16"]
 
+    # a1 / a2 on the prefill weight alone, L2 flushed between calls (inside the step the requant
+    # also absorbs the write-back of the previous step's GEMM output)
+    wp = torch.randn((N_, K_), device=device).mul_(0.02).to(torch.bfloat16)
+    for fmt, name in ((fq.FP8Q_SCALE_F32, "a1_requant_f32_prefill_W_flushed"),
+                      (fq.FP8Q_SCALE_E8M0, "a2_requant_e8m0_prefill_W_flushed")):
+        qp, sp = fq.quant_weight_block(wp, fmt)
+        ms, _ = timed_loop(lambda: fq.quant_weight_block(wp, fmt, out_q=qp, out_s=sp), steps,
+                           warmup, flush)
+        byts = N_ * K_ * 3 + sp.numel() * sp.element_size()
+        rows[name] = {"ms": ms, "GB/s": byts / ms / 1e6, "frac": byts / ms / 1e6 / hbm,
+                      "workload": "W [24576, 4096] alone"}
+        del qp, sp
+    del wp
+
     # requant sweep: all 252 weights of the 36-layer model, fp32 and E8M0 scales
     ws = [inputs.sweep_matrix(l, i, device) for l in range(inputs.SWEEP_LAYERS)
           for i in range(len(inputs.SWEEP_MATRICES))]
