@@ -16,6 +16,7 @@ are timed separately and reported under "rows".
 workload; it is the deliberately slow baseline, not a GPU implementation.
 """
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -87,7 +88,9 @@ def peaks():
 # clocks during the timed region
 # ---------------------------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling every 20 ms; start() returns once the first sample is in, and stop()
+    keeps the samples whose timestamps fall inside the timed window."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -106,32 +109,47 @@ class ClockSampler:
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < 10.0 and self.proc.poll() is None:
+            if os.path.getsize(self.file.name) > 0:
+                break
+            time.sleep(0.01)
 
-    def stop(self):
+    def stop(self, window=None):
+        """window = (t_begin, t_end) in host epoch seconds: only samples inside it are used (all
+        samples, flagged, if none falls inside)."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.15)
         self.proc.terminate()
         self.proc.wait(timeout=10)
         self.file.seek(0)
         rows = [ln.split(",") for ln in self.file.read().strip().splitlines() if ln.strip()]
         os.unlink(self.file.name)
-        sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        parsed = []
         for r in rows:
             r = [c.strip() for c in r]
-            if len(r) < 9:
+            if len(r) < 10:
                 continue
             try:
-                sm.append(float(r[1]))
-                smax = float(r[2])
+                ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                parsed.append((ts, float(r[2]), float(r[3]),
+                               {n for n, v in zip(names, r[6:10]) if v.lower() == "active"}))
             except ValueError:
                 continue
-            for n, v in zip(names, r[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = parsed if window is None else \
+            [p for p in parsed if window[0] - 0.005 <= p[0] <= window[1] + 0.005]
+        out = {}
+        if window is not None and not inside:
+            inside = parsed
+            out["window"] = "no sample inside the timed window; all samples"
+        sm = [p[1] for p in inside]
+        out.update({"sm_mhz": statistics.median(sm) if sm else None,
+                    "sm_max_mhz": inside[-1][2] if inside else None,
+                    "reasons": sorted(set().union(*[p[3] for p in inside])) if inside else [],
+                    "samples": len(sm)})
+        return out
 
 
 # ---------------------------------------------------------------------------------------------
@@ -672,7 +690,9 @@ def run_ours(args):
         step.run(evs[i])
     t_end.record()
     torch.cuda.synchronize()
-    clk = clocks.stop()
+    t_host_end = time.time()
+    ms_local = t_start.elapsed_time(t_end)
+    clk = clocks.stop((t_host_end - ms_local / 1000.0, t_host_end))
     if dist is not None:
         dist.barrier()
     ms_total = max_over_ranks(t_start.elapsed_time(t_end), dist, device)
