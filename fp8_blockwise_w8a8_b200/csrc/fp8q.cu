@@ -521,6 +521,21 @@ int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, in
   const int rc = device_state(&st);
   if (rc != FP8Q_OK) return rc;
   const bool norm = gamma_bf16 != nullptr;
+  if (!norm && K <= 4096) {  // the row fits in registers: one pass over memory
+    const auto *x = static_cast<const uint16_t *>(x_bf16);
+    auto *q = static_cast<uint8_t *>(q_e4m3);
+    const int Ki = static_cast<int>(K);
+    int per_sm = 0;
+    auto launch = [&](auto kern) {
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+      const int64_t need = (M + 7) / 8, cap = static_cast<int64_t>(st->sms) * (per_sm > 0 ? per_sm : 1);
+      kern<<<static_cast<int>(need < cap ? need : cap), 256, 0, stream>>>(x, ldx, M, Ki, q, ldq, s);
+    };
+    if (K <= 1024) launch(fp8q::k_quant_rowwise_regs<4>);
+    else if (K <= 2048) launch(fp8q::k_quant_rowwise_regs<8>);
+    else launch(fp8q::k_quant_rowwise_regs<16>);
+    return launch_status();
+  }
   const int budget = 227 * 1024;
   int best_wpc = 0, best_ctas = 0, best_smem = 0;
   for (int wpc : {16, 12, 8, 4, 2, 1}) {

@@ -620,6 +620,45 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
 // ---------------------------------------------------------------------------------------------
 // ADD (with NORM): as in k_rmsnorm_quant_token, each row is first replaced by
 // h = bf16(fp32(x) + fp32(res)) in res, and h is normalised and quantized.
+// Per-row quantization without RMSNorm for rows of up to 32 C 16-byte chunks (K <= 256 C): the warp
+// loads the whole row into registers at once (lane l holds chunks l, l + 32, ...), takes its amax
+// and writes the codes from the same registers -- one pass over memory with C loads in flight per
+// lane.  Same arithmetic as k_quant_rowwise<false>.
+template <int C>
+__global__ void __launch_bounds__(256) k_quant_rowwise_regs(const uint16_t *__restrict__ x, int64_t ldx,
+                                                            int64_t M, int K, uint8_t *__restrict__ q,
+                                                            int64_t ldq, float *__restrict__ s_out) {
+  __shared__ ScaleTab tab;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int wpc = blockDim.x >> 5;
+  const int KC = K >> 3;
+  build_scale_tab(&tab, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
+  for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < M; m += stride) {
+    const uint16_t *xr = x + m * ldx;
+    uint4 v[C];
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const int j = lane + 32 * i;
+      v[i] = j < KC ? ld_stream_v4(xr + j * 8) : make_uint4(0u, 0u, 0u, 0u);  // zeros: no effect on amax
+    }
+    uint32_t m2 = 0u;
+#pragma unroll
+    for (int i = 0; i < C; ++i) m2 = absmax_uint4(m2, v[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+    const QParams p = qparams_tab(absmax_finish(m2), &tab);
+    uint8_t *qr = q + m * ldq;
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const int j = lane + 32 * i;
+      if (j < KC) *reinterpret_cast<uint2 *>(qr + j * 8) = quant8_f32(v[i], p);
+    }
+    if (lane == 0) s_out[m] = p.s;
+  }
+}
+
 template <bool NORM, bool ADD = false>
 __global__ void __launch_bounds__(512) k_quant_rowwise(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
