@@ -369,6 +369,9 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   const int wpc = best_wpc, smem = best_smem;
   // the plain kernel spreads (row, step) units over the warps, the fused one whole rows
   const int64_t units = norm ? M : M * ((K / 128 + 7) / 8);
+  // plain, K/128 not a multiple of the 8 blocks of a warp step: the packed walk (8 consecutive
+  // blocks of the flattened (row, block) sequence per warp step)
+  const bool packed = !norm && (K / 128) % 8 != 0;
   const int64_t need = (units + wpc - 1) / wpc;
   const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
   const int grid = static_cast<int>(need < cap ? need : cap);
@@ -378,7 +381,12 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   if (norm)
     fp8q::k_rmsnorm_quant_token<true><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
-  else if (M < static_cast<int64_t>(grid) * wpc)  // fewer rows than warps: spread the steps
+  else if (packed) {
+    const int64_t pneed = ((M * (K / 128) + 7) / 8 + wpc - 1) / wpc;
+    const int pgrid = static_cast<int>(pneed < cap ? pneed : cap);
+    fp8q::k_rmsnorm_quant_token<false, false, false, true><<<pgrid, 32 * wpc, smem, stream>>>(
+        x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
+  } else if (M < static_cast<int64_t>(grid) * wpc)  // fewer rows than warps: spread the steps
     fp8q::k_rmsnorm_quant_token<false, true><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
   else

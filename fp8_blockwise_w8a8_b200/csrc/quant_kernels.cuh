@@ -438,7 +438,8 @@ __host__ __device__ constexpr int token_smem_bytes(int K, bool norm, int wpc) {
 
 // ADD (with NORM): each row is first replaced by h = bf16(fp32(x) + fp32(res)) in res (row
 // stride ldr), and h is what gets normalised and quantized.
-template <bool NORM, bool SPREAD = false, bool ADD = false>
+// PACKED (plain, K/128 not a multiple of the step's BPS blocks): see the packed walk below.
+template <bool NORM, bool SPREAD = false, bool ADD = false, bool PACKED = false>
 __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
     int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ sa, int64_t lds,
@@ -467,6 +468,57 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
   __syncthreads();
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
+  if constexpr (!NORM && PACKED) {
+    // Plain 1x128 quant, packed walk: the warp's BPS lane groups take BPS consecutive blocks of the
+    // flattened (row, block) sequence, so a step may finish one row and start the next and no group
+    // idles when K/128 is not a multiple of BPS.  Group g of warp w starts at flat block
+    // BPS w + g and advances by BPS stride blocks (dm rows and db blocks, with a carry); its next
+    // block's loads are in flight while the current one is converted.
+    const int64_t f0 = (static_cast<int64_t>(blockIdx.x) * wpc + warp) * BPS + grp;
+    int64_t m = f0 / KB;
+    int b = static_cast<int>(f0 - m * KB);
+    const int64_t df = stride * BPS;
+    const int64_t dm = df / KB;
+    const int db = static_cast<int>(df - dm * KB);
+    uint4 v0[CPL], v1[CPL];
+    auto load_blk = [&](int64_t mm, int bb, uint4 (&dst)[CPL]) {
+      if (mm < M) {
+        const uint16_t *src = x + mm * ldx + bb * 128;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) dst[c] = ld_stream_v4(src + (sub + LPB * c) * 8);
+      }
+    };
+    load_blk(m, b, v0);
+    while (__any_sync(0xffffffffu, m < M)) {
+      int64_t m1 = m + dm;
+      int b1 = b + db;
+      if (b1 >= KB) {
+        b1 -= KB;
+        ++m1;
+      }
+      load_blk(m1, b1, v1);
+      const bool active = m < M;
+      uint32_t mx = 0u;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) mx = absmax_uint4(mx, v0[c]);
+#pragma unroll
+      for (int o = LPB / 2; o > 0; o >>= 1)
+        mx = absmax_bf16x2(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (active) {
+        const QParams p = qparams_tab(absmax_finish(mx), tab);
+        uint8_t *qb = q + m * ldq + b * 128;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+          *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = quant8_f32(v0[c], p);
+        if (sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
+      }
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) v0[c] = v1[c];
+      m = m1;
+      b = b1;
+    }
+    return;
+  }
   if (!NORM) {
     // Plain 1x128 quant over (row, step) units, a step being BPS blocks of one row; the next
     // unit's loads are in flight while the current one is converted.  With at least as many rows
