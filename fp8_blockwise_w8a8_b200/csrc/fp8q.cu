@@ -653,18 +653,26 @@ int fp8q_silu_mul_quant(const void *h_bf16, int64_t R, int64_t I, int64_t ldh, v
   int best_wpc = 0, best_ctas = 0;
   for (int wpc : {16, 8, 4}) {
     int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_silu_mul_quant, 32 * wpc,
-                                                  smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_silu_mul_quant<false>,
+                                                  32 * wpc, smem);
     if (per_sm * wpc > best_ctas * best_wpc) {
       best_wpc = wpc;
       best_ctas = per_sm;
     }
   }
   if (best_wpc == 0) return FP8Q_ERR_LAUNCH;
-  const int64_t need = (R + best_wpc - 1) / best_wpc;
   const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
+  if ((I / 128) % 4 != 0) {  // packed walk: 4 consecutive blocks of the flattened (row, block) order
+    const int64_t need = ((R * (I / 128) + 3) / 4 + best_wpc - 1) / best_wpc;
+    const int grid = static_cast<int>(need < cap ? need : cap);
+    fp8q::k_silu_mul_quant<true><<<grid, 32 * best_wpc, smem, stream>>>(
+        static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
+        static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
+    return launch_status();
+  }
+  const int64_t need = (R + best_wpc - 1) / best_wpc;
   const int grid = static_cast<int>(need < cap ? need : cap);
-  fp8q::k_silu_mul_quant<<<grid, 32 * best_wpc, smem, stream>>>(
+  fp8q::k_silu_mul_quant<false><<<grid, 32 * best_wpc, smem, stream>>>(
       static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
       static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
   return launch_status();

@@ -857,6 +857,11 @@ __device__ __forceinline__ uint4 silu_mul8(const uint4 g, const uint4 u) {
 // One warp per row at a time; 8 lanes per 128-block (4 blocks per warp step), lane `sub` of a
 // block owns the 16-byte chunks sub + 8 c, c = 0, 1.  The gate and up loads of the next step
 // are issued before the current step is processed.
+// PACKED (I/128 not a multiple of the 4 blocks of a warp step): the warp's 4 lane groups take 4
+// consecutive blocks of the flattened (row, block) sequence, so a step may finish one row and
+// start the next and no group computes exponentials for nothing; each group advances by a
+// precomputed (rows, blocks) stride with a carry, its next block's loads in flight.
+template <bool PACKED = false>
 __global__ void __launch_bounds__(512) k_silu_mul_quant(
     const uint16_t *__restrict__ h, int64_t ldh, int64_t R, int I, uint8_t *__restrict__ q,
     int64_t ldq, float *__restrict__ sa, int64_t lds) {
@@ -871,6 +876,55 @@ __global__ void __launch_bounds__(512) k_silu_mul_quant(
   __syncthreads();
 
   const int64_t stride = static_cast<int64_t>(gridDim.x) * wpc;
+  if constexpr (PACKED) {
+    const int64_t f0 = (static_cast<int64_t>(blockIdx.x) * wpc + warp) * BPS + grp;
+    int64_t m = f0 / IB;
+    int b = static_cast<int>(f0 - m * IB);
+    const int64_t df = stride * BPS;
+    const int64_t dm = df / IB;
+    const int db = static_cast<int>(df - dm * IB);
+    uint4 gn[CPL], un[CPL];
+    auto load_blk = [&](int64_t mm, int bb) {
+      if (mm < R) {
+        const uint16_t *gr = h + mm * ldh + bb * 128, *ur = gr + I;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          gn[c] = ld_stream_v4(gr + (sub + LPB * c) * 8);
+          un[c] = ld_stream_v4(ur + (sub + LPB * c) * 8);
+        }
+      }
+    };
+    load_blk(m, b);
+    while (__any_sync(0xffffffffu, m < R)) {
+      const bool active = m < R;
+      uint4 v[CPL];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) v[c] = silu_mul8(gn[c], un[c]);
+      int64_t m1 = m + dm;
+      int b1 = b + db;
+      if (b1 >= IB) {
+        b1 -= IB;
+        ++m1;
+      }
+      load_blk(m1, b1);
+      uint32_t m2 = 0u;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) m2 = absmax_uint4(m2, v[c]);
+#pragma unroll
+      for (int o = LPB / 2; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+      if (active) {
+        const QParams p = qparams_tab(absmax_finish(m2), tab);
+        uint8_t *qb = q + m * ldq + b * 128;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c)
+          *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = quant8_f32(v[c], p);
+        if (sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
+      }
+      m = m1;
+      b = b1;
+    }
+    return;
+  }
   for (int64_t m = static_cast<int64_t>(blockIdx.x) * wpc + warp; m < R; m += stride) {
     const uint16_t *gr = h + m * ldh, *ur = gr + I;
     uint4 gn[CPL], un[CPL];
