@@ -891,6 +891,15 @@ def run_ncu_case(name):
         out = torch.empty((R, 1536), dtype=torch.bfloat16, device=dev)
         fn = lambda: fq.grouped_gemm_w8a8_block(aq, sa, wq.view(128, 1536, 2048),
                                                 sw.view(128, 12, 16), offd, out=out)
+    elif name == "grouped_down":
+        tok, off = inputs.moe_routing()
+        R = int(off[-1])
+        aq, sa = fq.rmsnorm_quant_token(randn((R, 768), 1.0))
+        wq, sw = fq.quant_weight_block(randn((128 * 2048, 768), 0.02), "f32")
+        offd = torch.from_numpy(off).to(dev)
+        out = torch.empty((R, 2048), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.grouped_gemm_w8a8_block(aq, sa, wq.view(128, 2048, 768),
+                                                sw.view(128, 16, 6), offd, out=out)
     elif name in ("inverse_rope_wo_a", "inverse_rope_wo_a_f32"):   # o [8192, 32, 512]: 268 MB in
         o = randn((8192, 32, 512), 1.0)
         pos = torch.randint(0, 16384, (8192,), generator=g, device=dev)
