@@ -891,6 +891,14 @@ def run_ncu_case(name):
         out = torch.empty((R, 1536), dtype=torch.bfloat16, device=dev)
         fn = lambda: fq.grouped_gemm_w8a8_block(aq, sa, wq.view(128, 1536, 2048),
                                                 sw.view(128, 12, 16), offd, out=out)
+    elif name == "silu_moe":              # [gate | up] [32768, 1536] -> codes [32768, 768]
+        hgu = randn((32768, 1536), 2.0)
+        fn = lambda: fq.silu_mul_quant(hgu)
+    elif name == "ptpc_gemm_prefill":     # M=4096 of the per-channel GEMM: A 17 MB, W 101 MB, out 201 MB
+        aq, sa = fq.quant_rowwise(randn((4096, K_), 1.0))
+        wq, sw = fq.quant_rowwise(randn((N_, K_), 0.02))
+        out = torch.empty((4096, N_), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.gemm_w8a8_rowwise(aq, sa, wq, sw, out=out)
     elif name == "grouped_down":
         tok, off = inputs.moe_routing()
         R = int(off[-1])
