@@ -101,7 +101,7 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
 }
 
 // ---------------------------------------------------------------------------------------------
-// TMA (no multicast anywhere in this library)
+// TMA (every load lands in the issuing CTA's own shared memory)
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
