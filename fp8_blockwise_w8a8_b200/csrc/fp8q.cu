@@ -257,6 +257,28 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
   return launch_status();
 }
 
+// Launch shape of the one-warp-per-row kernels: the warps per CTA (16, 12, 8, 4, 2 or 1) that keep
+// the most warps resident per SM within the shared-memory budget; wpc == 0 if none fits.
+struct RowLaunch {
+  int wpc = 0, ctas = 0, smem = 0;
+};
+template <typename Kern>
+RowLaunch pick_row_launch(Kern kern, int K, bool norm) {
+  RowLaunch best;
+  for (int wpc : {16, 12, 8, 4, 2, 1}) {
+    const int smem = fp8q::token_smem_bytes(K, norm, wpc);
+    if (smem > 227 * 1024) continue;
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 32 * wpc, smem);
+    if (per_sm * wpc > best.ctas * best.wpc) {
+      best.wpc = wpc;
+      best.ctas = per_sm;
+      best.smem = smem;
+    }
+  }
+  return best;
+}
+
 }  // namespace
 
 extern "C" {
@@ -346,34 +368,18 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   const int rc = device_state(&st);
   if (rc != FP8Q_OK) return rc;
   const bool norm = gamma_bf16 != nullptr;
-  const int budget = 227 * 1024;
-  // Warps per CTA: the choice that keeps the most warps resident per SM.
-  int best_wpc = 0, best_ctas = 0, best_smem = 0;
-  for (int wpc : {16, 12, 8, 4, 2, 1}) {
-    const int smem = fp8q::token_smem_bytes(static_cast<int>(K), norm, wpc);
-    if (smem > budget) continue;
-    int per_sm = 0;
-    if (norm)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_rmsnorm_quant_token<true>,
-                                                    32 * wpc, smem);
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_rmsnorm_quant_token<false>,
-                                                    32 * wpc, smem);
-    if (per_sm * wpc > best_ctas * best_wpc) {
-      best_wpc = wpc;
-      best_ctas = per_sm;
-      best_smem = smem;
-    }
-  }
-  if (best_wpc == 0) return FP8Q_ERR_SHAPE;
-  const int wpc = best_wpc, smem = best_smem;
+  const RowLaunch L =
+      norm ? pick_row_launch(fp8q::k_rmsnorm_quant_token<true>, static_cast<int>(K), true)
+           : pick_row_launch(fp8q::k_rmsnorm_quant_token<false>, static_cast<int>(K), false);
+  if (L.wpc == 0) return FP8Q_ERR_SHAPE;
+  const int wpc = L.wpc, smem = L.smem;
   // the plain kernel spreads (row, step) units over the warps, the fused one whole rows
   const int64_t units = norm ? M : M * ((K / 128 + 7) / 8);
   // plain, K/128 not a multiple of the 8 blocks of a warp step: the packed walk (8 consecutive
   // blocks of the flattened (row, block) sequence per warp step)
   const bool packed = !norm && (K / 128) % 8 != 0;
   const int64_t need = (units + wpc - 1) / wpc;
-  const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
+  const int64_t cap = static_cast<int64_t>(st->sms) * L.ctas;
   const int grid = static_cast<int>(need < cap ? need : cap);
   const auto *x = static_cast<const uint16_t *>(x_bf16);
   const auto *g = static_cast<const uint16_t *>(gamma_bf16);
@@ -544,28 +550,13 @@ int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, in
     else launch(fp8q::k_quant_rowwise_regs<16>);
     return launch_status();
   }
-  const int budget = 227 * 1024;
-  int best_wpc = 0, best_ctas = 0, best_smem = 0;
-  for (int wpc : {16, 12, 8, 4, 2, 1}) {
-    const int smem = fp8q::token_smem_bytes(static_cast<int>(K), norm, wpc);
-    if (smem > budget) continue;
-    int per_sm = 0;
-    if (norm)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_quant_rowwise<true>,
-                                                    32 * wpc, smem);
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_quant_rowwise<false>,
-                                                    32 * wpc, smem);
-    if (per_sm * wpc > best_ctas * best_wpc) {
-      best_wpc = wpc;
-      best_ctas = per_sm;
-      best_smem = smem;
-    }
-  }
-  if (best_wpc == 0) return FP8Q_ERR_SHAPE;
-  const int wpc = best_wpc, smem = best_smem;
+  const RowLaunch L = norm
+                           ? pick_row_launch(fp8q::k_quant_rowwise<true>, static_cast<int>(K), true)
+                           : pick_row_launch(fp8q::k_quant_rowwise<false>, static_cast<int>(K), false);
+  if (L.wpc == 0) return FP8Q_ERR_SHAPE;
+  const int wpc = L.wpc, smem = L.smem;
   const int64_t need = (M + wpc - 1) / wpc;
-  const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
+  const int64_t cap = static_cast<int64_t>(st->sms) * L.ctas;
   const int grid = static_cast<int>(need < cap ? need : cap);
   const auto *x = static_cast<const uint16_t *>(x_bf16);
   const auto *g = static_cast<const uint16_t *>(gamma_bf16);
@@ -601,28 +592,14 @@ int fp8q_add_rmsnorm_quant(const void *x_bf16, int64_t ldx, void *residual_bf16,
   DeviceState *st = nullptr;
   const int rc = device_state(&st);
   if (rc != FP8Q_OK) return rc;
-  const int budget = 227 * 1024;
-  int best_wpc = 0, best_ctas = 0, best_smem = 0;
-  for (int wpc : {16, 12, 8, 4, 2, 1}) {
-    const int smem = fp8q::token_smem_bytes(static_cast<int>(K), true, wpc);
-    if (smem > budget) continue;
-    int per_sm = 0;
-    if (per_token)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fp8q::k_quant_rowwise<true, true>,
-                                                    32 * wpc, smem);
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-          &per_sm, fp8q::k_rmsnorm_quant_token<true, false, true>, 32 * wpc, smem);
-    if (per_sm * wpc > best_ctas * best_wpc) {
-      best_wpc = wpc;
-      best_ctas = per_sm;
-      best_smem = smem;
-    }
-  }
-  if (best_wpc == 0) return FP8Q_ERR_SHAPE;
-  const int wpc = best_wpc, smem = best_smem;
+  const RowLaunch L =
+      per_token
+          ? pick_row_launch(fp8q::k_quant_rowwise<true, true>, static_cast<int>(K), true)
+          : pick_row_launch(fp8q::k_rmsnorm_quant_token<true, false, true>, static_cast<int>(K), true);
+  if (L.wpc == 0) return FP8Q_ERR_SHAPE;
+  const int wpc = L.wpc, smem = L.smem;
   const int64_t need = (M + wpc - 1) / wpc;
-  const int64_t cap = static_cast<int64_t>(st->sms) * best_ctas;
+  const int64_t cap = static_cast<int64_t>(st->sms) * L.ctas;
   const int grid = static_cast<int>(need < cap ? need : cap);
   const auto *x = static_cast<const uint16_t *>(x_bf16);
   auto *res = static_cast<uint16_t *>(residual_bf16);
