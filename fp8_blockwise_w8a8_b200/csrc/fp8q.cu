@@ -283,7 +283,7 @@ RowLaunch pick_row_launch(Kern kern, int K, bool norm) {
 
 extern "C" {
 
-int fp8q_abi_version(void) { return (1 << 16) | 3; }
+int fp8q_abi_version(void) { return (1 << 16) | 4; }
 
 const char *fp8q_status_string(int status) {
   switch (status) {
