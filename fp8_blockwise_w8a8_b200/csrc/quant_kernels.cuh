@@ -436,9 +436,15 @@ __host__ __device__ constexpr int token_smem_bytes(int K, bool norm, int wpc) {
   return static_cast<int>(sizeof(ScaleTab)) + (norm ? K * 4 + wpc * (K / 128) * 8 : 0);
 }
 
-// ADD (with NORM): each row is first replaced by h = bf16(fp32(x) + fp32(res)) in res (row
-// stride ldr), and h is what gets normalised and quantized.
-// PACKED (plain, K/128 not a multiple of the step's BPS blocks): see the packed walk below.
+// 1x128 token quant, optionally after RMSNorm.  Instantiations:
+//   NORM    one warp per row: fp64 sums of squares (lane per 128-block, ascending k), lane 0 adds
+//           them in block order and forms r; then the normalised row is quantized, 8 lanes per block;
+//   ADD     (with NORM) each row is first replaced by h = bf16(fp32(x) + fp32(res)) in res (row
+//           stride ldr), and h is what gets normalised and quantized;
+//   !NORM   plain quant, 4 lanes per block, over (row, step) units with the next unit's loads in
+//           flight: whole rows per warp; SPREAD (fewer rows than warps) spreads the units over all
+//           warps; PACKED (K/128 not a multiple of the 8 blocks of a step) packs each step with
+//           consecutive blocks of the flattened (row, block) sequence.
 template <bool NORM, bool SPREAD = false, bool ADD = false, bool PACKED = false>
 __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
