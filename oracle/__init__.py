@@ -53,6 +53,8 @@ def lib():
                                                           ctypes.c_int, P, I64, I64, I64, P,
                                                           I64, P, P]
         L.oracle_e4m3_encode_array.restype = None
+        L.oracle_exp_constants.restype = None
+        L.oracle_exp_constants.argtypes = [P, ctypes.c_int]
         L.oracle_exp_f32.argtypes = [ctypes.c_float]
         L.oracle_exp_f32.restype = ctypes.c_float
         L.oracle_silu_f32.argtypes = [ctypes.c_float]
@@ -269,6 +271,13 @@ def gemm_w8a8_block_diag(aq, sa, wq, sw, sw_fmt: int = SCALE_F32, rows=None):
 def exp_f32(x: float) -> float:
     """e^x in fp32 by the method of reading R8 (Cody-Waite reduction, degree-7 Taylor)."""
     return float(lib().oracle_exp_f32(float(x)))
+
+
+def exp_constants() -> np.ndarray:
+    """The exponential's constants: [1/ln 2, c1, c2, 1/7!, 1/6!, ..., 1/1!, 1/0!] as fp32."""
+    out = np.zeros(11, np.float32)
+    lib().oracle_exp_constants(_ptr(out), 11)
+    return out
 
 
 def silu_f32(g: float) -> float:

@@ -338,6 +338,28 @@ void oracle_rmsnorm_quant_token(const uint16_t *x, const uint16_t *gamma, float 
 /* SiLU-and-mul + 1x128 quant, reading R8                                                      */
 /* ------------------------------------------------------------------------------------------ */
 
+/* Constants of the fp32 exponential below: 1/ln 2 rounded to fp32; ln 2 = c1 + c2 with c1 holding
+ * few enough significant bits that k c1 is exact for |k| <= 150 and c2 = RN_fp32(ln 2 - c1);
+ * then the Taylor coefficients 1/n! rounded to fp32, n = 7 down to 0. */
+static const float EXP_CONST[11] = {
+    0x1.715476p+0f,                                    /* 1/ln 2 */
+    0x1.62e400p-1f,                                    /* c1 */
+    0x1.7f7d1cp-20f,                                   /* c2 */
+    0x1.a01a02p-13f,                                   /* 1/7! */
+    0x1.6c16c2p-10f,                                   /* 1/6! */
+    0x1.111112p-7f,                                    /* 1/5! */
+    0x1.555556p-5f,                                    /* 1/4! */
+    0x1.555556p-3f,                                    /* 1/3! */
+    0x1.000000p-1f,                                    /* 1/2! */
+    1.0f,                                              /* 1/1! */
+    1.0f,                                              /* 1/0! */
+};
+
+/* The constants above, for the oracle's own pins (n <= 11 values). */
+void oracle_exp_constants(float *out, int n) {
+    for (int i = 0; i < n && i < 11; ++i) out[i] = EXP_CONST[i];
+}
+
 /* e^x in fp32 by the method of Cody and Waite (1980): k = rint(x / ln 2); r = (x - k c1) - k c2
  * with ln 2 = c1 + c2 split so that k c1 is exact for |k| <= 150; e^r from its Taylor series to
  * degree 7 by Horner's rule (|r| <= ln2 / 2, truncation below 2^-27 relative); then the exact
@@ -346,17 +368,11 @@ void oracle_rmsnorm_quant_token(const uint16_t *x, const uint16_t *gamma, float 
 float oracle_exp_f32(float x) {
     if (x > 0x1.62e430p+6f) return INFINITY;          /* above ln(FLT_MAX) */
     if (x < -104.0f) return 0.0f;                      /* below half the smallest subnormal */
-    const float inv_ln2 = 0x1.715476p+0f, c1 = 0x1.62e400p-1f, c2 = 0x1.7f7d1cp-20f;
+    const float inv_ln2 = EXP_CONST[0], c1 = EXP_CONST[1], c2 = EXP_CONST[2];
     float kf = rintf(x * inv_ln2);
     float r = (x - kf * c1) - kf * c2;
-    float p = 0x1.a01a02p-13f;                         /* 1/7! */
-    p = p * r + 0x1.6c16c2p-10f;                       /* 1/6! */
-    p = p * r + 0x1.111112p-7f;                        /* 1/5! */
-    p = p * r + 0x1.555556p-5f;                        /* 1/4! */
-    p = p * r + 0x1.555556p-3f;                        /* 1/3! */
-    p = p * r + 0x1.000000p-1f;                        /* 1/2! */
-    p = p * r + 1.0f;
-    p = p * r + 1.0f;
+    float p = EXP_CONST[3];
+    for (int n = 4; n < 11; ++n) p = p * r + EXP_CONST[n];
     int k = (int)kf;
     if (k > 127) { p = p * 0x1p127f; k -= 127; }
     if (k < -126) { p = p * 0x1p-126f; k += 126; }

@@ -2,7 +2,10 @@
 written at per-token cache slots): the maxima against numpy, the scale rule, the 448 code at each
 tensor's maximum, every code against a brute-force nearest search over all finite E4M3 values
 (ties to the even code), and the slot semantics (negative slots write nothing, other rows stay
-untouched)."""
+untouched).  Every code of every tensor is also checked against numpy's IEEE fp32 quotient
+encoded by ml_dtypes' E4M3 cast (round to nearest even, clamped to +-448), which catches a
+reciprocal-multiply slip that a sample of a few hundred elements would miss."""
+import ml_dtypes
 import numpy as np
 
 import oracle
@@ -65,11 +68,38 @@ def test_codes_against_brute_force_and_slots():
         idx = rng.choice(x.size, 400, replace=False)
         quot = (x.ravel()[idx] / sc).astype(np.float32)
         assert np.array_equal(codes.ravel()[idx], _nearest_codes(quot))
+        # every element: IEEE fp32 division (numpy), then ml_dtypes' E4M3 rounding
+        every = np.clip((x / np.float32(sc)).astype(np.float32), -448, 448)
+        assert np.array_equal(codes, every.astype(ml_dtypes.float8_e4m3fn).view(np.uint8))
         # the tensor's maximum lands on the largest code
         i = np.argmax(np.abs(x))
         assert codes.ravel()[i] & 0x7F == 0x7E
     untouched = np.setdiff1d(np.arange(ns), slots[slots >= 0])
     assert (kc[untouched] == 0xAA).all() and (vc[untouched] == 0xAA).all()
+
+
+def test_full_size_every_code_and_negative_control():
+    """The bench's KV workload (8192 tokens, 32 + 2 x 8 heads of 128): all codes of Q, K and V
+    against the independent chain; the reciprocal-multiply slip must change some of them."""
+    d = inputs.kv_cache()
+    Hq, Hkv, D, ns = d["Hq"], d["Hkv"], d["D"], d["num_slots"]
+    s = oracle.qkv_scales(oracle.qkv_amax(d["qkv"], Hq, Hkv, D))
+    kc = np.zeros((ns, Hkv * D), np.uint8)
+    vc = np.zeros((ns, Hkv * D), np.uint8)
+    slots = d["slots"]
+    qc = oracle.kv_cache_write(d["qkv"], Hq, Hkv, D, slots, s, kc, vc)
+    q, k, v = _parts(d)
+    live = slots >= 0
+    planted = 0
+    for codes, x, sc in ((qc, q, s[0]), (kc[slots[live]], k[live], s[1]),
+                         (vc[slots[live]], v[live], s[2])):
+        t = np.clip((x / np.float32(sc)).astype(np.float32), -448, 448)
+        assert np.array_equal(codes, t.astype(ml_dtypes.float8_e4m3fn).view(np.uint8))
+        inv = np.float32(1.0) / np.float32(sc)
+        slip = np.clip((x * inv).astype(np.float32), -448, 448)
+        planted += int(np.count_nonzero(
+            codes != slip.astype(ml_dtypes.float8_e4m3fn).view(np.uint8)))
+    assert planted > 0
 
 
 def test_negative_slot_only_writes_q():

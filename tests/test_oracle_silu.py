@@ -3,6 +3,7 @@ reduction + degree-7 Taylor polynomial) against float64 math.exp, SiLU's sign an
 product against a float64 evaluation, and the fused quant against the pinned 1x128 quant of the
 product."""
 import math
+from fractions import Fraction
 
 import numpy as np
 
@@ -21,6 +22,42 @@ def test_exp_f32_within_two_ulp_of_float64():
         e = oracle.exp_f32(float(x))
         t = math.exp(float(x))
         assert abs(e - t) <= 2 * _ulp32(t), (x, e, t)
+
+
+# ln 2 to 40 decimal places (far beyond the 2^-60 needed below)
+LN2 = Fraction("0.6931471805599453094172321214581765680755")
+
+
+def _rn32(q: Fraction) -> np.float32:
+    """Round a positive rational to the nearest fp32 (ties to even), exactly."""
+    lo = np.float32(float(q))
+    while Fraction(float(lo)) > q:
+        lo = np.nextafter(lo, np.float32(0))
+    while Fraction(float(np.nextafter(lo, np.float32(np.inf)))) <= q:
+        lo = np.nextafter(lo, np.float32(np.inf))
+    hi = np.nextafter(lo, np.float32(np.inf))
+    dlo, dhi = q - Fraction(float(lo)), Fraction(float(hi)) - q
+    if dlo < dhi or (dlo == dhi and (lo.view(np.uint32) & 1) == 0):
+        return lo
+    return hi
+
+
+def _significant_bits(v: np.float32) -> int:
+    m = int(v.view(np.uint32) & 0x7FFFFF) | 0x800000
+    return 24 - ((m & -m).bit_length() - 1)
+
+
+def test_exp_f32_constants_from_their_definitions():
+    """Cody-Waite: c1 + c2 splits ln 2 with k c1 exact for |k| <= 150 (8 bits) and c2 the fp32
+    rounding of ln 2 - c1; the Taylor coefficients are 1/n! rounded to fp32; 1/ln 2 likewise."""
+    c = oracle.exp_constants()
+    assert c[0] == _rn32(1 / LN2)
+    c1, c2 = c[1], c[2]
+    assert _significant_bits(c1) + 8 <= 24            # k c1 exact for |k| < 256
+    assert abs(LN2 - Fraction(float(c1))) < Fraction(1, 2 ** 16)
+    assert c2 == _rn32(LN2 - Fraction(float(c1)))
+    for i, n in enumerate(range(7, -1, -1)):
+        assert c[3 + i] == _rn32(Fraction(1, math.factorial(n))), n
 
 
 def test_exp_f32_special_values_and_subnormal_range():
