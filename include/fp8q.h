@@ -179,7 +179,10 @@ int fp8q_gemm_splitk_workspace_bytes(int64_t M, int64_t N, int64_t K, int splits
  *   S <= 4 fits.  A resolved S of 1 runs fp8q_gemm_w8a8_block and touches no scratch.
  *   Nothing in the buffer needs to start at zero: each call writes every partial it reads.
  *   The first call on each device looks the buffer's address up (cudaGetSymbolAddress, with
- *   that device current); make that first call before any stream capture.
+ *   that device current); make that first call before any stream capture.  The address and
+ *   the kernels' function attributes are cached per device for the life of the process and
+ *   are not refreshed after cudaDeviceReset: do not call this entry point on a device after
+ *   resetting it.
  *   Each device has one such buffer (per process), shared by every caller: two calls on one
  *   device that are not ordered with respect to each other (unsynchronized streams, host
  *   threads) race on it and give wrong results.  Order them.

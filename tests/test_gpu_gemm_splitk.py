@@ -11,7 +11,7 @@ import oracle
 import fp8_blockwise_w8a8_b200 as fq
 from fp8_blockwise_w8a8_b200 import inputs
 
-from helpers import assert_within_gemm_tolerance, dev_f32, dev_u8, host_bf16_f64
+from helpers import assert_within_gemm_tolerance, dev_f32, dev_u8, host_bf16_f64, promoted_steps
 
 pytestmark = pytest.mark.gpu
 
@@ -41,7 +41,7 @@ def test_splitk_ragged(M, N, K, splits, fmt):
     assert fq.check_device_error() == 0
     assert torch.isnan(buf[:, N:].float()).all()
     ref, absref = oracle.gemm_w8a8_block(aq, sa, wq, sw, fmt)
-    assert_within_gemm_tolerance(host_bf16_f64(o), ref, absref)
+    assert_within_gemm_tolerance(host_bf16_f64(o), ref, absref, steps=promoted_steps(K, splits))
     # the same workspace serves the next call, even filled with garbage (every partial is written
     # before it is read); the fixed summation order makes the second result bit-identical
     ws.fill_(0xFF)
@@ -59,7 +59,8 @@ def test_splits_equal_k_blocks_and_single_split():
     for s in (1, K // 128):
         o = fq.gemm_w8a8_block_splitk(*d, 0, splits=s)
         assert fq.check_device_error() == 0
-        assert_within_gemm_tolerance(host_bf16_f64(o), ref, absref, what=f"splits={s}")
+        assert_within_gemm_tolerance(host_bf16_f64(o), ref, absref, what=f"splits={s}",
+                                     steps=promoted_steps(K, s))
     # one split is the unsplit kernel
     o1 = fq.gemm_w8a8_block_splitk(*d, 0, splits=1, workspace=torch.empty(0, device="cuda"))
     o0 = fq.gemm_w8a8_block(*d, 0)
@@ -80,7 +81,9 @@ def test_decode_long_k_auto_splits_sampled_rows():
     assert fq.check_device_error() == 0
     rows = [0, 1, 63, 64, 126, 127]
     ref, absref = oracle.gemm_w8a8_block(aq, sa, wq, sw, 0, rows=rows)
-    assert_within_gemm_tolerance(host_bf16_f64(o)[rows], ref, absref)
+    # the library picks at most one split per K-block
+    assert_within_gemm_tolerance(host_bf16_f64(o)[rows], ref, absref,
+                                 steps=promoted_steps(K, K // 128))
 
 
 def test_decode_auto_choice_does_not_split_short_k():

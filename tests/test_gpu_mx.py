@@ -12,7 +12,8 @@ import oracle
 import fp8_blockwise_w8a8_b200 as fq
 from fp8_blockwise_w8a8_b200 import inputs
 
-from helpers import assert_within_gemm_tolerance, dev_f32, dev_u8, host_bf16_f64
+from helpers import (assert_within_gemm_tolerance, dev_f32, dev_u8, host_bf16_f64,
+                     promoted_steps, tmem_steps)
 
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +49,7 @@ def test_mx_dense_small(M, N, K):
     wq, sw = _weights(1, N, K, 80 + N)
     got = _run(aq, sa, wq, sw)
     ref, absref = oracle.gemm_w8a8_block(aq, sa, wq[0], sw[0], E8M0)
-    assert_within_gemm_tolerance(got, ref, absref, f"mx {M}x{N}x{K}")
+    assert_within_gemm_tolerance(got, ref, absref, f"mx {M}x{N}x{K}", steps=tmem_steps(K))
 
 
 def test_mx_wide_scale_range():
@@ -66,7 +67,7 @@ def test_mx_wide_scale_range():
     wq, sw = oracle.quant_weight_block(inputs.to_bf16_bits(w), E8M0)
     got = _run(aq, sa, wq[None], sw[None])
     ref, absref = oracle.gemm_w8a8_block(aq, sa, wq, sw, E8M0)
-    assert_within_gemm_tolerance(got, ref, absref, "mx wide range")
+    assert_within_gemm_tolerance(got, ref, absref, "mx wide range", steps=tmem_steps(K))
 
 
 @pytest.mark.parametrize("G,M,N_g,K_g", [(3, 200, 256, 384), (4, 64, 512, 256)])
@@ -76,7 +77,7 @@ def test_mx_block_diag_small(G, M, N_g, K_g):
     wq, sw = _weights(G, N_g, K_g, 82)
     got = _run(aq, sa, wq, sw)
     ref, absref = oracle.gemm_w8a8_block_diag(aq, sa, wq, sw, E8M0)
-    assert_within_gemm_tolerance(got, ref, absref, f"mx diag G={G}")
+    assert_within_gemm_tolerance(got, ref, absref, f"mx diag G={G}", steps=tmem_steps(K_g))
 
 
 def test_mx_matches_software_promotion_closely():
@@ -91,7 +92,8 @@ def test_mx_matches_software_promotion_closely():
     sp = host_bf16_f64(fq.gemm_w8a8_block(dev_u8(aq), dev_f32(sa), dev_u8(wq[0]),
                                           dev_f32(sw_f32), 0))
     ref, absref = oracle.gemm_w8a8_block(aq, sa, wq[0], sw[0], E8M0)
-    assert_within_gemm_tolerance(sp, ref, absref, "software promotion")
+    assert_within_gemm_tolerance(sp, ref, absref, "software promotion", steps=promoted_steps(K))
+    assert_within_gemm_tolerance(mx, ref, absref, "hardware scaling", steps=tmem_steps(K))
     assert np.all(np.abs(mx - sp) <= 4 * oracle.bf16_ulp(ref) + 2e-3 * absref)
 
 
@@ -128,7 +130,7 @@ def test_mx_wo_a_full_size_sampled_rows():
                                            True, 1)
     ref, absref = oracle.gemm_w8a8_block_diag(aq_r, sa_r, wq, sw, E8M0, rows=rows)
     got = host_bf16_f64(out[torch.from_numpy(rows).cuda()])
-    assert_within_gemm_tolerance(got, ref, absref, "mx wo_a full size")
+    assert_within_gemm_tolerance(got, ref, absref, "mx wo_a full size", steps=tmem_steps(K_g))
 
 
 def test_mx_prefill_full_size_sampled_rows():
@@ -142,4 +144,4 @@ def test_mx_prefill_full_size_sampled_rows():
                                      np.random.default_rng(7).integers(0, M, 40)]))
     ref, absref = oracle.gemm_w8a8_block(aq, sa, wq, sw, E8M0, rows=rows)
     got = host_bf16_f64(out[torch.from_numpy(rows).cuda()])
-    assert_within_gemm_tolerance(got, ref, absref, "mx prefill full size")
+    assert_within_gemm_tolerance(got, ref, absref, "mx prefill full size", steps=tmem_steps(K))

@@ -133,3 +133,50 @@ def test_tolerance_helper():
     assert tol[1] == 8e-3 * 2 + 2.0 ** -7
     assert tol[2] == 8e-3 * 3 + 2.0 ** -6
     assert tol[3] == 2.0 ** -133
+
+
+# --- the tight fp32 bound the GPU tests apply, and its negative control ---------------------------
+
+def _bf16_round(x):
+    return inputs.bf16_bits_to_f32(inputs.to_bf16_bits(np.asarray(x, np.float32))).astype(
+        np.float64)
+
+
+def _promoted_model(aq, sa, wq, sw, bf16_partials: bool):
+    """A model of per-K-block promotion run on the CPU from the decoded codes: fp32 partials P_kb
+    (exact here), c = fp32(sa sw), acc = fp32(acc + P_kb c) with one rounding per K-block, bf16
+    out.  With bf16_partials the planted mistake rounds P_kb and c to bf16 first."""
+    dec = oracle.e4m3_decode_all()
+    M, K = aq.shape
+    N = wq.shape[0]
+    KB = K // 128
+    A = dec[aq].reshape(M, KB, 128)
+    W = dec[wq].reshape(N, KB, 128)
+    P = np.einsum("mbk,nbk->mnb", A, W)                     # exact in fp64
+    c = (sa.T[:, None, :].astype(np.float32) *
+         np.repeat(sw, 128, axis=0)[None, :, :].astype(np.float32)).astype(np.float32)
+    acc = np.zeros((M, N), np.float32)
+    for b in range(KB):
+        p = P[:, :, b].astype(np.float32).astype(np.float64)
+        cb = c[:, :, b].astype(np.float64)
+        if bf16_partials:
+            p, cb = _bf16_round(p), _bf16_round(cb)
+        acc = (acc.astype(np.float64) + p * cb).astype(np.float32)   # one rounding (as an FMA)
+    return _bf16_round(acc)
+
+
+def test_tight_bound_admits_fp32_promotion_and_rejects_bf16_partials():
+    """The GPU tests' second gate, |out - ref| <= ulp_bf16(|ref|)/2 + (K/128 + 8) 2^-23 absref,
+    holds for a faithful fp32 promotion model on every element, and rejects a kernel that rounds
+    each K-block partial and each sa*sw to bf16 on a large share of the elements (that mistake
+    passes the stated 8e-3 tolerance everywhere)."""
+    from helpers import promoted_steps, tight_gemm_bound
+    for M, N, K, seed in ((16, 1024, 4096, 0), (64, 512, 512, 1)):
+        aq, sa, wq, sw = _quantized_pair(M, N, K, 90 + seed)
+        ref, absref = oracle.gemm_w8a8_block(aq, sa, wq, sw)
+        bound = tight_gemm_bound(ref, absref, promoted_steps(K))
+        good = _promoted_model(aq, sa, wq, sw, False)
+        bad = _promoted_model(aq, sa, wq, sw, True)
+        assert np.all(np.abs(good - ref) <= bound)
+        assert np.all(np.abs(bad - ref) <= oracle.gemm_tolerance(ref, absref))
+        assert np.mean(np.abs(bad - ref) > bound) > 0.2

@@ -11,17 +11,17 @@ import torch
 import oracle
 from fp8_blockwise_w8a8_b200 import _lib, inputs
 
-from helpers import assert_within_gemm_tolerance, dev_f32, dev_u8, host_bf16_f64
+from helpers import assert_within_gemm_tolerance, dev_f32, dev_u8, host_bf16_f64, promoted_steps
 
 pytestmark = pytest.mark.gpu
 
 
-def _operands(M, N, K, seed):
+def _operands(M, N, K, seed, fmt=oracle.SCALE_F32):
     a = inputs.randn_bf16((M, K), 1.0, seed, 0)
     w = inputs.randn_bf16((N, K), 0.02, seed, 1)
     lds = (M + 3) // 4 * 4
     aq, sa = oracle.quant_token_1x128(a, lds=lds)
-    wq, sw = oracle.quant_weight_block(w, oracle.SCALE_F32)
+    wq, sw = oracle.quant_weight_block(w, fmt)
     return aq, sa, wq, sw
 
 
@@ -29,23 +29,22 @@ def _stream():
     return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
 
-def _call_noalloc(L, d, M, N, K, out, splits):
+def _call_noalloc(L, d, M, N, K, out, splits, fmt=_lib.FP8Q_SCALE_F32):
     aq, sa, wq, sw = d
     return L.fp8q_gemm_w8a8_block_splitk_noalloc(
         aq.data_ptr(), aq.stride(0), sa.data_ptr(), sa.stride(0), wq.data_ptr(), wq.stride(0),
-        sw.data_ptr(), _lib.FP8Q_SCALE_F32, M, N, K, out.data_ptr(), out.stride(0), splits,
-        _stream())
+        sw.data_ptr(), fmt, M, N, K, out.data_ptr(), out.stride(0), splits, _stream())
 
 
-def _call_workspace(L, d, M, N, K, out, splits):
+def _call_workspace(L, d, M, N, K, out, splits, fmt=_lib.FP8Q_SCALE_F32):
     aq, sa, wq, sw = d
     nbytes = ctypes.c_int64(0)
     assert L.fp8q_gemm_splitk_workspace_bytes(M, N, K, splits, ctypes.byref(nbytes)) == 0
     ws = torch.empty(max(16, nbytes.value), dtype=torch.uint8, device="cuda")
     st = L.fp8q_gemm_w8a8_block_splitk(
         aq.data_ptr(), aq.stride(0), sa.data_ptr(), sa.stride(0), wq.data_ptr(), wq.stride(0),
-        sw.data_ptr(), _lib.FP8Q_SCALE_F32, M, N, K, out.data_ptr(), out.stride(0), splits,
-        ws.data_ptr(), ws.numel(), _stream())
+        sw.data_ptr(), fmt, M, N, K, out.data_ptr(), out.stride(0), splits, ws.data_ptr(),
+        ws.numel(), _stream())
     return st
 
 
@@ -71,9 +70,34 @@ def test_noalloc_matches_workspace_entry_twice(M, N, K, splits, rows):
         got = host_bf16_f64(out)
         # against the workspace entry point: within the GEMM tolerance (in fact bit-identical,
         # since both run the same kernel with the same split order)
-        assert_within_gemm_tolerance(got[sel], expect[sel], absref, what="vs workspace entry")
+        steps = promoted_steps(K, splits if splits else K // 128)
+        assert_within_gemm_tolerance(got[sel], expect[sel], absref, what="vs workspace entry",
+                                     steps=steps)
         assert np.array_equal(got, expect)
-        assert_within_gemm_tolerance(got[sel], ref, absref, what="vs oracle")
+        assert_within_gemm_tolerance(got[sel], ref, absref, what="vs oracle", steps=steps)
+
+
+def test_noalloc_e8m0_weight_scales_twice():
+    """E8M0 weight scales through the same scratch: decode shape, 3 splits."""
+    L = _lib.lib()
+    M, N, K, splits = 128, 12288, 4096, 3
+    E8M0 = oracle.SCALE_E8M0
+    aq, sa, wq, sw = _operands(M, N, K, 77, E8M0)
+    d = (dev_u8(aq), dev_f32(sa), dev_u8(wq), dev_u8(sw))
+    ref_out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    assert _call_workspace(L, d, M, N, K, ref_out, splits, E8M0) == _lib.FP8Q_OK
+    assert L.fp8q_check_device_error(_stream()) == _lib.FP8Q_OK
+    rows = [0, 1, 64, 127]
+    ref, absref = oracle.gemm_w8a8_block(aq, sa, wq, sw, E8M0, rows=rows)
+    expect = host_bf16_f64(ref_out)
+    for _ in range(2):
+        out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        assert _call_noalloc(L, d, M, N, K, out, splits, E8M0) == _lib.FP8Q_OK
+        assert L.fp8q_check_device_error(_stream()) == _lib.FP8Q_OK
+        got = host_bf16_f64(out)
+        assert np.array_equal(got, expect)
+        assert_within_gemm_tolerance(got[rows], ref, absref, what="e8m0 vs oracle",
+                                     steps=promoted_steps(K, splits))
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
