@@ -39,12 +39,12 @@ def lib():
         L.oracle_quant_weight_block.restype = None
         L.oracle_quant_weight_block.argtypes = [P, I64, I64, I64, P, I64, P, ctypes.c_int]
         L.oracle_quant_token_1x128.restype = None
-        L.oracle_quant_token_1x128.argtypes = [P, I64, I64, I64, P, I64, P, I64]
+        L.oracle_quant_token_1x128.argtypes = [P, I64, I64, I64, P, I64, P, I64, ctypes.c_int]
         L.oracle_rmsnorm_bf16.restype = None
         L.oracle_rmsnorm_bf16.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64]
         L.oracle_rmsnorm_quant_token.restype = None
         L.oracle_rmsnorm_quant_token.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64,
-                                                 P, I64]
+                                                 P, I64, ctypes.c_int]
         L.oracle_gemm_w8a8_block_rows.restype = None
         L.oracle_gemm_w8a8_block_rows.argtypes = [P, I64, P, I64, P, I64, P, ctypes.c_int,
                                                   I64, I64, P, I64, P, P]
@@ -59,7 +59,7 @@ def lib():
         L.oracle_exp_f32.restype = ctypes.c_float
         L.oracle_silu_f32.argtypes = [ctypes.c_float]
         L.oracle_silu_f32.restype = ctypes.c_float
-        L.oracle_silu_mul_quant.argtypes = [P, I64, I64, I64, P, I64, P, I64]
+        L.oracle_silu_mul_quant.argtypes = [P, I64, I64, I64, P, I64, P, I64, ctypes.c_int]
         L.oracle_silu_mul_quant.restype = None
         L.oracle_silu_mul_bf16.argtypes = [P, I64, I64, I64, P]
         L.oracle_silu_mul_bf16.restype = None
@@ -77,7 +77,7 @@ def lib():
         L.oracle_quant_rowwise.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64, P]
         L.oracle_quant_rowwise.restype = None
         L.oracle_add_rmsnorm_quant.argtypes = [P, I64, P, I64, P, ctypes.c_float, I64, I64,
-                                               ctypes.c_int, P, I64, P, I64]
+                                               ctypes.c_int, ctypes.c_int, P, I64, P, I64]
         L.oracle_add_rmsnorm_quant.restype = None
         L.oracle_gemm_w8a8_rowwise_rows.argtypes = [P, I64, P, P, I64, P, I64, I64, P, I64, P, P]
         L.oracle_gemm_w8a8_rowwise_rows.restype = None
@@ -167,14 +167,15 @@ def quant_weight_block(w_bf16: np.ndarray, fmt: int = SCALE_F32):
     return q, sw
 
 
-def quant_token_1x128(x_bf16: np.ndarray, lds: int = None):
-    """X bf16 [M, K] -> (codes [M, K], sa fp32 [K/128, lds]) with sa[kb, m] the scale."""
+def quant_token_1x128(x_bf16: np.ndarray, lds: int = None, fmt: int = SCALE_F32):
+    """X bf16 [M, K] -> (codes [M, K], sa fp32 [K/128, lds]) with sa[kb, m] the scale: amax/448
+    (fmt SCALE_F32) or the E8M0 power of two stored as fp32 (fmt SCALE_E8M0, reading R12)."""
     x = _c(x_bf16, np.uint16)
     M, K = x.shape
     lds = M if lds is None else lds
     q = np.empty((M, K), dtype=np.uint8)
     sa = np.zeros((K // 128, lds), dtype=np.float32)
-    lib().oracle_quant_token_1x128(_ptr(x), M, K, K, _ptr(q), K, _ptr(sa), lds)
+    lib().oracle_quant_token_1x128(_ptr(x), M, K, K, _ptr(q), K, _ptr(sa), lds, int(fmt))
     return q, sa
 
 
@@ -188,8 +189,9 @@ def rmsnorm_bf16(x_bf16: np.ndarray, gamma_bf16: np.ndarray, eps: float = 1e-6):
 
 
 def rmsnorm_quant_token(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6,
-                        lds: int = None):
-    """Fused RMSNorm + 1x128 token quant (gamma None: plain token quant)."""
+                        lds: int = None, fmt: int = SCALE_F32):
+    """Fused RMSNorm + 1x128 token quant (gamma None: plain token quant); fmt as
+    quant_token_1x128."""
     x = _c(x_bf16, np.uint16)
     M, K = x.shape
     lds = M if lds is None else lds
@@ -201,7 +203,7 @@ def rmsnorm_quant_token(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6,
         g = _c(gamma_bf16, np.uint16)
         gp = _ptr(g)
     lib().oracle_rmsnorm_quant_token(_ptr(x), gp, float(eps), M, K, K, _ptr(q), K, _ptr(sa),
-                                     lds)
+                                     lds, int(fmt))
     return q, sa
 
 
@@ -293,15 +295,16 @@ def silu_mul_bf16(h_bf16: np.ndarray) -> np.ndarray:
     return y
 
 
-def silu_mul_quant(h_bf16: np.ndarray, lds: int = None):
-    """SiLU-and-mul then 1x128 token quant (reading R8): codes [R, I] and sa [I/128, lds]."""
+def silu_mul_quant(h_bf16: np.ndarray, lds: int = None, fmt: int = SCALE_F32):
+    """SiLU-and-mul then 1x128 token quant (reading R8): codes [R, I] and sa [I/128, lds]; fmt as
+    quant_token_1x128."""
     h = _c(h_bf16, np.uint16)
     R, I2 = h.shape
     I = I2 // 2
     lds = R if lds is None else lds
     q = np.empty((R, I), np.uint8)
     sa = np.zeros((I // 128, lds), np.float32)
-    lib().oracle_silu_mul_quant(_ptr(h), R, I, I2, _ptr(q), I, _ptr(sa), lds)
+    lib().oracle_silu_mul_quant(_ptr(h), R, I, I2, _ptr(q), I, _ptr(sa), lds, int(fmt))
     return q, sa
 
 
@@ -382,10 +385,14 @@ def quant_rowwise(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6):
 
 
 def add_rmsnorm_quant(x_bf16: np.ndarray, res_bf16: np.ndarray, gamma_bf16: np.ndarray,
-                      eps: float = 1e-6, per_token: bool = False, lds: int = None):
+                      eps: float = 1e-6, per_token: bool = False, lds: int = None,
+                      fmt: int = SCALE_F32):
     """Residual add + RMSNorm + quant, reading R11: h = bf16(fp32(x) + fp32(res)); returns
     (h, codes, scales) -- h the updated residual, scales [K/128, lds] K-block-major (1x128 groups)
-    or [M] (per_token).  The inputs are not modified."""
+    or [M] (per_token).  fmt (1x128 groups only) as quant_token_1x128.  The inputs are not
+    modified."""
+    if per_token and fmt != SCALE_F32:
+        raise ValueError("per-token scales are fp32 only")
     x = _c(x_bf16, np.uint16)
     h = np.array(_c(res_bf16, np.uint16), copy=True)
     g = _c(gamma_bf16, np.uint16)
@@ -400,7 +407,7 @@ def add_rmsnorm_quant(x_bf16: np.ndarray, res_bf16: np.ndarray, gamma_bf16: np.n
         lds = M if lds is None else lds
         sa = np.zeros((K // 128, lds), np.float32)
     lib().oracle_add_rmsnorm_quant(_ptr(x), K, _ptr(h), K, _ptr(g), float(eps), M, K,
-                                   1 if per_token else 0, _ptr(q), K, _ptr(sa), lds)
+                                   1 if per_token else 0, int(fmt), _ptr(q), K, _ptr(sa), lds)
     return h, q, sa
 
 

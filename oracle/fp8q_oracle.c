@@ -74,6 +74,11 @@
  *       residual]: h_k = bf16_RNE( fp32(x_k) + fp32(res_k) ), the value an unfused bf16 add
  *       writes; h replaces res (the updated residual stream, as a pre-norm block carries it),
  *       and the RMSNorm and quant of R4 (1x128 groups) or R7 (one scale per row) run on h.
+ *   R12 E8M0 activation scales for the 1x128 front ends (plain token quant, RMSNorm + quant,
+ *       SiLU-and-mul + quant, residual add + RMSNorm + quant) [DSv4-WOA sections 1 and 3: the
+ *       MX-scaled GEMM takes E8M0 scales on both operands]: the group's scale is R2's power of
+ *       two 2^e (the smallest with 2^e >= fp32(amax / 448), clamped to [-127, 127]), stored as
+ *       its fp32 value, as R9 stores it; codes are RNEsat(y / 2^e), a division that is exact.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math -fopenmp.
  * fp32 arithmetic below relies on FLT_EVAL_METHOD == 0 (SSE on x86-64), so every float
@@ -248,28 +253,30 @@ void oracle_quant_weight_block(const uint16_t *w, int64_t N, int64_t K, int64_t 
 /* ------------------------------------------------------------------------------------------ */
 
 /* Quantize one 128-wide group of fp32 values (already bf16-representable).  Writes 128 codes
- * and returns the fp32 scale. */
-static float quant_group_1x128(const float *y, uint8_t *q) {
+ * and returns the scale as fp32: amax/448 (fmt 0, reading R1) or the E8M0 power of two of
+ * reading R2 (fmt 1, reading R12). */
+static float quant_group_1x128_fmt(const float *y, uint8_t *q, int fmt) {
     float amax = 0.0f;
     for (int j = 0; j < 128; ++j) {
         float a = fabsf(y[j]);
         if (a > amax) amax = a;
     }
-    float s = scale_f32_from_amax(amax);
+    float s = (fmt == 0) ? scale_f32_from_amax(amax) : e8m0_value(e8m0_from_amax(amax));
     for (int j = 0; j < 128; ++j) q[j] = oracle_e4m3_encode(y[j] / s);
     return s;
 }
 
-/* X bf16 [M, K] (leading dimension ldx) -> codes [M, K] (ldq) and fp32 scales sa[kb*lds + m]. */
+/* X bf16 [M, K] (leading dimension ldx) -> codes [M, K] (ldq) and scales sa[kb*lds + m]
+ * (fmt 0: fp32 amax/448; fmt 1: E8M0 powers of two stored as fp32, reading R12). */
 void oracle_quant_token_1x128(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
-                              uint8_t *q, int64_t ldq, float *sa, int64_t lds) {
+                              uint8_t *q, int64_t ldq, float *sa, int64_t lds, int fmt) {
     int64_t KB = K / 128;
     #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t m = 0; m < M; ++m) {
         float y[128];
         for (int64_t kb = 0; kb < KB; ++kb) {
             for (int j = 0; j < 128; ++j) y[j] = bf16_to_f32(x[m * ldx + kb * 128 + j]);
-            sa[kb * lds + m] = quant_group_1x128(y, q + m * ldq + kb * 128);
+            sa[kb * lds + m] = quant_group_1x128_fmt(y, q + m * ldq + kb * 128, fmt);
         }
     }
 }
@@ -309,12 +316,12 @@ void oracle_rmsnorm_bf16(const uint16_t *x, const uint16_t *gamma, float eps, in
 }
 
 /* Fused front end: RMSNorm (gamma != NULL) then 1x128 token quant; gamma == NULL is the plain
- * token quant of a3.  The normalised row is never stored. */
+ * token quant of a3.  The normalised row is never stored.  fmt as oracle_quant_token_1x128. */
 void oracle_rmsnorm_quant_token(const uint16_t *x, const uint16_t *gamma, float eps, int64_t M,
                                 int64_t K, int64_t ldx, uint8_t *q, int64_t ldq, float *sa,
-                                int64_t lds) {
+                                int64_t lds, int fmt) {
     if (gamma == NULL) {
-        oracle_quant_token_1x128(x, M, K, ldx, q, ldq, sa, lds);
+        oracle_quant_token_1x128(x, M, K, ldx, q, ldq, sa, lds, fmt);
         return;
     }
     int64_t KB = K / 128;
@@ -329,7 +336,7 @@ void oracle_rmsnorm_quant_token(const uint16_t *x, const uint16_t *gamma, float 
                 float u = t * bf16_to_f32(gamma[k]);
                 y[j] = bf16_to_f32(f32_to_bf16_rne(u));
             }
-            sa[kb * lds + m] = quant_group_1x128(y, q + m * ldq + kb * 128);
+            sa[kb * lds + m] = quant_group_1x128_fmt(y, q + m * ldq + kb * 128, fmt);
         }
     }
 }
@@ -386,9 +393,10 @@ float oracle_silu_f32(float g) {
 }
 
 /* h bf16 [R, 2I] (leading dimension ldh): gate = h[:, 0:I], up = h[:, I:2I].  Writes the codes
- * of y = bf16(silu(gate) * up) [R, I] (ldq) and fp32 scales sa[kb * lds + m] (1x128 groups). */
+ * of y = bf16(silu(gate) * up) [R, I] (ldq) and scales sa[kb * lds + m] (1x128 groups; fmt as
+ * oracle_quant_token_1x128). */
 void oracle_silu_mul_quant(const uint16_t *h, int64_t R, int64_t I, int64_t ldh, uint8_t *q,
-                           int64_t ldq, float *sa, int64_t lds) {
+                           int64_t ldq, float *sa, int64_t lds, int fmt) {
     int64_t IB = I / 128;
     #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t m = 0; m < R; ++m) {
@@ -399,7 +407,7 @@ void oracle_silu_mul_quant(const uint16_t *h, int64_t R, int64_t I, int64_t ldh,
                 float g = bf16_to_f32(h[m * ldh + k]), u = bf16_to_f32(h[m * ldh + I + k]);
                 y[j] = bf16_to_f32(f32_to_bf16_rne(oracle_silu_f32(g) * u));
             }
-            sa[kb * lds + m] = quant_group_1x128(y, q + m * ldq + kb * 128);
+            sa[kb * lds + m] = quant_group_1x128_fmt(y, q + m * ldq + kb * 128, fmt);
         }
     }
 }
@@ -487,17 +495,7 @@ void oracle_inverse_rope_quant(const uint16_t *o, const int64_t *pos, const floa
                                  : inverse_rope_element(x, D, R, d - (D - R), cs, sn,
                                                         interleaved);
             }
-            uint8_t *qg = q + t * K + kb * 128;
-            if (fmt == 0) {
-                sa[kb * lds + t] = quant_group_1x128(y, qg);
-            } else {
-                float amax = 0.0f;
-                for (int j = 0; j < 128; ++j)
-                    if (fabsf(y[j]) > amax) amax = fabsf(y[j]);
-                float s = e8m0_value(e8m0_from_amax(amax));
-                for (int j = 0; j < 128; ++j) qg[j] = oracle_e4m3_encode(y[j] / s);
-                sa[kb * lds + t] = s;
-            }
+            sa[kb * lds + t] = quant_group_1x128_fmt(y, q + t * K + kb * 128, fmt);
         }
     }
 }
@@ -583,10 +581,12 @@ void oracle_quant_rowwise(const uint16_t *x, const uint16_t *gamma, float eps, i
 
 /* res[m, k] <- bf16_RNE(fp32(x[m, k]) + fp32(res[m, k])) for every row, then the RMSNorm front
  * end on the updated res: 1x128 groups with K-block-major scales sa[kb * lds + m]
- * (per_token == 0, reading R4) or one scale per row in sa[m] (per_token != 0, reading R7). */
+ * (per_token == 0, reading R4; fmt as oracle_quant_token_1x128) or one fp32 scale per row in
+ * sa[m] (per_token != 0, reading R7; fmt must be 0). */
 void oracle_add_rmsnorm_quant(const uint16_t *x, int64_t ldx, uint16_t *res, int64_t ldr,
                               const uint16_t *gamma, float eps, int64_t M, int64_t K,
-                              int per_token, uint8_t *q, int64_t ldq, float *sa, int64_t lds) {
+                              int per_token, int fmt, uint8_t *q, int64_t ldq, float *sa,
+                              int64_t lds) {
     #pragma omp parallel for schedule(static)
     for (int64_t m = 0; m < M; ++m)
         for (int64_t k = 0; k < K; ++k) {
@@ -596,7 +596,7 @@ void oracle_add_rmsnorm_quant(const uint16_t *x, int64_t ldx, uint16_t *res, int
     if (per_token)
         oracle_quant_rowwise(res, gamma, eps, M, K, ldr, q, ldq, sa);
     else
-        oracle_rmsnorm_quant_token(res, gamma, eps, M, K, ldr, q, ldq, sa, lds);
+        oracle_rmsnorm_quant_token(res, gamma, eps, M, K, ldr, q, ldq, sa, lds, fmt);
 }
 
 /* ------------------------------------------------------------------------------------------ */
