@@ -107,19 +107,27 @@ class WeightBatch:
 
 
 def rmsnorm_quant_token(x: torch.Tensor, gamma=None, eps: float = 1e-6, lds=None, out_q=None,
-                        out_sa=None, stream=None):
+                        out_sa=None, stream=None, scale_fmt="f32"):
     """bf16 X [M, K] -> (codes uint8 [M, K], sa fp32 [K/128, lds]); sa[kb, m] is the scale of
-    row m, K-block kb.  gamma=None: plain 1x128 token quant without RMSNorm."""
+    row m, K-block kb.  gamma=None: plain 1x128 token quant without RMSNorm.  scale_fmt "e8m0":
+    power-of-two scales (stored as fp32) through fp8q_rmsnorm_quant_token_fmt."""
+    f = scale_format(scale_fmt)
     M, K = x.shape
     if lds is None:
         lds = max(4, (M + 3) // 4 * 4)
     q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if out_q is None else out_q
     sa = (torch.empty((K // 128, lds), dtype=torch.float32, device=x.device)
           if out_sa is None else out_sa)
-    st = _lib.lib().fp8q_rmsnorm_quant_token(_ptr(x), _ptr(gamma), float(eps), M, K, _ld(x),
-                                             _ptr(q), _ld(q), _ptr(sa), sa.stride(0),
-                                             _stream(stream))
-    _lib.check(st, "fp8q_rmsnorm_quant_token")
+    if f == FP8Q_SCALE_F32:
+        st = _lib.lib().fp8q_rmsnorm_quant_token(_ptr(x), _ptr(gamma), float(eps), M, K, _ld(x),
+                                                 _ptr(q), _ld(q), _ptr(sa), sa.stride(0),
+                                                 _stream(stream))
+        _lib.check(st, "fp8q_rmsnorm_quant_token")
+    else:
+        st = _lib.lib().fp8q_rmsnorm_quant_token_fmt(_ptr(x), _ptr(gamma), float(eps), M, K,
+                                                     _ld(x), _ptr(q), _ld(q), _ptr(sa),
+                                                     sa.stride(0), f, _stream(stream))
+        _lib.check(st, "fp8q_rmsnorm_quant_token_fmt")
     return q, sa
 
 
@@ -197,9 +205,12 @@ def grouped_gemm_w8a8_block(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor
     return o
 
 
-def silu_mul_quant(h: torch.Tensor, lds=None, out_q=None, out_sa=None, stream=None):
+def silu_mul_quant(h: torch.Tensor, lds=None, out_q=None, out_sa=None, stream=None,
+                   scale_fmt="f32"):
     """h = [gate | up] bf16 [R, 2I] -> (codes uint8 [R, I] of bf16(silu(gate) * up),
-    sa fp32 [I/128, lds]): the front end of an MoE down projection."""
+    sa fp32 [I/128, lds]): the front end of an MoE down projection.  scale_fmt "e8m0":
+    power-of-two scales stored as fp32."""
+    f = scale_format(scale_fmt)
     R, I2 = h.shape
     I = I2 // 2
     if lds is None:
@@ -208,7 +219,7 @@ def silu_mul_quant(h: torch.Tensor, lds=None, out_q=None, out_sa=None, stream=No
     sa = (torch.empty((I // 128, lds), dtype=torch.float32, device=h.device)
           if out_sa is None else out_sa)
     st = _lib.lib().fp8q_silu_mul_quant(_ptr(h), R, I, _ld(h), _ptr(q), _ld(q), _ptr(sa),
-                                        sa.stride(0), _stream(stream))
+                                        sa.stride(0), f, _stream(stream))
     _lib.check(st, "fp8q_silu_mul_quant")
     return q, sa
 
@@ -339,10 +350,12 @@ def quant_rowwise(x: torch.Tensor, gamma=None, eps: float = 1e-6, out_q=None, ou
 
 def add_rmsnorm_quant(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tensor,
                       eps: float = 1e-6, per_token: bool = False, out_q=None, out_sa=None,
-                      lds: int = None, stream=None):
+                      lds: int = None, stream=None, scale_fmt="f32"):
     """Residual add + RMSNorm + quant: residual <- bf16(x + residual) (in place), then the codes
-    of RMSNorm(residual) with 1x128 scales (sa fp32 [K/128, lds], K-block-major) or, per_token,
-    one scale per row (sa fp32 [M]).  Returns (codes, sa)."""
+    of RMSNorm(residual) with 1x128 scales (sa fp32 [K/128, lds], K-block-major; scale_fmt
+    "e8m0": powers of two stored as fp32) or, per_token, one fp32 scale per row (sa [M]).
+    Returns (codes, sa)."""
+    f = scale_format(scale_fmt)
     M, K = x.shape
     q = torch.empty((M, K), dtype=torch.uint8, device=x.device) if out_q is None else out_q
     if per_token:
@@ -356,7 +369,7 @@ def add_rmsnorm_quant(x: torch.Tensor, residual: torch.Tensor, gamma: torch.Tens
         lds = sa.stride(0)
     st = _lib.lib().fp8q_add_rmsnorm_quant(_ptr(x), _ld(x), _ptr(residual), _ld(residual),
                                            _ptr(gamma), float(eps), M, K, 1 if per_token else 0,
-                                           _ptr(q), _ld(q), _ptr(sa), lds, _stream(stream))
+                                           f, _ptr(q), _ld(q), _ptr(sa), lds, _stream(stream))
     _lib.check(st, "fp8q_add_rmsnorm_quant")
     return q, sa
 

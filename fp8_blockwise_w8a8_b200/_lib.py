@@ -31,6 +31,8 @@ SIGNATURES = {
     "fp8q_quant_weight_block": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I, _P]),
     "fp8q_rmsnorm_quant_token": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P,
                                       _I64, _P]),
+    "fp8q_rmsnorm_quant_token_fmt": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P,
+                                          _I64, _I, _P]),
     "fp8q_gemm_w8a8_block": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64, _I64, _P,
                                   _I64, _P]),
     "fp8q_gemm_w8a8_block_splitk": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64, _I64,
@@ -40,7 +42,7 @@ SIGNATURES = {
     "fp8q_gemm_splitk_workspace_bytes": (_I, [_I64, _I64, _I64, _I, ctypes.POINTER(_I64)]),
     "fp8q_grouped_gemm_w8a8_block": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _P, _I64, _I64,
                                           _I64, _I64, _P, _I64, _P]),
-    "fp8q_silu_mul_quant": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _P]),
+    "fp8q_silu_mul_quant": (_I, [_P, _I64, _I64, _I64, _P, _I64, _P, _I64, _I, _P]),
     "fp8q_inverse_rope_quant": (_I, [_P, _I64, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _I, _I,
                                      _P, _I64, _P, _I64, _P]),
     "fp8q_gemm_w8a8_block_diag": (_I, [_P, _I64, _P, _I64, _P, _I64, _P, _I, _I64, _I64, _I64,
@@ -53,8 +55,8 @@ SIGNATURES = {
                                  _P]),
     "fp8q_quant_rowwise": (_I, [_P, _P, ctypes.c_float, _I64, _I64, _I64, _P, _I64, _P, _P]),
     "fp8q_gemm_w8a8_rowwise": (_I, [_P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64, _P, _I64, _P]),
-    "fp8q_add_rmsnorm_quant": (_I, [_P, _I64, _P, _I64, _P, ctypes.c_float, _I64, _I64, _I, _P,
-                                    _I64, _P, _I64, _P]),
+    "fp8q_add_rmsnorm_quant": (_I, [_P, _I64, _P, _I64, _P, ctypes.c_float, _I64, _I64, _I, _I,
+                                    _P, _I64, _P, _I64, _P]),
     "fp8q_selftest_timeout": (_I, [_I64, _P]),
     "fp8q_check_device_error": (_I, [_P]),
     "fp8q_status_string": (ctypes.c_char_p, [_I]),

@@ -86,7 +86,19 @@ int device_state(DeviceState **out) {
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              fp8q::kGemmSmemDense) != cudaSuccess ||
         cudaFuncSetAttribute(fp8q::k_gemm_w8a8_mx, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             fp8q::kGemmSmemDense) != cudaSuccess)
+                             fp8q::kGemmSmemDense) != cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<true, false, false, false,
+                                                         fp8q::kScaleE8M0>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<false, false, false, false,
+                                                         fp8q::kScaleE8M0>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<true, false, true, false,
+                                                         fp8q::kScaleE8M0>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess)
       return FP8Q_ERR_LAUNCH;
     st.attrs_set = true;
   }
@@ -283,7 +295,7 @@ RowLaunch pick_row_launch(Kern kern, int K, bool norm) {
 
 extern "C" {
 
-int fp8q_abi_version(void) { return (1 << 16) | 4; }
+int fp8q_abi_version(void) { return (1 << 16) | 5; }
 
 const char *fp8q_status_string(int status) {
   switch (status) {
@@ -354,7 +366,12 @@ int fp8q_quant_weight_block_batched(const fp8q_weight_desc *descs, int64_t count
   return launch_status();
 }
 
-int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
+}  // extern "C"
+
+namespace {
+
+template <int FMT>
+int rmsnorm_quant_token_impl(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
                              int64_t K, int64_t ldx, void *xq_e4m3, int64_t ldq, float *sa,
                              int64_t lds, cudaStream_t stream) {
   if (M < 0 || K <= 0 || K % 128 || K > kMaxTokenK) return FP8Q_ERR_SHAPE;
@@ -369,8 +386,10 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   if (rc != FP8Q_OK) return rc;
   const bool norm = gamma_bf16 != nullptr;
   const RowLaunch L =
-      norm ? pick_row_launch(fp8q::k_rmsnorm_quant_token<true>, static_cast<int>(K), true)
-           : pick_row_launch(fp8q::k_rmsnorm_quant_token<false>, static_cast<int>(K), false);
+      norm ? pick_row_launch(fp8q::k_rmsnorm_quant_token<true, false, false, false, FMT>,
+                             static_cast<int>(K), true)
+           : pick_row_launch(fp8q::k_rmsnorm_quant_token<false, false, false, false, FMT>,
+                             static_cast<int>(K), false);
   if (L.wpc == 0) return FP8Q_ERR_SHAPE;
   const int wpc = L.wpc, smem = L.smem;
   // the plain kernel spreads (row, step) units over the warps, the fused one whole rows
@@ -385,20 +404,43 @@ int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float e
   const auto *g = static_cast<const uint16_t *>(gamma_bf16);
   auto *q = static_cast<uint8_t *>(xq_e4m3);
   if (norm)
-    fp8q::k_rmsnorm_quant_token<true><<<grid, 32 * wpc, smem, stream>>>(
+    fp8q::k_rmsnorm_quant_token<true, false, false, false, FMT><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
   else if (packed) {
     const int64_t pneed = ((M * (K / 128) + 7) / 8 + wpc - 1) / wpc;
     const int pgrid = static_cast<int>(pneed < cap ? pneed : cap);
-    fp8q::k_rmsnorm_quant_token<false, false, false, true><<<pgrid, 32 * wpc, smem, stream>>>(
+    fp8q::k_rmsnorm_quant_token<false, false, false, true, FMT><<<pgrid, 32 * wpc, smem, stream>>>(
         x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
   } else if (M < static_cast<int64_t>(grid) * wpc)  // fewer rows than warps: spread the steps
-    fp8q::k_rmsnorm_quant_token<false, true><<<grid, 32 * wpc, smem, stream>>>(
+    fp8q::k_rmsnorm_quant_token<false, true, false, false, FMT><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
   else
-    fp8q::k_rmsnorm_quant_token<false><<<grid, 32 * wpc, smem, stream>>>(
+    fp8q::k_rmsnorm_quant_token<false, false, false, false, FMT><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, nullptr, eps, M, static_cast<int>(K), q, ldq, sa, lds, nullptr, 0);
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
+                             int64_t K, int64_t ldx, void *xq_e4m3, int64_t ldq, float *sa,
+                             int64_t lds, cudaStream_t stream) {
+  return rmsnorm_quant_token_impl<fp8q::kScaleF32>(x_bf16, gamma_bf16, eps, M, K, ldx, xq_e4m3,
+                                                   ldq, sa, lds, stream);
+}
+
+int fp8q_rmsnorm_quant_token_fmt(const void *x_bf16, const void *gamma_bf16, float eps,
+                                 int64_t M, int64_t K, int64_t ldx, void *xq_e4m3, int64_t ldq,
+                                 float *sa, int64_t lds, int sa_fmt, cudaStream_t stream) {
+  if (sa_fmt == FP8Q_SCALE_F32)
+    return rmsnorm_quant_token_impl<fp8q::kScaleF32>(x_bf16, gamma_bf16, eps, M, K, ldx,
+                                                     xq_e4m3, ldq, sa, lds, stream);
+  if (sa_fmt == FP8Q_SCALE_E8M0)
+    return rmsnorm_quant_token_impl<fp8q::kScaleE8M0>(x_bf16, gamma_bf16, eps, M, K, ldx,
+                                                      xq_e4m3, ldq, sa, lds, stream);
+  return FP8Q_ERR_ARG;
 }
 
 int fp8q_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, int64_t lds,
@@ -572,10 +614,12 @@ int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, in
 
 int fp8q_add_rmsnorm_quant(const void *x_bf16, int64_t ldx, void *residual_bf16, int64_t ldr,
                            const void *gamma_bf16, float eps, int64_t M, int64_t K, int per_token,
-                           void *q_e4m3, int64_t ldq, float *sa, int64_t lds,
+                           int sa_fmt, void *q_e4m3, int64_t ldq, float *sa, int64_t lds,
                            cudaStream_t stream) {
   if (M < 0 || K <= 0 || K % 128 || K > kMaxTokenK) return FP8Q_ERR_SHAPE;
   if (per_token != 0 && per_token != 1) return FP8Q_ERR_ARG;
+  if (sa_fmt != FP8Q_SCALE_F32 && sa_fmt != FP8Q_SCALE_E8M0) return FP8Q_ERR_ARG;
+  if (per_token && sa_fmt != FP8Q_SCALE_F32) return FP8Q_ERR_ARG;
   if (ldx < K || ldr < K || ldq < K || (!per_token && lds < M)) return FP8Q_ERR_SHAPE;
   if (M == 0) return FP8Q_OK;
   if (!x_bf16 || !residual_bf16 || !gamma_bf16 || !q_e4m3 || !sa) return FP8Q_ERR_NULL;
@@ -608,6 +652,10 @@ int fp8q_add_rmsnorm_quant(const void *x_bf16, int64_t ldx, void *residual_bf16,
   if (per_token)
     fp8q::k_quant_rowwise<true, true><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, res, ldr);
+  else if (sa_fmt == FP8Q_SCALE_E8M0)
+    fp8q::k_rmsnorm_quant_token<true, false, true, false, fp8q::kScaleE8M0>
+        <<<grid, 32 * wpc, smem, stream>>>(x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa,
+                                           lds, res, ldr);
   else
     fp8q::k_rmsnorm_quant_token<true, false, true><<<grid, 32 * wpc, smem, stream>>>(
         x, ldx, g, eps, M, static_cast<int>(K), q, ldq, sa, lds, res, ldr);
@@ -615,8 +663,9 @@ int fp8q_add_rmsnorm_quant(const void *x_bf16, int64_t ldx, void *residual_bf16,
 }
 
 int fp8q_silu_mul_quant(const void *h_bf16, int64_t R, int64_t I, int64_t ldh, void *q_e4m3,
-                        int64_t ldq, float *sa, int64_t lds, cudaStream_t stream) {
+                        int64_t ldq, float *sa, int64_t lds, int sa_fmt, cudaStream_t stream) {
   if (R < 0 || I <= 0 || I % 128 || I > kMaxTokenK) return FP8Q_ERR_SHAPE;
+  if (sa_fmt != FP8Q_SCALE_F32 && sa_fmt != FP8Q_SCALE_E8M0) return FP8Q_ERR_ARG;
   if (ldh < 2 * I || ldq < I || lds < R) return FP8Q_ERR_SHAPE;
   if (R == 0) return FP8Q_OK;
   if (!h_bf16 || !q_e4m3 || !sa) return FP8Q_ERR_NULL;
@@ -642,16 +691,26 @@ int fp8q_silu_mul_quant(const void *h_bf16, int64_t R, int64_t I, int64_t ldh, v
   if ((I / 128) % 4 != 0) {  // packed walk: 4 consecutive blocks of the flattened (row, block) order
     const int64_t need = ((R * (I / 128) + 3) / 4 + best_wpc - 1) / best_wpc;
     const int grid = static_cast<int>(need < cap ? need : cap);
-    fp8q::k_silu_mul_quant<true><<<grid, 32 * best_wpc, smem, stream>>>(
-        static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
-        static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
+    if (sa_fmt == FP8Q_SCALE_E8M0)
+      fp8q::k_silu_mul_quant<true, fp8q::kScaleE8M0><<<grid, 32 * best_wpc, smem, stream>>>(
+          static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
+          static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
+    else
+      fp8q::k_silu_mul_quant<true><<<grid, 32 * best_wpc, smem, stream>>>(
+          static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
+          static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
     return launch_status();
   }
   const int64_t need = (R + best_wpc - 1) / best_wpc;
   const int grid = static_cast<int>(need < cap ? need : cap);
-  fp8q::k_silu_mul_quant<false><<<grid, 32 * best_wpc, smem, stream>>>(
-      static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
-      static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
+  if (sa_fmt == FP8Q_SCALE_E8M0)
+    fp8q::k_silu_mul_quant<false, fp8q::kScaleE8M0><<<grid, 32 * best_wpc, smem, stream>>>(
+        static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
+        static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
+  else
+    fp8q::k_silu_mul_quant<false><<<grid, 32 * best_wpc, smem, stream>>>(
+        static_cast<const uint16_t *>(h_bf16), ldh, R, static_cast<int>(I),
+        static_cast<uint8_t *>(q_e4m3), ldq, sa, lds);
   return launch_status();
 }
 

@@ -349,6 +349,32 @@ __device__ __forceinline__ QParams qparams_tab(float amax, const ScaleTab *t) {
   return p;
 }
 
+// Scale and codes of one 1x128 activation group in either format: fp32 amax/448 with the exact
+// bracket quantizer, or the E8M0 power of two 2^e (the least with 2^e >= fp32(amax/448), clamped
+// to [-127, 127]) stored as its fp32 value, where x * 2^-e is exact and one product per element
+// gives the code.
+template <int FMT>
+struct TokScale {
+  QParams p;       // FMT == kScaleF32
+  float2 inv2;     // FMT == kScaleE8M0: {2^-e, 2^-e}
+  float s;         // the scale written to sa
+  __device__ __forceinline__ TokScale(float amax, const ScaleTab *tab) {
+    if constexpr (FMT == kScaleF32) {
+      p = qparams_tab(amax, tab);
+      s = p.s;
+    } else {
+      const int e = e8m0_exponent(amax);
+      s = pow2_f32(e);
+      const float inv = pow2_f32(-e);
+      inv2 = make_float2(inv, inv);
+    }
+  }
+  __device__ __forceinline__ uint2 codes(const uint4 v) const {
+    if constexpr (FMT == kScaleF32) return quant8_f32(v, p);
+    else return quant8_pow2(v, inv2);
+  }
+};
+
 // ---------------------------------------------------------------------------------------------
 // 1x128 token groups, optionally preceded by RMSNorm.  One warp per row at a time.
 //
@@ -445,7 +471,9 @@ __host__ __device__ constexpr int token_smem_bytes(int K, bool norm, int wpc) {
 //           flight: whole rows per warp; SPREAD (fewer rows than warps) spreads the units over all
 //           warps; PACKED (K/128 not a multiple of the 8 blocks of a step) packs each step with
 //           consecutive blocks of the flattened (row, block) sequence.
-template <bool NORM, bool SPREAD = false, bool ADD = false, bool PACKED = false>
+// FMT selects the group scale: fp32 amax/448 or the E8M0 power of two (TokScale).
+template <bool NORM, bool SPREAD = false, bool ADD = false, bool PACKED = false,
+          int FMT = kScaleF32>
 __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
     const uint16_t *__restrict__ x, int64_t ldx, const uint16_t *__restrict__ gamma, float eps,
     int64_t M, int K, uint8_t *__restrict__ q, int64_t ldq, float *__restrict__ sa, int64_t lds,
@@ -511,11 +539,11 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
       for (int o = LPB / 2; o > 0; o >>= 1)
         mx = absmax_bf16x2(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       if (active) {
-        const QParams p = qparams_tab(absmax_finish(mx), tab);
+        const TokScale<FMT> p(absmax_finish(mx), tab);
         uint8_t *qb = q + m * ldq + b * 128;
 #pragma unroll
         for (int c = 0; c < CPL; ++c)
-          *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = quant8_f32(v0[c], p);
+          *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = p.codes(v0[c]);
         if (sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
       }
 #pragma unroll
@@ -574,11 +602,11 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
 #pragma unroll
       for (int o = LPB / 2; o > 0; o >>= 1)
         mx = absmax_bf16x2(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const QParams p = qparams_tab(absmax_finish(mx), tab);
+      const TokScale<FMT> p(absmax_finish(mx), tab);
       uint8_t *qb = q + m * ldq + b * 128;
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
-        const uint2 codes = quant8_f32(v0[c], p);
+        const uint2 codes = p.codes(v0[c]);
         if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
       }
       if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
@@ -656,11 +684,11 @@ __global__ void __launch_bounds__(512) k_rmsnorm_quant_token(
       for (int c = 0; c < CPL; ++c) m2 = absmax_uint4(m2, v[c]);
 #pragma unroll
       for (int o = LPB / 2; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-      const QParams p = qparams_tab(absmax_finish(m2), tab);
+      const TokScale<FMT> p(absmax_finish(m2), tab);
       uint8_t *qb = q + m * ldq + b * 128;
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
-        const uint2 codes = quant8_f32(v[c], p);
+        const uint2 codes = p.codes(v[c]);
         if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
       }
       if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
@@ -867,7 +895,7 @@ __device__ __forceinline__ uint4 silu_mul8(const uint4 g, const uint4 u) {
 // consecutive blocks of the flattened (row, block) sequence, so a step may finish one row and
 // start the next and no group computes exponentials for nothing; each group advances by a
 // precomputed (rows, blocks) stride with a carry, its next block's loads in flight.
-template <bool PACKED = false>
+template <bool PACKED = false, int FMT = kScaleF32>
 __global__ void __launch_bounds__(512) k_silu_mul_quant(
     const uint16_t *__restrict__ h, int64_t ldh, int64_t R, int I, uint8_t *__restrict__ q,
     int64_t ldq, float *__restrict__ sa, int64_t lds) {
@@ -919,11 +947,11 @@ __global__ void __launch_bounds__(512) k_silu_mul_quant(
 #pragma unroll
       for (int o = LPB / 2; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
       if (active) {
-        const QParams p = qparams_tab(absmax_finish(m2), tab);
+        const TokScale<FMT> p(absmax_finish(m2), tab);
         uint8_t *qb = q + m * ldq + b * 128;
 #pragma unroll
         for (int c = 0; c < CPL; ++c)
-          *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = quant8_f32(v[c], p);
+          *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = p.codes(v[c]);
         if (sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;
       }
       m = m1;
@@ -961,11 +989,11 @@ __global__ void __launch_bounds__(512) k_silu_mul_quant(
       for (int c = 0; c < CPL; ++c) m2 = absmax_uint4(m2, v[c]);
 #pragma unroll
       for (int o = LPB / 2; o > 0; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-      const QParams p = qparams_tab(absmax_finish(m2), tab);
+      const TokScale<FMT> p(absmax_finish(m2), tab);
       uint8_t *qb = q + m * ldq + b * 128;
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
-        const uint2 codes = quant8_f32(v[c], p);
+        const uint2 codes = p.codes(v[c]);
         if (active) *reinterpret_cast<uint2 *>(qb + (sub + LPB * c) * 8) = codes;
       }
       if (active && sub == 0) sa[static_cast<int64_t>(b) * lds + m] = p.s;

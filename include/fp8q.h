@@ -27,7 +27,9 @@
  * Conventions:
  *   - Every pointer argument is a DEVICE pointer on the current CUDA device, except where a
  *     comment says otherwise.  The caller owns all buffers; the library never allocates device
- *     memory and never synchronizes, except fp8q_check_device_error.  Work is enqueued on
+ *     memory at call time (its one buffer of its own is the fixed 24 MiB split-K scratch of
+ *     fp8q_gemm_w8a8_block_splitk_noalloc, a __device__ array reserved on each device when the
+ *     library's module loads there) and never synchronizes, except fp8q_check_device_error.  Work is enqueued on
  *     `stream` (0 = legacy default stream).
  *   - Leading dimensions are in ELEMENTS of the buffer's type.  Matrices are row-major.
  *   - Shapes: K and N must be multiples of 128 ("... vLLM PR 54894 analysis", section 2: the
@@ -124,6 +126,19 @@ int fp8q_quant_weight_block_batched(const fp8q_weight_desc *descs, int64_t count
 int fp8q_rmsnorm_quant_token(const void *x_bf16, const void *gamma_bf16, float eps, int64_t M,
                              int64_t K, int64_t ldx, void *xq_e4m3, int64_t ldq, float *sa,
                              int64_t lds, cudaStream_t stream);
+
+/* fp8q_rmsnorm_quant_token with a choice of activation scale (sa_fmt):
+ *   FP8Q_SCALE_F32   s = fp32(amax / 448) (1 for an all-zero group): the call above;
+ *   FP8Q_SCALE_E8M0  s = 2^e, e the smallest integer with 2^e >= fp32(amax / 448), clamped to
+ *                    [-127, 127] (1 for an all-zero group), written to sa as its fp32 value; the
+ *                    codes are RNEsat(y / 2^e), a division that is exact.  These scales feed
+ *                    fp8q_gemm_w8a8_mx (hardware block scaling) as well as the other GEMMs.
+ * Other arguments, rules and errors as fp8q_rmsnorm_quant_token; another sa_fmt is FP8Q_ERR_ARG.
+ * Source: vLLM PR 54894 analysis, sections 1 and 3 (E8M0 scales with bias 127; the group-128
+ * quant feeds a GEMM that takes MX scales on both operands); SGLang PR 21403 analysis, section 1. */
+int fp8q_rmsnorm_quant_token_fmt(const void *x_bf16, const void *gamma_bf16, float eps,
+                                 int64_t M, int64_t K, int64_t ldx, void *xq_e4m3, int64_t ldq,
+                                 float *sa, int64_t lds, int sa_fmt, cudaStream_t stream);
 
 /* Block-scaled W8A8 GEMM (a5): out[m, n] = bf16( sum_kb sa[m, kb] * sw[n/128, kb] * P_kb[m, n] )
  * where P_kb is the fp32 tensor-core dot product of the E4M3 codes over K-block kb and each
@@ -287,12 +302,13 @@ int fp8q_grouped_gemm_w8a8_block(const void *aq, int64_t lda, const float *sa, i
  *   sa       fp32 scales, sa[kb * lds + r] (1x128 groups of y), written for r < R only
  * silu(g) = g / (1 + e^-g) in fp32 with an IEEE division; e^x in fp32 by Cody-Waite range
  * reduction and a degree-7 Taylor polynomial with every step an IEEE fp32 rounding (reproducible
- * bit for bit; within 2 ulp of the true e^x).  Scales and codes as fp8q_rmsnorm_quant_token.
+ * bit for bit; within 2 ulp of the true e^x).  Scales (per sa_fmt, FP8Q_SCALE_F32 or
+ * FP8Q_SCALE_E8M0) and codes as fp8q_rmsnorm_quant_token_fmt.
  * I % 128 == 0, I <= 16384, ldh >= 2 I.  Bit-exact against the CPU oracle.  Source: FP8-RL
  * abstract, item (i) (W8A8 linear layers of MoE models: the down projection's input is the
  * activated gate/up output, quantized 1x128 like every activation here). */
 int fp8q_silu_mul_quant(const void *h_bf16, int64_t R, int64_t I, int64_t ldh, void *q_e4m3,
-                        int64_t ldq, float *sa, int64_t lds, cudaStream_t stream);
+                        int64_t ldq, float *sa, int64_t lds, int sa_fmt, cudaStream_t stream);
 
 /* Inverse RoPE + 1x128 quant: the front end of the attention output projection (wo_a), whose
  * output feeds the per-head-group GEMM fp8q_gemm_w8a8_block_diag.
@@ -345,6 +361,8 @@ int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, in
  *   per_token     0: 1x128 groups, sa [K/128][lds] K-block-major as fp8q_rmsnorm_quant_token
  *                 (lds >= M, lds % 4 == 0, 16-byte aligned); 1: one scale per row, sa [M]
  *                 (4-byte aligned; lds unused), as fp8q_quant_rowwise
+ *   sa_fmt        FP8Q_SCALE_F32, or FP8Q_SCALE_E8M0 with per_token == 0 (the power-of-two
+ *                 scales of fp8q_rmsnorm_quant_token_fmt); anything else is FP8Q_ERR_ARG
  *   q_e4m3        [M][ldq] uint8 codes of RMSNorm(h), written
  * The norm and quant arithmetic are those of fp8q_rmsnorm_quant_token / fp8q_quant_rowwise, on h.
  * The x and residual row ranges must not overlap (FP8Q_ERR_ARG otherwise); ldx, ldr % 8 == 0,
@@ -355,7 +373,7 @@ int fp8q_quant_rowwise(const void *x_bf16, const void *gamma_bf16, float eps, in
  * residual add is the reading above: what an unfused bf16 add writes). */
 int fp8q_add_rmsnorm_quant(const void *x_bf16, int64_t ldx, void *residual_bf16, int64_t ldr,
                            const void *gamma_bf16, float eps, int64_t M, int64_t K, int per_token,
-                           void *q_e4m3, int64_t ldq, float *sa, int64_t lds,
+                           int sa_fmt, void *q_e4m3, int64_t ldq, float *sa, int64_t lds,
                            cudaStream_t stream);
 
 /* Per-token x per-channel W8A8 GEMM:

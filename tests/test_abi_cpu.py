@@ -54,6 +54,18 @@ def test_weight_quant_host_checks(L):
     assert f(FAKE, 0, 128, 128, FAKE, 128, FAKE, 0, None) == _lib.FP8Q_OK      # empty: no-op
 
 
+def test_token_quant_fmt_host_checks(L):
+    f = L.fp8q_rmsnorm_quant_token_fmt
+    assert f(FAKE, None, 1e-6, 4, 128, 128, FAKE, 128, FAKE, 4, 2, None) == _lib.FP8Q_ERR_ARG
+    assert f(FAKE, None, 1e-6, 4, 100, 100, FAKE, 112, FAKE, 4, 1, None) == _lib.FP8Q_ERR_SHAPE
+    assert f(None, None, 1e-6, 4, 128, 128, FAKE, 128, FAKE, 4, 1, None) == _lib.FP8Q_ERR_NULL
+    assert f(FAKE, None, 1e-6, 4, 128, 128, FAKE, 128, FAKE + 4, 4, 1, None) == _lib.FP8Q_ERR_ALIGN
+    assert f(None, None, 1e-6, 0, 128, 128, None, 128, None, 4, 1, None) == _lib.FP8Q_OK
+    import torch
+    if not torch.cuda.is_available():
+        assert f(FAKE, FAKE, 1e-6, 4, 128, 128, FAKE, 128, FAKE, 4, 1, None) == _lib.FP8Q_ERR_ARCH
+
+
 def test_token_quant_host_checks(L):
     f = L.fp8q_rmsnorm_quant_token
     assert f(FAKE, None, 1e-6, 4, 100, 100, FAKE, 112, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE
@@ -160,18 +172,20 @@ def test_rowwise_host_checks(L):
 def test_add_rmsnorm_quant_host_checks(L):
     f = L.fp8q_add_rmsnorm_quant
     R2 = FAKE + (1 << 24)                 # a residual that does not overlap x
-    ok = dict(x=FAKE, ldx=256, res=R2, ldr=256, g=FAKE, M=8, K=256, pt=0, q=FAKE, ldq=256,
-              sa=FAKE, lds=8)
+    ok = dict(x=FAKE, ldx=256, res=R2, ldr=256, g=FAKE, M=8, K=256, pt=0, fmt=0, q=FAKE,
+              ldq=256, sa=FAKE, lds=8)
 
     def call(**kw):
         b = dict(ok, **kw)
         return f(b["x"], b["ldx"], b["res"], b["ldr"], b["g"], 1e-6, b["M"], b["K"], b["pt"],
-                 b["q"], b["ldq"], b["sa"], b["lds"], None)
+                 b["fmt"], b["q"], b["ldq"], b["sa"], b["lds"], None)
     assert call(K=200, ldx=208, ldr=208, ldq=208) == _lib.FP8Q_ERR_SHAPE   # K % 128
     assert call(K=32768, ldx=32768, ldr=32768, ldq=32768) == _lib.FP8Q_ERR_SHAPE
     assert call(lds=4) == _lib.FP8Q_ERR_SHAPE                              # lds < M
     assert call(ldr=128) == _lib.FP8Q_ERR_SHAPE                            # ldr < K
     assert call(pt=2) == _lib.FP8Q_ERR_ARG
+    assert call(fmt=2) == _lib.FP8Q_ERR_ARG
+    assert call(pt=1, lds=0, fmt=1) == _lib.FP8Q_ERR_ARG                   # per-token: fp32 only
     assert call(g=None) == _lib.FP8Q_ERR_NULL                              # gamma is required
     assert call(res=None) == _lib.FP8Q_ERR_NULL
     assert call(ldr=260) == _lib.FP8Q_ERR_ALIGN
@@ -183,17 +197,19 @@ def test_add_rmsnorm_quant_host_checks(L):
     import torch
     if not torch.cuda.is_available():     # valid arguments reach the device query
         assert call() == _lib.FP8Q_ERR_ARCH
+        assert call(fmt=1) == _lib.FP8Q_ERR_ARCH
         assert call(pt=1, lds=0) == _lib.FP8Q_ERR_ARCH
 
 
 def test_silu_mul_quant_host_checks(L):
     f = L.fp8q_silu_mul_quant
-    assert f(FAKE, 4, 100, 200, FAKE, 112, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE   # I % 128
-    assert f(FAKE, 4, 128, 200, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE   # ldh < 2I
-    assert f(FAKE, 8, 128, 256, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE   # lds < R
-    assert f(FAKE, 4, 128, 260, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_ALIGN   # ldh % 8
-    assert f(None, 4, 128, 256, FAKE, 128, FAKE, 4, None) == _lib.FP8Q_ERR_NULL
-    assert f(None, 0, 128, 256, None, 128, None, 4, None) == _lib.FP8Q_OK
+    assert f(FAKE, 4, 100, 200, FAKE, 112, FAKE, 4, 0, None) == _lib.FP8Q_ERR_SHAPE   # I % 128
+    assert f(FAKE, 4, 128, 200, FAKE, 128, FAKE, 4, 0, None) == _lib.FP8Q_ERR_SHAPE   # ldh < 2I
+    assert f(FAKE, 8, 128, 256, FAKE, 128, FAKE, 4, 0, None) == _lib.FP8Q_ERR_SHAPE   # lds < R
+    assert f(FAKE, 4, 128, 260, FAKE, 128, FAKE, 4, 0, None) == _lib.FP8Q_ERR_ALIGN   # ldh % 8
+    assert f(None, 4, 128, 256, FAKE, 128, FAKE, 4, 0, None) == _lib.FP8Q_ERR_NULL
+    assert f(FAKE, 4, 128, 256, FAKE, 128, FAKE, 4, 3, None) == _lib.FP8Q_ERR_ARG    # format
+    assert f(None, 0, 128, 256, None, 128, None, 4, 1, None) == _lib.FP8Q_OK
 
 
 def test_inverse_rope_quant_host_checks(L):

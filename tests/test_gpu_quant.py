@@ -237,3 +237,24 @@ def test_weight_batch_bad_descriptor_is_reported_and_skipped():
     for i in (0, 2):
         q_ref, s_ref = oracle.quant_weight_block(ws[i].cpu().view(torch.int16).numpy().view(np.uint16), 0)
         assert np.array_equal(qs[i].cpu().numpy(), q_ref) and np.array_equal(ss[i].cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("K", [768, 4096])
+def test_rmsnorm_blocks_with_zeros_and_subnormals(K):
+    """Every 128-block of these rows holds a zero, a subnormal or a value 2^-20 below its
+    neighbours, so the fused kernel's fast (any-order) block sums are not certified and each block
+    is summed again in ascending k; rows of N(0,1) blocks with a few such blocks mixed in take both
+    paths within one row."""
+    rng = np.random.default_rng(96)
+    M = 300
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    KB = K // 128
+    for m in range(M):
+        for b in range(KB):
+            if m < 150 or rng.random() < 0.25:
+                k = b * 128 + int(rng.integers(0, 128))
+                x[m, k] = [0.0, -0.0, 1e-40, -3e-39, 2.0 ** -20][int(rng.integers(0, 5))]
+    x[7, :128] = 0.0                                  # an all-zero block
+    x[8] = 0.0                                        # an all-zero row
+    g = inputs.to_bf16_bits(rng.uniform(0.5, 1.5, K).astype(np.float32))
+    _token_case(inputs.to_bf16_bits(x), g, 1e-6)
