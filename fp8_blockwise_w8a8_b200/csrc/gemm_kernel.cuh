@@ -1100,7 +1100,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// Split-K reduction: out[m, n] = bf16( sum over j = 0 .. S - 1, in that order, of partial_j )."""
+// Split-K reduction: out[m, n] = bf16( sum over j = 0 .. S - 1, in that order, of partial_j ).
 
 // Partials: [tile][split][half h][chunk c][row r] float4 = columns 128 h + 4 c .. + 3 of row r.
 // Grid: 8 CTAs of 256 threads per dense tile; thread (r, g) adds row r, columns 16 g .. 16 g + 15
