@@ -45,7 +45,6 @@ constexpr int kTileBBytes = kBN * kBK;            // 32 KB
 constexpr int kStageBytes = kTileABytes + kTileBBytes;
 constexpr int kStagingBytesPerWarp = 32 * 64;     // 32 rows x 32 bf16 columns
 constexpr int kMaxExperts = 1024;
-constexpr int kGroupM = 16;                       // rasterization: m-blocks per group
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
 constexpr int kOffA = 0;
@@ -110,6 +109,7 @@ struct GemmArgs {
   int64_t ldo;
   int num_n;            // ceil(N / 256)
   int num_m;            // dense: ceil(M / 128)
+  int group_m;          // dense rasterization: m-blocks per group (>= 1)
   int splits;           // K-splits per tile (1: no split)
   float *ws;            // splits > 1: fp32 partials, [tile][split][2][32][128] float4
   int n_tiles_per_group;  // block-diagonal: 256-column tiles per group (0: plain dense); group
@@ -139,13 +139,14 @@ struct Tile {
   int a_kb;      // first K-block of the tile's slice of A (block-diagonal groups; else 0)
 };
 
-// Dense rasterization: groups of kGroupM m-blocks, m fastest inside a group, so that the CTAs
-// running at the same time share A and B tiles in L2.
+// Dense rasterization: groups of group_m m-blocks, m fastest inside a group, so that the CTAs
+// running at the same time share B tiles and the group's A rows stay in L2 while B streams past
+// once per group (the host sizes a group's A slice to a fraction of L2).
 __device__ __forceinline__ Tile dense_tile(const GemmArgs &a, int t) {
-  const int per_group = kGroupM * a.num_n;
+  const int per_group = a.group_m * a.num_n;
   const int g = t / per_group;
-  const int first_m = g * kGroupM;
-  const int gm = min(a.num_m - first_m, kGroupM);
+  const int first_m = g * a.group_m;
+  const int gm = min(a.num_m - first_m, a.group_m);
   const int r = t - g * per_group;
   Tile tl;
   tl.m0 = (first_m + r % gm) * kBM;
@@ -617,6 +618,7 @@ struct RowwiseArgs {
   uint16_t *out;
   int64_t ldo;
   int num_n, num_m;
+  int group_m;          // dense rasterization: m-blocks per group
 };
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -641,6 +643,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   GemmArgs ga{};
   ga.num_m = args.num_m;
   ga.num_n = args.num_n;
+  ga.group_m = args.group_m;
   ga.M = args.M;
 
   if (threadIdx.x == 0) {
@@ -829,6 +832,7 @@ struct MxArgs {
   uint16_t *out;
   int64_t ldo;
   int num_n, num_m;
+  int group_m;          // dense rasterization: m-blocks per group
   int n_tiles_per_group;
 };
 
@@ -889,6 +893,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   GemmArgs ga{};
   ga.num_m = args.num_m;
   ga.num_n = args.num_n;
+  ga.group_m = args.group_m;
   ga.M = args.M;
   ga.K = args.K;
   ga.n_tiles_per_group = args.n_tiles_per_group;
@@ -1107,14 +1112,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // (4 float4 per split, read coalesced across rows) and writes 32 contiguous output bytes.
 constexpr int kReduceThreads = 256;
 __global__ void __launch_bounds__(kReduceThreads)
-    k_splitk_reduce(const float4 *__restrict__ ws, int splits, int num_m, int num_n, int M, int N,
-                    uint16_t *__restrict__ out, int64_t ldo) {
+    k_splitk_reduce(const float4 *__restrict__ ws, int splits, int num_m, int num_n, int group_m,
+                    int M, int N, uint16_t *__restrict__ out, int64_t ldo) {
   const int t = blockIdx.x >> 3;                  // dense tile, same order as dense_tile()
   const int r = threadIdx.x & 127;
   const int g = ((blockIdx.x & 7) << 1) | (threadIdx.x >> 7);  // 16-column group, 0 .. 15
   GemmArgs a{};
   a.num_m = num_m;
   a.num_n = num_n;
+  a.group_m = group_m;
   a.M = M;
   const Tile tl = dense_tile(a, t);
   const int row = tl.m0 + r, col = tl.n0 + 16 * g;
