@@ -1122,6 +1122,13 @@ def run_ncu_case(name):
     elif name == "token_prefill":        # plain 1x128 token quant of X [8192, 4096]
         x = randn((M_, K_), 1.0)
         fn = lambda: fq.rmsnorm_quant_token(x)
+    elif name == "rmsnorm_prefill_e8m0":  # the fused front end with E8M0 activation scales
+        x = randn((M_, K_), 1.0)
+        gam = randn((K_,), 0.5) + 1.0
+        fn = lambda: fq.rmsnorm_quant_token(x, gam, 1e-6, scale_fmt="e8m0")
+    elif name == "token_prefill_e8m0":   # plain 1x128 token quant with E8M0 scales
+        x = randn((M_, K_), 1.0)
+        fn = lambda: fq.rmsnorm_quant_token(x, scale_fmt="e8m0")
     elif name == "requant_prefill":      # W [24576, 4096]: 201 MB in, 101 MB out
         w = randn((N_, K_), 0.02)
         fn = lambda: fq.quant_weight_block(w, "f32")

@@ -102,6 +102,21 @@ def test_gemm_host_checks(L):
               None) == _lib.FP8Q_ERR_NULL
 
 
+def test_size_limits_are_rejected_on_the_host(L):
+    """K beyond 32768 (256 K-blocks of staged scales), more than 1024 experts, K beyond 16384 for
+    the token quant, more than 2048 matrices in a batch."""
+    g = L.fp8q_gemm_w8a8_block
+    K = 32768 + 128
+    assert g(FAKE, K, FAKE, 64, FAKE, K, FAKE, 0, 64, 256, K, FAKE, 256, None) == _lib.FP8Q_ERR_SHAPE
+    gg = L.fp8q_grouped_gemm_w8a8_block
+    assert gg(FAKE, 256, FAKE, 64, FAKE, 256, FAKE, 0, FAKE, 1025, 64, 256, 256, FAKE, 256,
+              None) == _lib.FP8Q_ERR_SHAPE
+    t = L.fp8q_rmsnorm_quant_token
+    assert t(FAKE, None, 1e-6, 4, 16512, 16512, FAKE, 16512, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE
+    b = L.fp8q_quant_weight_block_batched
+    assert b(FAKE, 2049, 2049, 0, None) == _lib.FP8Q_ERR_SHAPE
+
+
 def test_valid_call_without_gpu_reports_arch(L):
     import torch
     if torch.cuda.is_available():
