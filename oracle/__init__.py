@@ -74,6 +74,9 @@ def lib():
         L.oracle_qkv_scales.restype = None
         L.oracle_kv_cache_write.argtypes = [P, I64, I64, I64, I64, I64, P, P, P, I64, P, P]
         L.oracle_kv_cache_write.restype = None
+        L.oracle_attention_decode.argtypes = [P, I64, P, P, P, P, I64, P, I64, I64, I64, I64,
+                                              I64, ctypes.c_float, P, P, P]
+        L.oracle_attention_decode.restype = None
         L.oracle_quant_rowwise.argtypes = [P, P, ctypes.c_float, I64, I64, I64, P, I64, P]
         L.oracle_quant_rowwise.restype = None
         L.oracle_add_rmsnorm_quant.argtypes = [P, I64, P, I64, P, ctypes.c_float, I64, I64,
@@ -369,6 +372,30 @@ def kv_cache_write(qkv_bf16: np.ndarray, Hq: int, Hkv: int, D: int, slots, scale
     lib().oracle_kv_cache_write(_ptr(x), T, x.shape[1], Hq, Hkv, D, _ptr(sl), _ptr(sc), _ptr(q),
                                 Hq * D, _ptr(k_cache), _ptr(v_cache))
     return q
+
+
+def attention_decode(q_codes, k_cache, v_cache, scales3, block_table, seq_lens, Hq: int,
+                     Hkv: int, D: int, block_size: int, sm_scale=None):
+    """Decode attention over the FP8 KV cache, reading R13: q_codes [B, Hq*D] uint8, caches
+    [slots, Hkv*D] uint8, scales3 (s_q, s_k, s_v), block_table [B, max_blocks] int32, seq_lens
+    [B] int32; sm_scale defaults to 1/sqrt(D) (as fp32).  Returns (out [B, Hq*D] fp64, absref
+    [B, Hq*D] = s_v sum_j p_j |dec(v_j)|, zabs [B, Hq] = the largest |scale| sum_d |dec(q)
+    dec(k_j)|)."""
+    q = _c(q_codes, np.uint8)
+    kc, vc = _c(k_cache, np.uint8), _c(v_cache, np.uint8)
+    sc = _c(np.asarray(scales3, np.float32), np.float32)
+    bt = _c(block_table, np.int32)
+    sl = _c(seq_lens, np.int32)
+    B = q.shape[0]
+    if sm_scale is None:
+        sm_scale = float(np.float32(1.0) / np.sqrt(np.float32(D)))
+    out = np.zeros((B, Hq * D), np.float64)
+    absref = np.zeros((B, Hq * D), np.float64)
+    zabs = np.zeros((B, Hq), np.float64)
+    lib().oracle_attention_decode(_ptr(q), q.shape[1], _ptr(kc), _ptr(vc), _ptr(sc), _ptr(bt),
+                                  bt.shape[1], _ptr(sl), B, Hq, Hkv, D, block_size,
+                                  float(sm_scale), _ptr(out), _ptr(absref), _ptr(zabs))
+    return out, absref, zabs
 
 
 def quant_rowwise(x_bf16: np.ndarray, gamma_bf16=None, eps: float = 1e-6):

@@ -79,12 +79,21 @@
  *       MX-scaled GEMM takes E8M0 scales on both operands]: the group's scale is R2's power of
  *       two 2^e (the smallest with 2^e >= fp32(amax / 448), clamped to [-127, 127]), stored as
  *       its fp32 value, as R9 stores it; codes are RNEsat(y / 2^e), a division that is exact.
+ *   R13 decode attention over the FP8 KV cache of R10 [FP8-RL abstract, item (ii): the cache
+ *       exists for the attention that reads it; the page gives no attention arithmetic]: plain
+ *       scaled dot-product attention on the dequantized tensors.  For sequence b (one query
+ *       token) and query head h, with kv head g = h / (Hq / Hkv) (grouped-query attention) and
+ *       the sequence's L positions j at cache slot block_table[b][j / bs] * bs + j % bs:
+ *       z_j = sm_scale * s_q * s_k * sum_d dec(q[h][d]) dec(k_j[g][d]), p = softmax(z),
+ *       o[h][d] = s_v * sum_j p_j dec(v_j[g][d]); the kernel writes bf16_RNE(o).  L = 0 gives
+ *       o = 0.  The reference is fp64 (exp from the C library).
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math -fopenmp.
  * fp32 arithmetic below relies on FLT_EVAL_METHOD == 0 (SSE on x86-64), so every float
  * operation rounds once to nearest-even, as IEEE 754 single precision.
  */
 #include <math.h>
+#include <stdlib.h>
 #include <stdint.h>
 #include <string.h>
 #include <float.h>
@@ -543,6 +552,72 @@ void oracle_kv_cache_write(const uint16_t *qkv, int64_t T, int64_t ld, int64_t H
             v_cache[slots[t] * wkv + c] =
                 oracle_e4m3_encode(bf16_to_f32(row[wq + wkv + c]) / scale3[2]);
         }
+    }
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Decode attention over the FP8 KV cache [FP8-RL (ii)], reading R13                            */
+/* ------------------------------------------------------------------------------------------ */
+
+/* q [B][ldq] codes (Hq heads of D), caches [slots][Hkv * D] codes, scale3 = (s_q, s_k, s_v),
+ * block_table [B][max_blocks] block ids, seq_lens [B].  Writes, per (b, h, d), out = o in fp64,
+ * absref = s_v * sum_j p_j |dec(v_j[g][d])|, and per (b, h) zabs = the largest
+ * |sm_scale * s_q * s_k| * sum_d |dec(q) dec(k_j)| over j (0 when L = 0). */
+void oracle_attention_decode(const uint8_t *q, int64_t ldq, const uint8_t *k_cache,
+                             const uint8_t *v_cache, const float *scale3,
+                             const int32_t *block_table, int64_t max_blocks,
+                             const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv,
+                             int64_t D, int64_t block_size, float sm_scale, double *out,
+                             double *absref, double *zabs) {
+    const int64_t G = Hq / Hkv, row = Hkv * D;
+    const double c = (double)sm_scale * (double)scale3[0] * (double)scale3[1];
+    const double sv = (double)scale3[2];
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * Hq; ++bh) {
+        const int64_t b = bh / Hq, h = bh % Hq, g = h / G;
+        const int64_t L = seq_lens[b];
+        double *o = out + bh * D, *a = absref + bh * D;
+        for (int64_t d = 0; d < D; ++d) o[d] = a[d] = 0.0;
+        zabs[bh] = 0.0;
+        if (L <= 0) continue;
+        double *z = (double *)malloc((size_t)L * sizeof(double));
+        int64_t *slot = (int64_t *)malloc((size_t)L * sizeof(int64_t));
+        double zmax = -INFINITY;
+        for (int64_t j = 0; j < L; ++j) {
+            slot[j] = (int64_t)block_table[b * max_blocks + j / block_size] * block_size +
+                      j % block_size;
+            const uint8_t *kr = k_cache + slot[j] * row + g * D;
+            const uint8_t *qr = q + b * ldq + h * D;
+            double dot = 0.0, dabs = 0.0;
+            for (int64_t d = 0; d < D; ++d) {
+                const double t = oracle_e4m3_decode(qr[d]) * oracle_e4m3_decode(kr[d]);
+                dot += t;
+                dabs += fabs(t);
+            }
+            z[j] = c * dot;
+            if (z[j] > zmax) zmax = z[j];
+            if (fabs(c) * dabs > zabs[bh]) zabs[bh] = fabs(c) * dabs;
+        }
+        double S = 0.0;
+        for (int64_t j = 0; j < L; ++j) {
+            z[j] = exp(z[j] - zmax);
+            S += z[j];
+        }
+        for (int64_t j = 0; j < L; ++j) {
+            const double p = z[j] / S;
+            const uint8_t *vr = v_cache + slot[j] * row + g * D;
+            for (int64_t d = 0; d < D; ++d) {
+                const double v = oracle_e4m3_decode(vr[d]);
+                o[d] += p * v;
+                a[d] += p * fabs(v);
+            }
+        }
+        for (int64_t d = 0; d < D; ++d) {
+            o[d] *= sv;
+            a[d] *= fabs(sv);
+        }
+        free(z);
+        free(slot);
     }
 }
 
