@@ -655,6 +655,40 @@ def measure_rows(fq, device, steps, warmup, pk):
     del kv, qkv, slots, kc, vc, qo
     torch.cuda.empty_cache()
 
+    # decode attention over the FP8 KV cache (the cache's reader): 64 sequences, contexts
+    # U[512, 4096], 32 query / 8 kv heads of 128; the cache is written by the library first
+    da = inputs.decode_attention(device=device)
+    Hq, Hkv, Dh = da["Hq"], da["Hkv"], da["D"]
+    S, Bd = da["num_slots"], da["q"].shape[0]
+    rows_c = torch.cat([torch.zeros((S, Hq * Dh), dtype=torch.bfloat16, device=device),
+                        da["k"], da["v"]], 1)
+    _, s3 = fq.qkv_scales(rows_c, Hq, Hkv, Dh)
+    kc = torch.empty((S, Hkv * Dh), dtype=torch.uint8, device=device)
+    vc = torch.empty_like(kc)
+    fq.kv_cache_write(rows_c, Hq, Hkv, Dh, torch.arange(S, device=device), s3, kc, vc,
+                      quantize_q=False)
+    del rows_c
+    rows_q = torch.cat([da["q"], torch.zeros((Bd, 2 * Hkv * Dh), dtype=torch.bfloat16,
+                                             device=device)], 1)
+    qc = fq.kv_cache_write(rows_q, Hq, Hkv, Dh, -torch.ones(Bd, dtype=torch.int64, device=device),
+                           s3, kc, vc)
+    bt = torch.from_numpy(da["block_table"]).to(device)
+    sl = torch.from_numpy(da["seq_lens"]).to(device)
+    wsa = torch.empty(fq.attention_decode_workspace_bytes(Bd, Hq, Hkv, Dh, da["max_seq_len"]),
+                      dtype=torch.uint8, device=device)
+    oa = torch.empty((Bd, Hq * Dh), dtype=torch.bfloat16, device=device)
+    ms, _ = timed_loop(lambda: fq.attention_decode(qc, kc, vc, s3, bt, sl, Hq, Hkv,
+                                                   da["block_size"], da["max_seq_len"],
+                                                   workspace=wsa, out=oa), steps, warmup, flush)
+    npos = int(da["seq_lens"].sum())
+    byts = npos * Hkv * Dh * 2 + Bd * Hq * Dh * 3     # K and V rows read, q codes, bf16 out
+    rows["attention_decode_fp8kv"] = {
+        "ms": ms, "GB/s": byts / ms / 1e6, "frac": byts / ms / 1e6 / hbm, "launches": 2,
+        "workload": f"{Bd} sequences, {npos} cached positions (contexts U[512, 4096]), 32 query "
+                    "/ 8 kv heads x 128, paged cache of 16-slot blocks"}
+    del da, kc, vc, qc, bt, sl, wsa, oa, rows_q
+    torch.cuda.empty_cache()
+
     # the prefill linear layer with power-of-two (E8M0) scales on both operands: the fused
     # RMSNorm + quant writes E8M0 activation scales, the weight requant E8M0 block scales, and
     # the GEMM applies both in the tensor core (hardware block scaling)
@@ -1175,6 +1209,29 @@ def run_ncu_case(name):
         out = torch.empty((8192, 4096), dtype=torch.bfloat16, device=dev)
         fn = lambda: fq.gemm_w8a8_block_diag(aq, sa, wq.view(4, 1024, 4096),
                                              sw.view(4, 8, 32), out=out)
+    elif name == "attention_decode":     # 64 sequences, 153K cached positions: K+V 314 MB
+        da = inputs.decode_attention(device=dev)
+        Hq, Hkv, Dh = da["Hq"], da["Hkv"], da["D"]
+        S, Bd = da["num_slots"], da["q"].shape[0]
+        rows_c = torch.cat([torch.zeros((S, Hq * Dh), dtype=torch.bfloat16, device=dev),
+                            da["k"], da["v"]], 1)
+        _, s3 = fq.qkv_scales(rows_c, Hq, Hkv, Dh)
+        kc = torch.empty((S, Hkv * Dh), dtype=torch.uint8, device=dev)
+        vc = torch.empty_like(kc)
+        fq.kv_cache_write(rows_c, Hq, Hkv, Dh, torch.arange(S, device=dev), s3, kc, vc,
+                          quantize_q=False)
+        del rows_c
+        rows_q = torch.cat([da["q"], torch.zeros((Bd, 2 * Hkv * Dh), dtype=torch.bfloat16,
+                                                 device=dev)], 1)
+        qc = fq.kv_cache_write(rows_q, Hq, Hkv, Dh,
+                               -torch.ones(Bd, dtype=torch.int64, device=dev), s3, kc, vc)
+        bt = torch.from_numpy(da["block_table"]).to(dev)
+        sl = torch.from_numpy(da["seq_lens"]).to(dev)
+        wsa = torch.empty(fq.attention_decode_workspace_bytes(Bd, Hq, Hkv, Dh, da["max_seq_len"]),
+                          dtype=torch.uint8, device=dev)
+        oa = torch.empty((Bd, Hq * Dh), dtype=torch.bfloat16, device=dev)
+        fn = lambda: fq.attention_decode(qc, kc, vc, s3, bt, sl, Hq, Hkv, da["block_size"],
+                                         da["max_seq_len"], workspace=wsa, out=oa)
     elif name == "gemm_mx_prefill":      # the prefill GEMM with E8M0 scales, hardware block scaling
         x = randn((M_, K_), 1.0)
         aq, sa = fq.inverse_rope_quant(x.view(M_, 1, K_), None, None, None, 0, True, "e8m0")

@@ -26,7 +26,7 @@ __all__ = ["quant_weight_block", "rmsnorm_quant_token", "add_rmsnorm_quant", "ge
            "gemm_w8a8_block_splitk", "gemm_splitk_workspace_bytes", "splitk_workspace",
            "quant_rowwise", "gemm_w8a8_rowwise", "silu_mul_quant", "inverse_rope_quant",
            "gemm_w8a8_block_diag", "gemm_w8a8_mx", "qkv_scales", "kv_cache_write", "WeightBatch",
-           "selftest_timeout",
+           "selftest_timeout", "attention_decode", "attention_decode_workspace_bytes",
            "grouped_gemm_w8a8_block", "check_device_error", "Fp8qError", "FP8Q_SCALE_F32",
            "FP8Q_SCALE_E8M0", "scale_format"]
 
@@ -179,6 +179,38 @@ def gemm_w8a8_block_splitk(aq: torch.Tensor, sa: torch.Tensor, wq: torch.Tensor,
                                                 workspace.numel() * workspace.element_size(),
                                                 _stream(stream))
     _lib.check(st, "fp8q_gemm_w8a8_block_splitk")
+    return o
+
+
+def attention_decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, max_seq_len: int) -> int:
+    b = ctypes.c_int64(0)
+    st = _lib.lib().fp8q_attention_decode_workspace_bytes(B, Hq, Hkv, D, max_seq_len,
+                                                          ctypes.byref(b))
+    _lib.check(st, "fp8q_attention_decode_workspace_bytes")
+    return b.value
+
+
+def attention_decode(q_codes: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                     scale3: torch.Tensor, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                     Hq: int, Hkv: int, block_size: int, max_seq_len: int, sm_scale=None,
+                     workspace=None, out=None, stream=None):
+    """Decode attention over the FP8 KV cache (fp8q_attention_decode): q_codes uint8 [B, Hq*D],
+    caches uint8 [slots, Hkv*D], scale3 fp32 [3] (s_q, s_k, s_v), block_table int32 [B, max
+    blocks], seq_lens int32 [B] -> bf16 [B, Hq*D].  sm_scale defaults to 1/sqrt(D)."""
+    B = q_codes.shape[0]
+    D = k_cache.shape[1] // Hkv
+    if sm_scale is None:
+        sm_scale = 1.0 / float(np.sqrt(D))
+    if workspace is None:
+        n = attention_decode_workspace_bytes(B, Hq, Hkv, D, max_seq_len)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q_codes.device)
+    o = torch.empty((B, Hq * D), dtype=torch.bfloat16, device=q_codes.device) if out is None else out
+    st = _lib.lib().fp8q_attention_decode(
+        _ptr(q_codes), _ld(q_codes), _ptr(k_cache), _ptr(v_cache), k_cache.shape[0],
+        _ptr(scale3), _ptr(block_table), block_table.shape[1], _ptr(seq_lens), B, Hq, Hkv, D,
+        block_size, max_seq_len, float(sm_scale), _ptr(o), _ld(o), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _lib.check(st, "fp8q_attention_decode")
     return o
 
 

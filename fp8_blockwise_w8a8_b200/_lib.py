@@ -60,6 +60,9 @@ SIGNATURES = {
     "fp8q_selftest_timeout": (_I, [_I64, _P]),
     "fp8q_check_device_error": (_I, [_P]),
     "fp8q_status_string": (ctypes.c_char_p, [_I]),
+    "fp8q_attention_decode": (_I, [_P, _I64, _P, _P, _I64, _P, _P, _I64, _P, _I64, _I64, _I64,
+                                   _I64, _I64, _I64, ctypes.c_float, _P, _I64, _P, _I64, _P]),
+    "fp8q_attention_decode_workspace_bytes": (_I, [_I64, _I64, _I64, _I64, _I64, _P]),
     "fp8q_abi_version": (_I, []),
 }
 

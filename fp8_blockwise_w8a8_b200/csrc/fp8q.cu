@@ -12,6 +12,7 @@
 #include "gemm_kernel.cuh"
 #include "ptx.cuh"
 #include "quant_kernels.cuh"
+#include "attn_kernels.cuh"
 
 namespace {
 
@@ -66,6 +67,18 @@ int device_state(DeviceState **out) {
                              fp8q::BlockLayout<true>::smemGrouped) != cudaSuccess ||
         cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_attn_decode_split<1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, fp8q::kAttnSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_attn_decode_split<2>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, fp8q::kAttnSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_attn_decode_split<4>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, fp8q::kAttnSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fp8q::k_attn_decode_split<8>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, fp8q::kAttnSmem) !=
             cudaSuccess ||
         cudaFuncSetAttribute(fp8q::k_rmsnorm_quant_token<false>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) !=
@@ -306,11 +319,39 @@ RowLaunch pick_row_launch(Kern kern, int K, bool norm) {
   return best;
 }
 
+// Decode attention: positions per split, chosen so that B * Hkv * splits is about 2048 CTAs (a
+// multiple of the tile, at least one tile, at most kAttnMaxChunk positions); depends on the sizes
+// only, so the workspace query needs no device.
+int attn_chunk(int64_t B, int64_t Hkv, int64_t max_seq_len) {
+  const int64_t work = (max_seq_len > 0 ? max_seq_len : 1) * (B > 0 ? B : 1) * Hkv;
+  int64_t c = (work + 2047) / 2048;
+  c = (c + fp8q::kAttnTile - 1) / fp8q::kAttnTile * fp8q::kAttnTile;
+  if (c < fp8q::kAttnTile) c = fp8q::kAttnTile;
+  if (c > fp8q::kAttnMaxChunk) c = fp8q::kAttnMaxChunk;
+  return static_cast<int>(c);
+}
+
+int attn_shape_status(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t block_size,
+                      int64_t max_seq_len) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D != fp8q::kAttnD || block_size <= 0 ||
+      max_seq_len < 0 || max_seq_len > (1 << 30) || B > (1 << 30) || Hkv > 1024)
+    return FP8Q_ERR_SHAPE;
+  const int64_t G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return FP8Q_ERR_SHAPE;
+  return FP8Q_OK;
+}
+
+int64_t attn_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t max_seq_len) {
+  const int64_t chunk = attn_chunk(B, Hkv, max_seq_len);
+  const int64_t nsplit = max_seq_len > 0 ? (max_seq_len + chunk - 1) / chunk : 1;
+  return B * Hkv * nsplit * (Hq / Hkv) * (fp8q::kAttnD + 2) * 4;
+}
+
 }  // namespace
 
 extern "C" {
 
-int fp8q_abi_version(void) { return (1 << 16) | 5; }
+int fp8q_abi_version(void) { return (1 << 16) | 6; }
 
 const char *fp8q_status_string(int status) {
   switch (status) {
@@ -829,6 +870,79 @@ int fp8q_kv_cache_write(const void *qkv_bf16, int64_t T, int64_t ld, int64_t Hq,
       static_cast<const uint16_t *>(qkv_bf16), ld, T, static_cast<int>(Hq * D / 8),
       static_cast<int>(Hkv * D / 8), slots, num_slots, scale3, static_cast<uint8_t *>(q_e4m3),
       ldq, static_cast<uint8_t *>(k_cache), static_cast<uint8_t *>(v_cache));
+  return launch_status();
+}
+
+int fp8q_attention_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t D,
+                                          int64_t max_seq_len, int64_t *bytes) {
+  if (!bytes) return FP8Q_ERR_NULL;
+  *bytes = 0;
+  const int rc = attn_shape_status(B, Hq, Hkv, D, 1, max_seq_len);
+  if (rc != FP8Q_OK) return rc;
+  *bytes = attn_workspace_bytes(B, Hq, Hkv, max_seq_len);
+  return FP8Q_OK;
+}
+
+int fp8q_attention_decode(const void *q_e4m3, int64_t ldq, const void *k_cache,
+                          const void *v_cache, int64_t num_slots, const float *scale3,
+                          const int32_t *block_table, int64_t max_blocks,
+                          const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv, int64_t D,
+                          int64_t block_size, int64_t max_seq_len, float sm_scale,
+                          void *out_bf16, int64_t ldo, void *workspace, int64_t workspace_bytes,
+                          cudaStream_t stream) {
+  int rc = attn_shape_status(B, Hq, Hkv, D, block_size, max_seq_len);
+  if (rc != FP8Q_OK) return rc;
+  if (num_slots < 0 || max_blocks < 0 || max_blocks * block_size < max_seq_len ||
+      ldq < Hq * D || ldo < Hq * D)
+    return FP8Q_ERR_SHAPE;
+  if (B == 0) return FP8Q_OK;
+  if (!q_e4m3 || !k_cache || !v_cache || !scale3 || !block_table || !seq_lens || !out_bf16 ||
+      !workspace)
+    return FP8Q_ERR_NULL;
+  if (!aligned16(q_e4m3) || ldq % 16 || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(scale3) & 3u) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(out_bf16) & 1u))
+    return FP8Q_ERR_ALIGN;
+  if (workspace_bytes < attn_workspace_bytes(B, Hq, Hkv, max_seq_len)) return FP8Q_ERR_SHAPE;
+  DeviceState *st = nullptr;
+  if ((rc = device_state(&st)) != FP8Q_OK) return rc;
+  fp8q::AttnArgs a;
+  a.q = static_cast<const uint8_t *>(q_e4m3);
+  a.ldq = ldq;
+  a.k_cache = static_cast<const uint8_t *>(k_cache);
+  a.v_cache = static_cast<const uint8_t *>(v_cache);
+  a.num_slots = num_slots;
+  a.scale3 = scale3;
+  a.block_table = block_table;
+  a.max_blocks = max_blocks;
+  a.seq_lens = seq_lens;
+  a.Hq = static_cast<int>(Hq);
+  a.Hkv = static_cast<int>(Hkv);
+  a.block_size = static_cast<int>(block_size);
+  a.max_seq_len = static_cast<int>(max_seq_len);
+  a.chunk = attn_chunk(B, Hkv, max_seq_len);
+  a.nsplit = max_seq_len > 0 ? static_cast<int>((max_seq_len + a.chunk - 1) / a.chunk) : 1;
+  a.sm_scale = sm_scale;
+  a.ws = static_cast<float *>(workspace);
+  a.out = static_cast<uint16_t *>(out_bf16);
+  a.ldo = ldo;
+  if (B > 65535) return FP8Q_ERR_SHAPE;
+  const dim3 gs(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(Hkv),
+                static_cast<unsigned>(B));
+  const dim3 gc(static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
+  const int64_t G = Hq / Hkv;
+  if (max_seq_len > 0) {
+    if (G == 1) fp8q::k_attn_decode_split<1><<<gs, fp8q::kAttnThreads, fp8q::kAttnSmem, stream>>>(a);
+    else if (G == 2) fp8q::k_attn_decode_split<2><<<gs, fp8q::kAttnThreads, fp8q::kAttnSmem, stream>>>(a);
+    else if (G == 4) fp8q::k_attn_decode_split<4><<<gs, fp8q::kAttnThreads, fp8q::kAttnSmem, stream>>>(a);
+    else fp8q::k_attn_decode_split<8><<<gs, fp8q::kAttnThreads, fp8q::kAttnSmem, stream>>>(a);
+    if ((rc = launch_status()) != FP8Q_OK) return rc;
+  }
+  if (G == 1) fp8q::k_attn_decode_combine<1><<<gc, fp8q::kAttnThreads, 0, stream>>>(a);
+  else if (G == 2) fp8q::k_attn_decode_combine<2><<<gc, fp8q::kAttnThreads, 0, stream>>>(a);
+  else if (G == 4) fp8q::k_attn_decode_combine<4><<<gc, fp8q::kAttnThreads, 0, stream>>>(a);
+  else fp8q::k_attn_decode_combine<8><<<gc, fp8q::kAttnThreads, 0, stream>>>(a);
   return launch_status();
 }
 

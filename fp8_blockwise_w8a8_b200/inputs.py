@@ -28,6 +28,13 @@ bf16 tensors are returned as numpy ``uint16`` bit patterns (host) or torch ``bfl
                    with 4 channels per head x 8, V ~ N(0, 0.5); a paged cache of 1024 blocks x 16
                    slots; each token gets a distinct random slot, 2 % of them -1 (padding, not
                    cached); seed 6
+* decode attention over the FP8 KV cache: a batch of B = 64 sequences (one query token each),
+                   context lengths ~ U[512, 4096]; a paged cache of block_size 16 whose blocks
+                   are dealt to the sequences in a seeded random order (plus 8 spare blocks);
+                   32 query heads, 8 kv heads, head_dim 128; Q ~ N(0,1), K ~ N(0,1) with 4
+                   channels per head x 8, V ~ N(0, 0.5) for every cache slot, drawn with torch's
+                   generator on the chosen device (bf16); seed 7.  A Llama/Qwen-8B-class decode
+                   step; the pages give no shapes.
 """
 import numpy as np
 import torch
@@ -173,3 +180,37 @@ def kv_cache(tokens: int = 8192, q_heads: int = 32, kv_heads: int = 8, head_dim:
     slots[r.random(tokens) < 0.02] = -1
     return {"qkv": qkv, "slots": slots, "num_slots": num_slots, "Hq": q_heads, "Hkv": kv_heads,
             "D": D}
+
+
+def decode_attention(B: int = 64, Hq: int = 32, Hkv: int = 8, D: int = 128,
+                     block_size: int = 16, lmin: int = 512, lmax: int = 4096, seed: int = 7,
+                     device="cpu", lengths=None):
+    """The decode-attention workload: bf16 q [B, Hq*D], k and v [num_slots, Hkv*D] (torch, on
+    ``device``), int32 block_table [B, max_blocks] and seq_lens [B] (numpy).  ``lengths``
+    replaces the drawn context lengths."""
+    r = rng_for(seed, 0)
+    seq_lens = r.integers(lmin, lmax + 1, size=B).astype(np.int32)
+    if lengths is not None:
+        seq_lens = np.asarray(lengths, np.int32)
+        B = seq_lens.size
+    nblk = -(-seq_lens // block_size)
+    max_blocks = int(nblk.max()) if B else 1
+    num_blocks = int(nblk.sum()) + 8
+    order = r.permutation(num_blocks).astype(np.int32)
+    block_table = np.zeros((B, max(max_blocks, 1)), np.int32)
+    at = 0
+    for b in range(B):
+        block_table[b, :nblk[b]] = order[at:at + nblk[b]]
+        at += nblk[b]
+    num_slots = num_blocks * block_size
+    g = torch.Generator(device=device)
+    g.manual_seed(1000 * seed + 1)
+    q = torch.randn((B, Hq * D), generator=g, device=device)
+    k = torch.randn((num_slots, Hkv, D), generator=g, device=device)
+    outl = torch.from_numpy(r.choice(D, size=4, replace=False)).to(device)
+    k[:, :, outl] *= 8.0
+    v = 0.5 * torch.randn((num_slots, Hkv * D), generator=g, device=device)
+    return {"q": q.to(torch.bfloat16), "k": k.reshape(num_slots, Hkv * D).to(torch.bfloat16),
+            "v": v.to(torch.bfloat16), "block_table": block_table, "seq_lens": seq_lens,
+            "num_slots": num_slots, "block_size": block_size, "Hq": Hq, "Hkv": Hkv, "D": D,
+            "max_seq_len": int(seq_lens.max()) if B else 0}

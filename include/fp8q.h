@@ -282,6 +282,48 @@ int fp8q_kv_cache_write(const void *qkv_bf16, int64_t T, int64_t ld, int64_t Hq,
                         void *q_e4m3, int64_t ldq, void *k_cache, void *v_cache,
                         cudaStream_t stream);
 
+/* FP8 KV cache, step 3: decode attention that reads the cache (one query token per sequence).
+ * For sequence b and query head h (kv head g = h / (Hq / Hkv), grouped-query attention), over the
+ * sequence's L = seq_lens[b] positions j, cached at slot block_table[b][j / block_size] *
+ * block_size + j % block_size:
+ *   z_j = sm_scale * s_q * s_k * sum_d dec(q[b][h D + d]) * dec(k_cache[slot_j][g D + d])
+ *   out[b][h D + d] = bf16( s_v * sum_j softmax(z)_j * dec(v_cache[slot_j][g D + d]) )
+ * with (s_q, s_k, s_v) = scale3 (as fp8q_kv_cache_write uses them); L = 0 gives 0.  fp32
+ * arithmetic (expf), results within |out - ref| <= ulp_bf16(|ref|)/2 + absref * (2 (D + 2)
+ * 2^-24 zabs + (L + 16) 2^-23) of the fp64 reference (absref = s_v sum_j p_j |dec(v_j)|, zabs =
+ * the largest |sm_scale s_q s_k| sum_d |dec(q) dec(k_j)|).  Two launches: the positions of each
+ * (sequence, kv head) are split into chunks whose partial softmax states go to `workspace`, then
+ * combined in chunk order.
+ *   q_e4m3       [B][ldq] uint8 codes (Hq heads of D; from fp8q_kv_cache_write), 16-byte aligned,
+ *                ldq % 16 == 0
+ *   k_cache, v_cache
+ *                [num_slots][Hkv * D] uint8, 16-byte aligned (the paged cache of
+ *                fp8q_kv_cache_write)
+ *   scale3       [3] fp32, DEVICE memory
+ *   block_table  [B][max_blocks] int32, DEVICE memory: block ids; an id outside [0, num_slots /
+ *                block_size) records FP8Q_ERR_RANGE and its positions are skipped
+ *   seq_lens     [B] int32, DEVICE memory; a length outside [0, max_seq_len] records
+ *                FP8Q_ERR_RANGE and is clamped
+ *   max_seq_len  a HOST bound on seq_lens (it sizes the split), <= max_blocks * block_size
+ *   out_bf16     [B][ldo] bf16, written (Hq * D values per row)
+ *   workspace    DEVICE memory of fp8q_attention_decode_workspace_bytes(...) bytes, 16-byte
+ *                aligned, caller-owned, reusable in stream order
+ * D == 128 and Hq / Hkv in {1, 2, 4, 8} (else FP8Q_ERR_SHAPE).  Source: FP8-RL abstract, item (ii)
+ * (the FP8 KV cache serves the attention of the rollout's decode steps; the page gives no
+ * attention arithmetic: plain scaled dot-product attention on the dequantized tensors). */
+int fp8q_attention_decode(const void *q_e4m3, int64_t ldq, const void *k_cache,
+                          const void *v_cache, int64_t num_slots, const float *scale3,
+                          const int32_t *block_table, int64_t max_blocks,
+                          const int32_t *seq_lens, int64_t B, int64_t Hq, int64_t Hkv, int64_t D,
+                          int64_t block_size, int64_t max_seq_len, float sm_scale,
+                          void *out_bf16, int64_t ldo, void *workspace, int64_t workspace_bytes,
+                          cudaStream_t stream);
+
+/* Workspace bytes of fp8q_attention_decode for these sizes, written to *bytes (HOST pointer);
+ * depends on the sizes only. */
+int fp8q_attention_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t D,
+                                          int64_t max_seq_len, int64_t *bytes);
+
 /* Grouped W8A8 GEMM for MoE experts (a6): for each expert e the rows
  * [group_offsets[e], group_offsets[e+1]) of aq/sa/out are multiplied by expert e's weight.
  *   wq             [E][N][ldw] uint8 codes (expert stride N * ldw)

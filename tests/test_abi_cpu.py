@@ -66,6 +66,39 @@ def test_token_quant_fmt_host_checks(L):
         assert f(FAKE, FAKE, 1e-6, 4, 128, 128, FAKE, 128, FAKE, 4, 1, None) == _lib.FP8Q_ERR_ARCH
 
 
+def test_attention_decode_host_checks(L):
+    q = L.fp8q_attention_decode_workspace_bytes
+    b = ctypes.c_int64(-1)
+    assert q(2, 8, 2, 128, 300, ctypes.byref(b)) == _lib.FP8Q_OK
+    assert b.value == 2 * 2 * 5 * 4 * 130 * 4     # 5 chunks of 64 positions, 4 heads per group
+    assert q(2, 8, 2, 64, 300, ctypes.byref(b)) == _lib.FP8Q_ERR_SHAPE      # D != 128
+    assert q(2, 12, 8, 128, 300, ctypes.byref(b)) == _lib.FP8Q_ERR_SHAPE    # Hq % Hkv
+    assert q(2, 24, 8, 128, 300, ctypes.byref(b)) == _lib.FP8Q_ERR_SHAPE    # group of 3
+    assert q(2, 8, 2, 128, 300, None) == _lib.FP8Q_ERR_NULL
+    f = L.fp8q_attention_decode
+    ws = 1 << 22
+
+    def call(**kw):
+        a = dict(q=FAKE, ldq=1024, k=FAKE, v=FAKE, slots=64, s3=FAKE, bt=FAKE, maxb=4, sl=FAKE,
+                 B=2, Hq=8, Hkv=2, D=128, bs=16, maxlen=64, sm=0.088, out=FAKE, ldo=1024,
+                 ws=FAKE, wsb=ws)
+        a.update(kw)
+        return f(a["q"], a["ldq"], a["k"], a["v"], a["slots"], a["s3"], a["bt"], a["maxb"],
+                 a["sl"], a["B"], a["Hq"], a["Hkv"], a["D"], a["bs"], a["maxlen"], a["sm"],
+                 a["out"], a["ldo"], a["ws"], a["wsb"], None)
+    assert call(D=64) == _lib.FP8Q_ERR_SHAPE
+    assert call(maxlen=65) == _lib.FP8Q_ERR_SHAPE               # beyond max_blocks * block_size
+    assert call(ldq=512) == _lib.FP8Q_ERR_SHAPE
+    assert call(B=0, q=None, out=None, ws=None) == _lib.FP8Q_OK
+    assert call(q=None) == _lib.FP8Q_ERR_NULL
+    assert call(q=FAKE + 8) == _lib.FP8Q_ERR_ALIGN
+    assert call(ldq=1032) == _lib.FP8Q_ERR_ALIGN
+    assert call(wsb=16) == _lib.FP8Q_ERR_SHAPE                 # workspace too small
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == _lib.FP8Q_ERR_ARCH
+
+
 def test_token_quant_host_checks(L):
     f = L.fp8q_rmsnorm_quant_token
     assert f(FAKE, None, 1e-6, 4, 100, 100, FAKE, 112, FAKE, 4, None) == _lib.FP8Q_ERR_SHAPE
