@@ -9,23 +9,26 @@
 // KV cache written with per-tensor scales by fp8q_kv_cache_write).
 //
 // Two kernels ("split-KV"):
-//   k_attn_decode_split   one CTA per (chunk of C positions, kv head g, sequence b), 128 threads,
+//   k_attn_decode_split   one CTA per (chunk of positions, kv head g, sequence b), 128 threads,
 //                         the G query heads of g together so every K and V row is read once.  The
 //                         cache slots of the chunk's positions are resolved once into shared
 //                         memory; the K and V rows of each tile of 64 positions are copied into
 //                         shared memory by cp.async, two tiles deep (the next tile's copies run
-//                         under this tile's arithmetic).  Per tile:
-//                           scores  8 lanes per position, lane `sub` holding dims 16 sub .. 16 sub
-//                                   + 15 of the G query rows in registers; each lane dequantizes
-//                                   its 16 bytes of the K row (cvt e4m3x2 -> f16x2 -> f32), takes
-//                                   G partial dot products in fp32 and the 8 lanes add them;
-//                           softmax running maximum and sum per head (online softmax): the tile's
-//                                   weights exp(z - m) and the rescale exp(m_old - m_new), expf;
-//                           values  thread t owns dim t of the G heads' fp32 accumulators and adds
-//                                   p_j dec(v_j[g][t]) for the tile's positions.
-//                         The chunk's (m, l, o) per head go to the workspace in fp32.
-//   k_attn_decode_combine one CTA per (kv head, sequence): o = s_v sum_s e^(m_s - M) o_s /
-//                         sum_s e^(m_s - M) l_s over the sequence's chunks (in chunk order), bf16.
+//                         under this tile's arithmetic).  Each warp takes 16 positions of every
+//                         tile with its own online-softmax state:
+//                           scores  mma.sync m16n8k16 (fp16 operands, exact for E4M3 codes,
+//                                   fp32 accumulation): rows = the G query heads (the rest of the
+//                                   16 zero), columns = positions, k = dims in an order that lets
+//                                   each lane read whole 32-bit words of a K row;
+//                           softmax per head in log2 units: the warp's maximum, weights
+//                                   2^(z - m) (exp2f), the rescale of the running state;
+//                           values  a second m16n8k16 whose A fragment is the score accumulators
+//                                   turned into fp16 weights, B = V (two positions' bytes of one
+//                                   dim paired by byte_perm), columns = dims (again permuted).
+//                         The four warps' states are merged in shared memory and the chunk's
+//                         (m, l, o) per head go to the workspace in fp32.
+//   k_attn_decode_combine one CTA per (kv head, sequence): the chunks' states merged in chunk
+//                         order, o = s_v num / den, bf16.
 // A block id outside the cache, or a sequence length outside [0, max_seq_len], records
 // FP8Q_ERR_RANGE (9) in the device error word; such positions are skipped and such lengths are
 // clamped, so no access leaves the buffers.
@@ -94,16 +97,42 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
                : "memory");
 }
 
+// Two E4M3 codes (low byte first) -> f16x2 (low half first), exactly.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t c2) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(c2 & 0xFFFFu)));
+  return h2;
+}
+
+__device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  uint32_t r;
+  memcpy(&r, &h, 4);
+  return r;
+}
+
+// d += A B for one m16n8k16 tile: A row-major fp16 (a0: row g, cols 2t..2t+1; a1: row g + 8;
+// a2: row g, cols 2t + 8..; a3: row g + 8, cols 2t + 8..), B column-major fp16 (b0: rows 2t..2t+1
+// of col g; b1: rows 2t + 8..), fp32 accumulators d (d0, d1: row g, cols 2t, 2t + 1; d2, d3: row
+// g + 8), g = lane / 4, t = lane % 4.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 template <int G>
 __global__ void __launch_bounds__(kAttnThreads) k_attn_decode_split(const AttnArgs a) {
   constexpr int D = kAttnD;
+  static_assert(G >= 1 && G <= 8, "the query heads of a group fill at most 8 of the 16 MMA rows");
   extern __shared__ __align__(128) uint8_t s_kv[];   // [stage][K | V][position][D] codes
   int32_t *s_slot = reinterpret_cast<int32_t *>(s_kv + 2 * kAttnStageBytes);  // or -1
-  __shared__ float s_z[G][kAttnTile];
-  __shared__ __align__(16) float s_p[kAttnTile][G];
-  __shared__ float s_red[4][G];
-  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int s = blockIdx.x, gk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;               // MMA fragment row group and column pair
   const int L = attn_seq_len(a, b);
   const int j_begin = s * a.chunk;
   if (j_begin >= L) return;                      // an empty chunk: the combine does not read it
@@ -111,23 +140,9 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_decode_split(const AttnAr
   const int ntiles = (j_end - j_begin + kAttnTile - 1) / kAttnTile;
   const int64_t row = static_cast<int64_t>(a.Hkv) * D;
   static_assert(kAttnThreads == 2 * kAttnTile, "one thread per K row and one per V row");
-  const float c = a.sm_scale * a.scale3[0] * a.scale3[1];
+  // scores in log2 units: z = c log2(e) q.k, weights 2^(z - m)
+  const float c2 = a.sm_scale * a.scale3[0] * a.scale3[1] * 1.4426950408889634f;
   const int64_t nslot_blocks = a.num_slots / a.block_size;
-
-  // this lane's 16 dims of the G query rows, decoded
-  const int sub = lane % kAttnLPP;
-  float2 qr[G][8];  // dims (2i, 2i + 1) of this lane's 16
-#pragma unroll
-  for (int h = 0; h < G; ++h) {
-    const uint4 qc = *reinterpret_cast<const uint4 *>(a.q + static_cast<int64_t>(b) * a.ldq +
-                                                      (g * G + h) * D + 16 * sub);
-    const uint32_t w[4] = {qc.x, qc.y, qc.z, qc.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      qr[h][2 * i] = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] & 0xFFFFu));
-      qr[h][2 * i + 1] = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] >> 16));
-    }
-  }
 
   // The cache slot of every position of the chunk (-1 where the block id is bad).
   for (int i = tid; i < j_end - j_begin; i += kAttnThreads) {
@@ -143,139 +158,164 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_decode_split(const AttnAr
   __syncthreads();
   // Tile t's K rows (threads 0..63, one position each) and V rows (threads 64..127) into stage
   // t & 1 by 16-byte cp.async, zero-filled for a position that is not read.
-  auto stage_tile = [&](int t) {
+  auto stage_tile = [&](int tt) {
     const int p = tid & (kAttnTile - 1), half = tid / kAttnTile;
-    const int i = t * kAttnTile + p;
+    const int i = tt * kAttnTile + p;
     const int32_t slot = i < j_end - j_begin ? s_slot[i] : -1;
-    const uint32_t dst = smem_u32(s_kv + (t & 1) * kAttnStageBytes + half * kAttnTile * D + p * D);
-    const uint8_t *src = (half ? a.v_cache : a.k_cache) + (slot >= 0 ? slot * row : 0) + g * D;
+    const uint32_t dst = smem_u32(s_kv + (tt & 1) * kAttnStageBytes + half * kAttnTile * D + p * D);
+    const uint8_t *src = (half ? a.v_cache : a.k_cache) + (slot >= 0 ? slot * row : 0) + gk * D;
     const uint32_t nb = slot >= 0 ? 16u : 0u;
 #pragma unroll
     for (int c = 0; c < D / 16; ++c) cp_async16(dst + 16 * c, src + 16 * c, nb);
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
-  float m_run[G], l_run[G], acc[G];
+  // Query fragments (A of the score MMAs): row g = query head g of the group (rows >= G and the
+  // rows g + 8 are zero).  The 128 dims are taken in an order of our choosing (the sum does not
+  // depend on it): in k-step ks, columns 2t, 2t + 1 are dims 16 ks + 4t, + 1 and columns 2t + 8,
+  // 2t + 9 are dims 16 ks + 4t + 2, + 3, so each lane reads 4 consecutive codes per row.
+  uint32_t qa0[8], qa2[8];
 #pragma unroll
-  for (int h = 0; h < G; ++h) {
-    m_run[h] = -INFINITY;
-    l_run[h] = 0.0f;
-    acc[h] = 0.0f;
+  for (int ks = 0; ks < 8; ++ks) {
+    uint32_t w = 0u;
+    if (g < G)
+      w = *reinterpret_cast<const uint32_t *>(a.q + static_cast<int64_t>(b) * a.ldq +
+                                              (gk * G + g) * D + 16 * ks + 4 * t);
+    qa0[ks] = e4m3x2_to_f16x2(w & 0xFFFFu);
+    qa2[ks] = e4m3x2_to_f16x2(w >> 16);
   }
 
+  // Output accumulators (row g = head g): n-tile J = 4 aa + cc, its columns 2t and 2t + 1 are
+  // dims 32 aa + 8t + cc and 32 aa + 8t + 4 + cc (again an order that makes each lane's V reads
+  // whole 32-bit words).
+  float o[16][2];
+#pragma unroll
+  for (int J = 0; J < 16; ++J) o[J][0] = o[J][1] = 0.0f;
+  float m_run = -INFINITY, l_run = 0.0f;               // this lane's part of head g's sum
+  const int p0 = 16 * warp;                            // the warp's positions in each tile
+
   stage_tile(0);
-  for (int t = 0; t < ntiles; ++t) {
-    const int n = min(kAttnTile, j_end - (j_begin + t * kAttnTile));
-    const int32_t *slots_t = s_slot + t * kAttnTile;
-    if (t + 1 < ntiles) {
-      stage_tile(t + 1);                                          // in flight during tile t
+  for (int tt = 0; tt < ntiles; ++tt) {
+    const int n = min(kAttnTile, j_end - (j_begin + tt * kAttnTile));
+    const int32_t *slots_t = s_slot + tt * kAttnTile;
+    if (tt + 1 < ntiles) {
+      stage_tile(tt + 1);                                          // in flight during tile tt
       asm volatile("cp.async.wait_group 1;" ::: "memory");
     } else {
       asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
-    __syncthreads();                                              // tile t's rows are in place
-    const uint8_t *sk = s_kv + (t & 1) * kAttnStageBytes;
+    __syncthreads();                                               // tile tt's rows are in place
+    const uint8_t *sk = s_kv + (tt & 1) * kAttnStageBytes + p0 * D;
     const uint8_t *sv = sk + kAttnTile * D;
-    // scores: round r, warp w, lane group -> tile position r * PPR + w * (32 / LPP) + lane / LPP
-    for (int r = 0; r < kAttnTile / kAttnPPR; ++r) {
-      const int jt = r * kAttnPPR + warp * (32 / kAttnLPP) + lane / kAttnLPP;
-      const bool valid = jt < n && slots_t[jt] >= 0;
-      float2 z2[G];  // even and odd dims summed apart (packed fp32x2 FMAs)
+    // scores S[head][position] for the warp's 16 positions (two n-tiles of 8)
+    float sc[2][4];
 #pragma unroll
-      for (int h = 0; h < G; ++h) z2[h] = make_float2(0.0f, 0.0f);
-      const uint4 kc = *reinterpret_cast<const uint4 *>(sk + jt * D + 16 * sub);
-      const uint32_t w[4] = {kc.x, kc.y, kc.z, kc.w};
+    for (int j = 0; j < 2; ++j) {
+      sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.0f;
+      const uint8_t *krow = sk + (8 * j + g) * D + 4 * t;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 lo = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] & 0xFFFFu));
-        const float2 hi = e4m3x2_to_f32x2(static_cast<uint16_t>(w[i] >> 16));
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          z2[h] = __ffma2_rn(qr[h][2 * i], lo, z2[h]);
-          z2[h] = __ffma2_rn(qr[h][2 * i + 1], hi, z2[h]);
-        }
-      }
-      float z[G];
-#pragma unroll
-      for (int h = 0; h < G; ++h) z[h] = z2[h].x + z2[h].y;
-#pragma unroll
-      for (int o = kAttnLPP / 2; o > 0; o >>= 1)
-#pragma unroll
-        for (int h = 0; h < G; ++h) z[h] += __shfl_xor_sync(0xffffffffu, z[h], o);
-      if (sub == 0)
-#pragma unroll
-        for (int h = 0; h < G; ++h) s_z[h][jt] = valid ? c * z[h] : -INFINITY;
-    }
-    __syncthreads();
-    // online softmax: the tile's maximum per head, its weights, the rescale of the running state
-    float zt[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      zt[h] = tid < kAttnTile ? s_z[h][tid] : -INFINITY;
-      float v = zt[h];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-      if (lane == 0) s_red[warp][h] = v;
-    }
-    __syncthreads();
-    float alpha[G];
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float mt = fmaxf(fmaxf(s_red[0][h], s_red[1][h]), fmaxf(s_red[2][h], s_red[3][h]));
-      const float m_new = fmaxf(m_run[h], mt);
-      // no finite score yet: nothing to weigh or rescale
-      alpha[h] = m_new == -INFINITY ? 1.0f : expf(m_run[h] - m_new);
-      if (tid < kAttnTile) s_p[tid][h] = zt[h] == -INFINITY ? 0.0f : expf(zt[h] - m_new);
-      m_run[h] = m_new;
-    }
-    __syncthreads();  // s_red is reused below; s_p complete
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float v = tid < kAttnTile ? s_p[tid][h] : 0.0f;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) s_red[warp][h] = v;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const float tsum = (s_red[0][h] + s_red[1][h]) + (s_red[2][h] + s_red[3][h]);
-      l_run[h] = fmaf(l_run[h], alpha[h], tsum);
-      acc[h] *= alpha[h];
-    }
-    // values: this thread's dim of the tile's positions, two positions per step (their two
-    // bytes converted together).  Positions past n hold zero rows and zero weights.
-    const int n2 = (n + 1) & ~1;
-#pragma unroll 4
-    for (int jt = 0; jt < n2; jt += 2) {
-      const uint16_t c2 = static_cast<uint16_t>(sv[jt * D + tid]) |
-                          static_cast<uint16_t>(static_cast<uint16_t>(sv[(jt + 1) * D + tid]) << 8);
-      const float2 v = e4m3x2_to_f32x2(c2);
-      if constexpr (G == 1) {
-        acc[0] = fmaf(s_p[jt][0], v.x, acc[0]);
-        acc[0] = fmaf(s_p[jt + 1][0], v.y, acc[0]);
-      } else {
-#pragma unroll
-        for (int h = 0; h < G; h += 2) {
-          float2 a2 = make_float2(acc[h], acc[h + 1]);
-          a2 = __ffma2_rn(make_float2(s_p[jt][h], s_p[jt][h + 1]), make_float2(v.x, v.x), a2);
-          a2 = __ffma2_rn(make_float2(s_p[jt + 1][h], s_p[jt + 1][h + 1]), make_float2(v.y, v.y),
-                          a2);
-          acc[h] = a2.x;
-          acc[h + 1] = a2.y;
-        }
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t w = *reinterpret_cast<const uint32_t *>(krow + 16 * ks);
+        mma_f16_16816(sc[j], qa0[ks], 0u, qa2[ks], 0u, e4m3x2_to_f16x2(w & 0xFFFFu),
+                      e4m3x2_to_f16x2(w >> 16));
       }
     }
-    __syncthreads();  // the stage, s_z, s_p and s_red are rewritten by the next tiles
+    // online softmax for head g over the warp's positions 8j + 2t + e
+    float z[2][2], mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int ip = p0 + 8 * j + 2 * t + e;
+        const bool valid = g < G && ip < n && slots_t[ip] >= 0;
+        z[j][e] = valid ? sc[j][e] * c2 : -INFINITY;
+        mx = fmaxf(mx, z[j][e]);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = m_new == -INFINITY ? 1.0f : exp2f(m_run - m_new);
+    float pw[2][2], psum = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        pw[j][e] = z[j][e] == -INFINITY ? 0.0f : exp2f(z[j][e] - m_new);
+        psum += pw[j][e];
+      }
+    l_run = fmaf(l_run, alpha, psum);
+    m_run = m_new;
+#pragma unroll
+    for (int J = 0; J < 16; ++J) {
+      o[J][0] *= alpha;
+      o[J][1] *= alpha;
+    }
+    // weights as the A fragment of the value MMA (k = the warp's 16 positions): columns 2t, 2t + 1
+    // are positions 2t, 2t + 1 (n-tile 0 of the scores), columns 2t + 8, 2t + 9 are 8 + 2t, 9 + 2t
+    const uint32_t pa0 = f32x2_to_f16x2(pw[0][0], pw[0][1]);
+    const uint32_t pa2 = f32x2_to_f16x2(pw[1][0], pw[1][1]);
+    // values: B[position][dim], four dims of two positions per pair of 32-bit reads
+#pragma unroll
+    for (int aa = 0; aa < 4; ++aa) {
+      const uint8_t *vcol = sv + 32 * aa + 4 * g;
+      const uint32_t w0 = *reinterpret_cast<const uint32_t *>(vcol + (2 * t) * D);
+      const uint32_t w1 = *reinterpret_cast<const uint32_t *>(vcol + (2 * t + 1) * D);
+      const uint32_t w2 = *reinterpret_cast<const uint32_t *>(vcol + (2 * t + 8) * D);
+      const uint32_t w3 = *reinterpret_cast<const uint32_t *>(vcol + (2 * t + 9) * D);
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint32_t sel = static_cast<uint32_t>(cc | ((cc + 4) << 4));
+        float d[4] = {o[4 * aa + cc][0], o[4 * aa + cc][1], 0.0f, 0.0f};
+        mma_f16_16816(d, pa0, 0u, pa2, 0u, e4m3x2_to_f16x2(__byte_perm(w0, w1, sel)),
+                      e4m3x2_to_f16x2(__byte_perm(w2, w3, sel)));
+        o[4 * aa + cc][0] = d[0];
+        o[4 * aa + cc][1] = d[1];
+      }
+    }
+    __syncthreads();  // the stage is rewritten by the copies of tile tt + 2
   }
-  // the chunk's partial state
-  float *part = a.ws + ((static_cast<int64_t>(b) * a.Hkv + g) * a.nsplit + s) * (G * (D + 2));
+
+  // merge the four warps' states (the stage memory is free now) and write the chunk's partial
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  float *s_m = reinterpret_cast<float *>(s_kv);                // [4][8]
+  float *s_l = s_m + 32;                                        // [4][8]
+  float *s_o = s_l + 32;                                        // [4][8][D]
+  if (g < G) {
+    if (t == 0) {
+      s_m[warp * 8 + g] = m_run;
+      s_l[warp * 8 + g] = l_run;
+    }
+#pragma unroll
+    for (int aa = 0; aa < 4; ++aa)
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        s_o[(warp * 8 + g) * D + 32 * aa + 8 * t + cc] = o[4 * aa + cc][0];
+        s_o[(warp * 8 + g) * D + 32 * aa + 8 * t + 4 + cc] = o[4 * aa + cc][1];
+      }
+  }
+  __syncthreads();
+  float *part = a.ws + ((static_cast<int64_t>(b) * a.Hkv + gk) * a.nsplit + s) * (G * (D + 2));
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    part[h * (D + 2) + tid] = acc[h];
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, s_m[w * 8 + h]);
+    float acc = 0.0f, lsum = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float mw = s_m[w * 8 + h];
+        if (mw == -INFINITY) continue;
+        const float f = exp2f(mw - M);
+        acc = fmaf(f, s_o[(w * 8 + h) * D + tid], acc);
+        lsum = fmaf(f, s_l[w * 8 + h], lsum);
+      }
+    }
+    part[h * (D + 2) + tid] = acc;
     if (tid == 0) {
-      part[h * (D + 2) + D] = m_run[h];
-      part[h * (D + 2) + D + 1] = l_run[h];
+      part[h * (D + 2) + D] = M;
+      part[h * (D + 2) + D + 1] = lsum;
     }
   }
 }
@@ -288,21 +328,35 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_decode_combine(const Attn
   const int ns = (L + a.chunk - 1) / a.chunk;
   const float sv = a.scale3[2];
   const float *base = a.ws + (static_cast<int64_t>(b) * a.Hkv + g) * a.nsplit * (G * (D + 2));
+  // one pass over the chunks in order, merging each into a running (M, num, den); m is in log2
+  // units (the split kernel's scores)
+  float M[G], num[G], den[G];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, base[s * (G * (D + 2)) + h * (D + 2) + D]);
-    float num = 0.0f, den = 0.0f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < ns; ++s) {
-        const float *p = base + s * (G * (D + 2)) + h * (D + 2);
-        if (p[D] == -INFINITY) continue;
-        const float w = expf(p[D] - M);
-        num = fmaf(w, p[tid], num);
-        den = fmaf(w, p[D + 1], den);
+    M[h] = -INFINITY;
+    num[h] = den[h] = 0.0f;
+  }
+#pragma unroll 2
+  for (int s = 0; s < ns; ++s) {
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float *p = base + s * (G * (D + 2)) + h * (D + 2);
+      const float ms = p[D], ls = p[D + 1], os = p[tid];
+      if (ms == -INFINITY) continue;
+      if (ms > M[h]) {
+        const float f = exp2f(M[h] - ms);                  // 0 while M is still -inf
+        num[h] *= f;
+        den[h] *= f;
+        M[h] = ms;
       }
+      const float f = exp2f(ms - M[h]);
+      num[h] = fmaf(f, os, num[h]);
+      den[h] = fmaf(f, ls, den[h]);
     }
-    const float o = den > 0.0f ? sv * (num / den) : 0.0f;
+  }
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const float o = den[h] > 0.0f ? sv * (num[h] / den[h]) : 0.0f;
     const __nv_bfloat16 ob = __float2bfloat16_rn(o);
     a.out[static_cast<int64_t>(b) * a.ldo + (g * G + h) * D + tid] =
         *reinterpret_cast<const uint16_t *>(&ob);

@@ -288,12 +288,14 @@ int fp8q_kv_cache_write(const void *qkv_bf16, int64_t T, int64_t ld, int64_t Hq,
  * block_size + j % block_size:
  *   z_j = sm_scale * s_q * s_k * sum_d dec(q[b][h D + d]) * dec(k_cache[slot_j][g D + d])
  *   out[b][h D + d] = bf16( s_v * sum_j softmax(z)_j * dec(v_cache[slot_j][g D + d]) )
- * with (s_q, s_k, s_v) = scale3 (as fp8q_kv_cache_write uses them); L = 0 gives 0.  fp32
- * arithmetic (expf), results within |out - ref| <= ulp_bf16(|ref|)/2 + absref * (2 (D + 2)
- * 2^-24 zabs + (L + 16) 2^-23) of the fp64 reference (absref = s_v sum_j p_j |dec(v_j)|, zabs =
- * the largest |sm_scale s_q s_k| sum_d |dec(q) dec(k_j)|).  Two launches: the positions of each
- * (sequence, kv head) are split into chunks whose partial softmax states go to `workspace`, then
- * combined in chunk order.
+ * with (s_q, s_k, s_v) = scale3 (as fp8q_kv_cache_write uses them); L = 0 gives 0.  The dot
+ * products run on the tensor cores (fp16 operands, exact for E4M3 codes, fp32 accumulation), the
+ * softmax in fp32 (exp2), the weights enter the value sums as fp16; results within
+ * |out - ref| <= ulp_bf16(|ref|)/2 + absref * (2^-11 + 2 (D + 2) 2^-24 zabs + (L + 16) 2^-23)
+ * of the fp64 reference (absref = s_v sum_j p_j |dec(v_j)|, zabs = the largest
+ * |sm_scale s_q s_k| sum_d |dec(q) dec(k_j)|).  Two launches: the positions of each (sequence,
+ * kv head) are split into chunks whose partial softmax states go to `workspace`, then combined
+ * in chunk order.
  *   q_e4m3       [B][ldq] uint8 codes (Hq heads of D; from fp8q_kv_cache_write), 16-byte aligned,
  *                ldq % 16 == 0
  *   k_cache, v_cache

@@ -4,11 +4,12 @@ size the kernel takes (Hq / Hkv = 1, 2, 4, 8), context lengths that fill, cross 
 of the 128-position tile and the split chunk (0, 1, 127, 128, 129, long), block sizes 1, 7 and 16,
 block tables in random order, and bad block ids and lengths (recorded, not read).
 
-The gate follows from the kernel's fp32 arithmetic: a score is a sum of D products then one
-scale multiply, so |dz| <= (D + 2) 2^-24 zabs (zabs = |c| sum_d |dec q dec k|); the weights move by
-at most 2|dz| relatively; the value sums, the softmax sums, the chunk merge and expf add at most
+The gate follows from the kernel's arithmetic: a score is a sum of D exact fp16 products in fp32
+then one scale multiply, so |dz| <= (D + 2) 2^-24 zabs (zabs = |c| sum_d |dec q dec k|); the weights
+move by at most 2|dz| relatively; they enter the value sums as fp16 (the tensor core's operand type:
+at most 2^-11 relative); the value sums, the softmax sums, the chunk merge and exp2 add at most
 (L + 16) 2^-23 of absref (= s_v sum_j p_j |dec v_j|); the bf16 rounding adds half an ulp:
-    |out - ref| <= ulp_bf16(|ref|) / 2 + absref * (2 (D + 2) 2^-24 zabs + (L + 16) 2^-23).
+    |out - ref| <= ulp_bf16(|ref|) / 2 + absref * (2^-11 + 2 (D + 2) 2^-24 zabs + (L + 16) 2^-23).
 
 Source: "FP8-RL ...", abstract, item (ii) (FP8 KV cache; plain scaled dot-product attention).
 """
@@ -62,7 +63,7 @@ def _check(o, qc, kc, vc, s3, bt, sl, Hq, Hkv, D, bs, sm_scale=None, rows=None):
     L = np.clip(sl, 0, None).astype(np.float64)[:, None]
     zb = np.repeat(zabs, D, axis=1)
     bound = (oracle.bf16_ulp(np.abs(ref)) / 2 +
-             absref * (2 * (D + 2) * 2.0 ** -24 * zb + (L + 16) * 2.0 ** -23))
+             absref * (2.0 ** -11 + 2 * (D + 2) * 2.0 ** -24 * zb + (L + 16) * 2.0 ** -23))
     err = np.abs(got[rows] - ref[rows])
     bad = err > bound[rows]
     assert not bad.any(), (f"{bad.sum()} of {bad.size} outside the bound; worst excess "
