@@ -333,8 +333,9 @@ int attn_chunk(int64_t B, int64_t Hkv, int64_t max_seq_len) {
 
 int attn_shape_status(int64_t B, int64_t Hq, int64_t Hkv, int64_t D, int64_t block_size,
                       int64_t max_seq_len) {
+  // B and Hkv are grid dimensions (z, y)
   if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D != fp8q::kAttnD || block_size <= 0 ||
-      max_seq_len < 0 || max_seq_len > (1 << 30) || B > (1 << 30) || Hkv > 1024)
+      max_seq_len < 0 || max_seq_len > (1 << 30) || B > 65535 || Hkv > 1024)
     return FP8Q_ERR_SHAPE;
   const int64_t G = Hq / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return FP8Q_ERR_SHAPE;
@@ -892,8 +893,9 @@ int fp8q_attention_decode(const void *q_e4m3, int64_t ldq, const void *k_cache,
                           cudaStream_t stream) {
   int rc = attn_shape_status(B, Hq, Hkv, D, block_size, max_seq_len);
   if (rc != FP8Q_OK) return rc;
-  if (num_slots < 0 || max_blocks < 0 || max_blocks * block_size < max_seq_len ||
-      ldq < Hq * D || ldo < Hq * D)
+  // slots are int32 in the kernel
+  if (num_slots < 0 || num_slots > INT32_MAX || max_blocks < 0 ||
+      max_blocks * block_size < max_seq_len || ldq < Hq * D || ldo < Hq * D)
     return FP8Q_ERR_SHAPE;
   if (B == 0) return FP8Q_OK;
   if (!q_e4m3 || !k_cache || !v_cache || !scale3 || !block_table || !seq_lens || !out_bf16 ||
@@ -927,7 +929,6 @@ int fp8q_attention_decode(const void *q_e4m3, int64_t ldq, const void *k_cache,
   a.ws = static_cast<float *>(workspace);
   a.out = static_cast<uint16_t *>(out_bf16);
   a.ldo = ldo;
-  if (B > 65535) return FP8Q_ERR_SHAPE;
   const dim3 gs(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(Hkv),
                 static_cast<unsigned>(B));
   const dim3 gc(static_cast<unsigned>(Hkv), static_cast<unsigned>(B));

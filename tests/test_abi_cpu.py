@@ -75,6 +75,7 @@ def test_attention_decode_host_checks(L):
     assert q(2, 12, 8, 128, 300, ctypes.byref(b)) == _lib.FP8Q_ERR_SHAPE    # Hq % Hkv
     assert q(2, 24, 8, 128, 300, ctypes.byref(b)) == _lib.FP8Q_ERR_SHAPE    # group of 3
     assert q(2, 8, 2, 128, 300, None) == _lib.FP8Q_ERR_NULL
+    assert q(65536, 8, 2, 128, 300, ctypes.byref(b)) == _lib.FP8Q_ERR_SHAPE   # grid z
     f = L.fp8q_attention_decode
     ws = 1 << 22
 
@@ -94,6 +95,7 @@ def test_attention_decode_host_checks(L):
     assert call(q=FAKE + 8) == _lib.FP8Q_ERR_ALIGN
     assert call(ldq=1032) == _lib.FP8Q_ERR_ALIGN
     assert call(wsb=16) == _lib.FP8Q_ERR_SHAPE                 # workspace too small
+    assert call(slots=2 ** 31) == _lib.FP8Q_ERR_SHAPE          # slots beyond int32
     import torch
     if not torch.cuda.is_available():
         assert call() == _lib.FP8Q_ERR_ARCH
