@@ -42,11 +42,9 @@
 namespace fp8q {
 
 constexpr int kAttnD = 128;         // head dimension handled
-constexpr int kAttnThreads = 128;   // one thread per output dim in the value pass
-constexpr int kAttnTile = 64;       // positions per tile
+constexpr int kAttnThreads = 128;   // four warps; also one thread per dim in the merge
+constexpr int kAttnTile = 64;       // positions per tile (16 per warp)
 constexpr int kAttnMaxChunk = 4096; // positions per split at most
-constexpr int kAttnLPP = kAttnD / 16;                 // lanes per position in the score pass
-constexpr int kAttnPPR = (kAttnThreads / 32) * (32 / kAttnLPP);  // positions per score round
 
 struct AttnArgs {
   const uint8_t *q;          // [B][ldq] codes
@@ -67,15 +65,6 @@ struct AttnArgs {
   uint16_t *out;             // [B][ldo] bf16
   int64_t ldo;
 };
-
-// Two E4M3 codes (low byte first) -> two fp32 values, exactly (E4M3 is a subset of fp16).
-__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t c2) {
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c2));
-  __half2 hv;
-  memcpy(&hv, &h2, 4);
-  return __half22float2(hv);
-}
 
 __device__ __forceinline__ int attn_seq_len(const AttnArgs &a, int b) {
   int L = a.seq_lens[b];
