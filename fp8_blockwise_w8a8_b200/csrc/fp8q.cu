@@ -290,9 +290,24 @@ int launch_gemm(bool grouped, const void *aq, int64_t lda, const float *sa, int6
                                             stream>>>(tm_a, tm_b, tm_out, a);
   if (splits > 1 && !grouped) {
     if ((rc = launch_status()) != FP8Q_OK) return rc;
-    fp8q::k_splitk_reduce<<<static_cast<unsigned>(tiles * 8), fp8q::kReduceThreads, 0, stream>>>(
-        static_cast<const float4 *>(workspace), splits, a.num_m, a.num_n, a.group_m, a.M, a.N,
-        a.out, ldo);
+    // the reduction as a programmatic dependent launch: it is scheduled while the GEMM drains and
+    // waits in-kernel (griddepcontrol.wait) for the GEMM's partials
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles * 8));
+    cfg.blockDim = dim3(fp8q::kReduceThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fp8q::k_splitk_reduce, static_cast<const float4 *>(workspace),
+                           splits, a.num_m, a.num_n, a.group_m, a.M, a.N, a.out, ldo) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return FP8Q_ERR_LAUNCH;
+    }
   }
   return launch_status();
 }

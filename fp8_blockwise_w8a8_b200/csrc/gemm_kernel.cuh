@@ -1124,6 +1124,9 @@ __global__ void __launch_bounds__(kReduceThreads)
   a.M = M;
   const Tile tl = dense_tile(a, t);
   const int row = tl.m0 + r, col = tl.n0 + 16 * g;
+  // Launched as a programmatic dependent of the GEMM (its launch overlaps the GEMM's tail): wait
+  // until the GEMM grid has completed and its partials are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (row >= M || col >= N) return;
   const int h = g >> 3, c0 = (g & 7) * 4;
   const float4 *p = ws + static_cast<size_t>(t) * splits * (2 * 32 * 128) + (h * 32 + c0) * 128 + r;
